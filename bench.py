@@ -1,0 +1,445 @@
+"""Benchmark of the Gated DeltaNet token mixer on B200 (prints ONE JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+A step is one pass of the hot path over one batch of synthetic input:
+gdn_chunk_fwd over the model-dims prefill workload (B=1, T=4096, 16 QK heads,
+48 V heads, head dim 128, bf16 q/k/v, fp32 gates and state, chunk 64).  The
+headline ``value`` is prefill tokens/s over all ranks with inputs resident in
+HBM; L2 is flushed (256 MiB write) before every timed step and each step is
+timed with CUDA events on the launching stream.  The decode step (B=256
+sequences, one token, state updated in place) is measured in the same run and
+reported under ``decode`` (steps/s).  ``e2e`` repeats the prefill through the
+same C entry point with pinned HOST buffers, the host<->device copies inside
+the timed region.  ``cpu_baseline`` times the fp64 oracle on rank 0 on a
+bounded sample.  ``--impl reference`` times that oracle alone (the CPU
+reference arm).
+
+Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
+sequences (weak scaling); the only collectives are the timing barrier and the
+max-reduction of the elapsed time.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_recurrence_07_b200 import binding, inputs  # noqa: E402
+
+METRIC = "Gated DeltaNet prefill tokens/s, decode steps/s; % of roofline (1 B200)"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- counts
+def prefill_flops_per_token(w, C=64):
+    """Algorithmic FLOPs of the chunkwise form per token: per V head the products
+    U~, W (2C(dk+dv)), U = U~ - W S, Q S, S update (2 dk dv each) and the masked
+    P U (2 C dv); the grams K K^T and Q K^T once per QK head (4 C dk)."""
+    return w.Hv * (6 * w.dk * w.dv + 2 * C * (w.dk + 2 * w.dv)) + 4 * C * w.dk * w.Hqk
+
+
+def prefill_bytes_per_token(w, elt=2):
+    """q, k (per QK head), v, o (per V head) in the input dtype; alpha, beta fp32."""
+    return 2 * w.Hqk * w.dk * elt + 2 * w.Hv * w.dv * elt + 2 * w.Hv * 4
+
+
+def prefill_state_bytes(w):
+    """S0 read (if any) and S_final write, per sequence."""
+    per = w.Hv * w.dk * w.dv * 4
+    return per * (2 if w.s0_std > 0 else 1)
+
+
+def decode_bytes_per_step(w, elt=2):
+    """State read + write (fp32) and the token's q, k, v, o, alpha, beta."""
+    state = 2 * w.B * w.Hv * w.dk * w.dv * 4
+    tok = w.B * (2 * w.Hqk * w.dk * elt + 2 * w.Hv * w.dv * elt + 2 * w.Hv * 4)
+    return state + tok
+
+
+# ----------------------------------------------------------------------------- env
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current source of that kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            entry = json.load(f)[kernel]
+        src = os.path.join(ROOT, entry["source"])
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if sha != entry["source_sha256_16"]:
+            return None
+        return float(entry["bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "utilization.gpu", "power.draw",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self):
+        rows = []
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        loaded = [r for r in rows if r[2] >= 50] or rows
+        reasons = sorted({name for r in loaded for name, val in zip(self.REASONS, r[3])
+                          if val.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_under_load": len([r for r in rows if r[2] >= 50])}
+
+
+# ----------------------------------------------------------------------------- dist
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- timing
+def time_prefill(w, steps, warmup, world, rank):
+    d = inputs.workload_inputs(w, device="cuda")
+    o = torch.empty((w.B, w.T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
+    S_final = torch.empty((w.B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S_final,
+                              stream=stream)
+
+    for _ in range(warmup):
+        flush.fill_(1)
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(world)
+    wall0 = time.perf_counter()
+    for i in range(steps):
+        flush.fill_(i & 0xff)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    times = [a.elapsed_time(b) for a, b in ev]            # ms, per launch
+    total_ms = max_over_ranks(sum(times), world)
+    return {"total_ms": total_ms, "per_launch_ms": sum(times) / steps,
+            "median_ms": statistics.median(times), "wall_s": wall, "launches": steps,
+            "o_checksum": float(o.float().abs().sum().item())}
+
+
+def time_prefill_e2e(w, steps, warmup, world):
+    """Same call with inputs from pinned host memory and results read back."""
+    host = {k: (None if v is None else v.cpu().pin_memory())
+            for k, v in inputs.workload_inputs(w, device="cpu").items()}
+    dev = {k: (None if v is None else torch.empty_like(v, device="cuda")) for k, v in host.items()}
+    o = torch.empty((w.B, w.T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
+    S_final = torch.empty((w.B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    S_h = torch.empty(S_final.shape, dtype=torch.float32).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * 4
+
+    def step():
+        for k_, v in host.items():
+            if v is not None:
+                dev[k_].copy_(v, non_blocking=True)
+        binding.gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], dev["S0"],
+                              o, S_final, stream=stream)
+        o_h.copy_(o, non_blocking=True)
+        S_h.copy_(S_final, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    barrier(world)
+    total_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    return {"total_ms": total_ms, "h2d": h2d, "d2h": d2h}
+
+
+def time_decode(w, steps, warmup, world, pool=16):
+    S = inputs.decode_state(w, device="cuda")
+    xs = [inputs.decode_inputs(w, s, device="cuda") for s in range(pool)]
+    o = torch.empty((w.B, w.Hv, w.dv), dtype=w.dtype, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        x = xs[i % pool]
+        binding.gdn_decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S, o, S,
+                                stream=stream)
+
+    for i in range(warmup):
+        step(i)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(world)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    barrier(world)
+    times = [a.elapsed_time(b) for a, b in ev]
+    total_ms = max_over_ranks(sum(times), world)
+    return {"total_ms": total_ms, "per_launch_ms": sum(times) / steps, "launches": steps}
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_prefill_sample(w, min_seconds=10.0, max_seconds=30.0):
+    """Times the fp64 oracle on the prefill workload (all heads), repeating whole
+    passes over the first `T_s` tokens until about `min_seconds` have elapsed."""
+    import oracle
+    T_s = min(w.T, 4096)
+    d = inputs.workload_inputs(w, device="cpu", T=T_s)
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], nthreads=cores)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or el * (reps + 1) / reps > max_seconds:
+            break
+    tok = reps * w.B * T_s
+    return {"value": tok / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps} x full oracle pass over B={w.B}, T={T_s} (all {w.Hv} V heads), "
+                      f"{el:.1f} s"}
+
+
+def oracle_decode_sample(w, min_seconds=5.0):
+    import oracle
+    B_s = w.B
+    S = inputs.decode_state(w, device="cpu", B=B_s).numpy()
+    cores = oracle.default_threads()
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        x = inputs.decode_inputs(w, n, device="cpu", B=B_s)
+        _, S64 = oracle.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S, nthreads=cores)
+        S = S64.astype("float32")
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": n / el, "unit": "steps/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} decode steps of B={B_s} x {w.Hv} heads, {el:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- main
+def roofline(bound, achieved, peak, unit, traffic):
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "traffic": traffic}
+
+
+def run_reference(args, rank, world):
+    """CPU reference arm: the fp64 oracle on a bounded sample of the same workload."""
+    if rank != 0:
+        return
+    w = inputs.PREFILL_4K
+    per_step_T = 256
+    d = inputs.workload_inputs(w, device="cpu", T=per_step_T)
+    import oracle
+    cores = oracle.default_threads()
+    run = lambda: oracle.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"],  # noqa
+                                 nthreads=cores)
+    for _ in range(args.warmup):
+        run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run()
+    el = time.perf_counter() - t0
+    value = args.steps * w.B * per_step_T / el
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hqk": w.Hqk, "Hv": w.Hv,
+                       "dk": w.dk, "dv": w.dv, "chunk": w.chunk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: oracle pass over B=1, T={per_step_T} "
+                                       f"(all {w.Hv} V heads) of the workload"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+
+    rank, world, local = dist_setup(args.gpus)
+    peaks, peak_src = load_peaks()
+    w = inputs.PREFILL_4K
+    wd = inputs.DECODE_B256
+
+    with ClockSampler(local) as clocks:
+        pre = time_prefill(w, args.steps, args.warmup, world, rank)
+        dec = time_decode(wd, args.decode_steps, args.warmup, world)
+    e2e = time_prefill_e2e(w, args.e2e_steps, 3, world)
+
+    tokens_per_step = w.B * w.T
+    value = world * tokens_per_step * args.steps / (pre["total_ms"] * 1e-3)
+    flops_launch = prefill_flops_per_token(w) * tokens_per_step
+    bytes_launch = prefill_bytes_per_token(w) * tokens_per_step + w.B * prefill_state_bytes(w)
+    t_launch = pre["per_launch_ms"] * 1e-3
+    dec_bytes = decode_bytes_per_step(wd)
+    t_dec = dec["per_launch_ms"] * 1e-3
+    clk = clocks.summary()
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": pre["total_ms"] / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "Hqk": w.Hqk, "Hv": w.Hv,
+                   "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "state": "fp32",
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"dp{world} (independent sequences per GPU)"},
+        "roofline": dict(roofline("tensor", flops_launch / t_launch / 1e12, peaks["bf16_tflops"],
+                                  "TFLOP/s", kernel_traffic("prefill")),
+                         peak_source=f"{peak_src} bf16 burst",
+                         algorithmic_flops_per_launch=flops_launch,
+                         hbm_frac=bytes_launch / t_launch / 1e9 / peaks["hbm_gbs"]),
+        "decode": {
+            "metric": "decode steps/s", "workload": wd.name, "B": wd.B,
+            "value": world * args.decode_steps / (dec["total_ms"] * 1e-3), "unit": "steps/s",
+            "ms_per_step": dec["total_ms"] / args.decode_steps,
+            "roofline": dict(roofline("hbm", dec_bytes / t_dec / 1e9, peaks["hbm_gbs"], "GB/s",
+                                      kernel_traffic("decode")),
+                             peak_source=f"{peak_src} copy bandwidth",
+                             algorithmic_bytes_per_launch=dec_bytes),
+            "gpu_launches": dec["launches"],
+        },
+        "e2e": {"value": world * tokens_per_step * args.e2e_steps / (e2e["total_ms"] * 1e-3),
+                "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
+                "d2h_bytes_per_step": e2e["d2h"]},
+        "gpu_launches": pre["launches"],
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = oracle_prefill_sample(w)
+        line["decode"]["cpu_baseline"] = oracle_decode_sample(wd)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

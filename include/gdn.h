@@ -1,0 +1,119 @@
+/*
+ * gdn.h -- C ABI of libgdn.so, the Gated DeltaNet token mixer on NVIDIA B200 (sm_100a).
+ *
+ * The method: "Qwen3.8-Flash-Next 技术总结 -- Qwen4 架构的探路者", section 2.1
+ * "Gated DeltaNet".  Per sequence and V head the recurrent state S_t is a dk x dv
+ * matrix (row index = key dimension) updated token by token as
+ *
+ *     S_t = alpha_t S_{t-1} + beta_t k_t (v_t - alpha_t S_{t-1}^T k_t)^T
+ *         = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *
+ * (the two equal forms the page gives), with alpha_t the forget gate and beta_t
+ * the write strength.  The page names no read-out; this library returns
+ * o_t = S_t^T q_t, taken with the state after token t's update, unscaled.
+ * The same section gives the model's head layout -- 48 V heads that share 16
+ * QK heads, head dim 128 -- and says the recurrence is evaluated chunk by chunk
+ * with the WY representation; gdn_chunk_fwd is that chunkwise evaluation,
+ * gdn_decode_step the one-token update.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layouts are dense and row-major; "[a, b, c]" lists dimensions outermost first.
+ *   q, k      [B, T, Hqk, dk]   (decode: [B, Hqk, dk])    dtype given by `dtype`
+ *   v, o      [B, T, Hv,  dv]   (decode: [B, Hv,  dv])    dtype given by `dtype`
+ *   alpha     [B, T, Hv]        (decode: [B, Hv])         float; alpha itself, not log alpha
+ *   beta      [B, T, Hv]        (decode: [B, Hv])         float
+ *   S0, S     [B, Hv, dk, dv]                             float (fp32 state)
+ * V head h reads q and k of QK head h / (Hv / Hqk) (contiguous groups of
+ * Hv / Hqk V heads share one QK head).  Gates are per token and V head.
+ * alpha is expected in (0, 1] (1 = no forgetting); the kernels clamp log alpha
+ * below at -87, so alpha = 0 acts as alpha = exp(-87).  beta may be any real.
+ *
+ * Ownership: every pointer is a DEVICE pointer to memory the caller owns; the
+ * library keeps no reference after the call returns and allocates no device
+ * memory.  Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ * default stream).  Input buffers must not be modified until the work on
+ * `stream` completes.
+ *
+ * Errors: argument checks run synchronously on the host before any launch and
+ * return GDN_ERR_INVALID_ARG (bad pointer, size or alignment) or
+ * GDN_ERR_UNSUPPORTED (a shape this build does not implement).  A failed launch
+ * returns GDN_ERR_CUDA (the CUDA error is also returned by gdn_last_cuda_error()).
+ * Kernels never trap.  Every pointer must be 16-byte aligned.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,
+    GDN_ERR_UNSUPPORTED = 2,
+    GDN_ERR_CUDA = 3
+} gdn_status;
+
+typedef enum {
+    GDN_F32 = 0,   /* q, k, v, o are float  (fp32 arithmetic end to end)          */
+    GDN_BF16 = 1   /* q, k, v, o are bfloat16; state, gates and accumulation fp32 */
+} gdn_dtype;
+
+/*
+ * gdn_chunk_fwd -- prefill: runs T tokens of every (sequence, V head) from S0.
+ *
+ * Defines: section 2.1 "Gated DeltaNet" of the page above (the update rule and
+ * the chunkwise WY evaluation it attributes to the Gated DeltaNet paper).
+ *
+ * In:  q, k, v, alpha, beta  as in the layout table, T tokens per sequence.
+ *      S0       initial state [B, Hv, dk, dv]; NULL means all zeros.
+ * Out: o        [B, T, Hv, dv], o_t = S_t^T q_t.
+ *      S_final  state after token T-1, [B, Hv, dk, dv]; NULL skips it.  It may
+ *               be the same buffer as S0 (in-place update); any other overlap
+ *               of outputs with inputs is undefined.
+ * Sizes: B >= 0, T >= 0 (T == 0 copies S0, or zeros, to S_final), Hqk >= 1,
+ *      Hv >= 1 with Hv % Hqk == 0, dk == dv == 128 and chunk == 64
+ *      (else GDN_ERR_UNSUPPORTED).
+ * dtype: GDN_F32 evaluates the chunk form in fp32 on CUDA cores; GDN_BF16 runs
+ *      the contractions on the tensor cores with fp32 accumulation and an fp32
+ *      state.
+ */
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta, const float *S0,
+                         void *o, float *S_final,
+                         int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                         gdn_dtype dtype, void *stream);
+
+/*
+ * gdn_decode_step -- one token for each of B sequences (autoregressive decode).
+ *
+ * Defines: the first form of the update in section 2.1 "Gated DeltaNet",
+ * applied once: p = S^T k, u = beta (v - alpha p), S' = alpha S + k u^T,
+ * o = S'^T q (evaluated as alpha S^T q + (k . q) u, which is equal).
+ *
+ * In:  q, k [B, Hqk, dk]; v [B, Hv, dv]; alpha, beta [B, Hv]; S [B, Hv, dk, dv].
+ * Out: o [B, Hv, dv]; S_new [B, Hv, dk, dv] -- may be the same buffer as S
+ *      (in-place update, the normal use); any other overlap is undefined.
+ * Sizes: B >= 0 (0 is a no-op), Hqk >= 1, Hv % Hqk == 0, dk == dv == 128.
+ */
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *alpha, const float *beta, const float *S,
+                           void *o, float *S_new,
+                           int B, int Hqk, int Hv, int dk, int dv,
+                           gdn_dtype dtype, void *stream);
+
+/* Static, NUL-terminated name of a status code. */
+const char *gdn_status_string(gdn_status status);
+
+/* The cudaError_t value behind the calling thread's last GDN_ERR_CUDA (0 if none). */
+int gdn_last_cuda_error(void);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

@@ -1,0 +1,158 @@
+"""ctypes binding of libgdn.so (see include/gdn.h).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, and their ``data_ptr()`` and the current CUDA stream are handed to
+the C entry points.  All computation happens in the library's CUDA kernels.
+PyTorch is used for device memory and streams.  If the shared library is
+missing, every call raises ``GdnError``: there is no fallback.
+"""
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_PKG, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA = 0, 1, 2, 3
+GDN_F32, GDN_BF16 = 0, 1
+_DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
+
+
+class GdnError(RuntimeError):
+    """A non-OK status from libgdn.so, or the library could not be loaded."""
+
+    def __init__(self, msg, status=None):
+        super().__init__(msg)
+        self.status = status
+
+
+_lib = None
+
+
+def library():
+    """Loads libgdn.so once (no build step at run time; see ``build.py``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIBRARY_PATH):
+            raise GdnError(f"libgdn.so not found at {LIBRARY_PATH}; build it with "
+                           "`python -m linear_attention_recurrence_07_b200.build`")
+        lib = ctypes.CDLL(LIBRARY_PATH)
+        vp, fp, I = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+        lib.gdn_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
+                                      I, I, I, I, I, I, I, I, vp]
+        lib.gdn_chunk_fwd.restype = I
+        lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
+                                        I, I, I, I, I, I, vp]
+        lib.gdn_decode_step.restype = I
+        lib.gdn_status_string.argtypes = [I]
+        lib.gdn_status_string.restype = ctypes.c_char_p
+        lib.gdn_last_cuda_error.argtypes = []
+        lib.gdn_last_cuda_error.restype = I
+        lib.gdn_version.argtypes = []
+        lib.gdn_version.restype = I
+        _lib = lib
+    return _lib
+
+
+def _check(status, what):
+    if status != GDN_OK:
+        lib = library()
+        name = lib.gdn_status_string(status).decode()
+        extra = ""
+        if status == GDN_ERR_CUDA:
+            extra = f" (cudaError {lib.gdn_last_cuda_error()})"
+        raise GdnError(f"{what} failed: {name}{extra}", status)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _expect_cuda(q):
+    if q.dtype not in _DTYPES:
+        raise GdnError(f"unsupported dtype {q.dtype}")
+    if q.device.type != "cuda":
+        raise GdnError(f"tensors must be on a CUDA device, got {q.device}")
+
+
+def _expect(t, name, shape, dtype, device):
+    if t is None:
+        raise GdnError(f"{name} is required")
+    if tuple(t.shape) != tuple(shape):
+        raise GdnError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise GdnError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise GdnError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise GdnError(f"{name} must be contiguous")
+
+
+def gdn_chunk_fwd(q, k, v, alpha, beta, S0, o, S_final, chunk=64, stream=None):
+    """Prefill of T tokens (C entry point ``gdn_chunk_fwd``); writes o and S_final.
+
+    q, k [B, T, Hqk, dk] and v, o [B, T, Hv, dv] (float32 or bfloat16, all the
+    same); alpha, beta [B, T, Hv] float32; S0, S_final [B, Hv, dk, dv] float32
+    or None.  Asynchronous on ``stream`` (default: the current stream)."""
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, T, Hv, dv), q.dtype),
+                               ("o", o, (B, T, Hv, dv), q.dtype),
+                               ("alpha", alpha, (B, T, Hv), torch.float32),
+                               ("beta", beta, (B, T, Hv), torch.float32)):
+        _expect(t, name, shape, dt, dev)
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None:
+            _expect(t, name, (B, Hv, dk, dv), torch.float32, dev)
+    _check(library().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                                   _ptr(o), _ptr(S_final), B, T, Hqk, Hv, dk, dv, chunk,
+                                   _DTYPES[q.dtype], _stream_handle(stream, dev)),
+           "gdn_chunk_fwd")
+
+
+def gdn_decode_step(q, k, v, alpha, beta, S, o, S_new, stream=None):
+    """One decode token (C entry point ``gdn_decode_step``); writes o and S_new
+    (S_new may be S itself).  q, k [B, Hqk, dk]; v, o [B, Hv, dv]; alpha, beta
+    [B, Hv] float32; S, S_new [B, Hv, dk, dv] float32."""
+    B, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, Hv, dv), q.dtype),
+                               ("o", o, (B, Hv, dv), q.dtype),
+                               ("alpha", alpha, (B, Hv), torch.float32),
+                               ("beta", beta, (B, Hv), torch.float32),
+                               ("S", S, (B, Hv, dk, dv), torch.float32),
+                               ("S_new", S_new, (B, Hv, dk, dv), torch.float32)):
+        _expect(t, name, shape, dt, dev)
+    _check(library().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+                                     _ptr(o), _ptr(S_new), B, Hqk, Hv, dk, dv,
+                                     _DTYPES[q.dtype], _stream_handle(stream, dev)),
+           "gdn_decode_step")
+
+
+def chunk_fwd(q, k, v, alpha, beta, S0=None, chunk=64, stream=None):
+    """Allocating convenience wrapper: returns (o, S_final)."""
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    o = torch.empty((B, T, Hv, dv), dtype=q.dtype, device=q.device)
+    S_final = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    gdn_chunk_fwd(q, k, v, alpha, beta, S0, o, S_final, chunk=chunk, stream=stream)
+    return o, S_final
+
+
+def decode_step(q, k, v, alpha, beta, S, stream=None):
+    """In-place decode convenience wrapper: updates S and returns o."""
+    B, Hv, dv = v.shape
+    o = torch.empty((B, Hv, dv), dtype=q.dtype, device=q.device)
+    gdn_decode_step(q, k, v, alpha, beta, S, o, S, stream=stream)
+    return o

@@ -1,0 +1,103 @@
+// C ABI of libgdn.so: argument checks and dispatch.  See include/gdn.h.
+#include <stdint.h>
+
+#include "gdn_internal.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn_status cuda_status(cudaError_t err)
+{
+    if (err == cudaSuccess) return GDN_OK;
+    g_last_cuda_error = (int)err;
+    return GDN_ERR_CUDA;
+}
+
+// Shape checks common to both entry points.
+gdn_status check_heads(int Hqk, int Hv, int dk, int dv)
+{
+    if (Hqk <= 0 || Hv <= 0 || dk <= 0 || dv <= 0) return GDN_ERR_INVALID_ARG;
+    if (Hv % Hqk != 0) return GDN_ERR_UNSUPPORTED;
+    if (dk != gdn::kHeadDim || dv != gdn::kHeadDim) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta, const float *S0,
+                         void *o, float *S_final,
+                         int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                         gdn_dtype dtype, void *stream)
+{
+    if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_heads(Hqk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (B > 65535) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = (size_t)B * Hv * dk * dv * sizeof(float);
+    if (T == 0) {
+        if (!S_final) return GDN_OK;
+        if (!aligned16(S_final) || (S0 && !aligned16(S0))) return GDN_ERR_INVALID_ARG;
+        if (S0 == S_final) return GDN_OK;
+        return cuda_status(S0 ? cudaMemcpyAsync(S_final, S0, state_bytes, cudaMemcpyDeviceToDevice, s)
+                              : cudaMemsetAsync(S_final, 0, state_bytes, s));
+    }
+    if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, beta, S0, o, S_final};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+
+    gdn::ChunkArgs a{q, k, v, alpha, beta, S0, o, S_final, B, T, Hqk, Hv};
+    cudaError_t err;
+    if (dtype == GDN_BF16 && gdn::chunk_tc_available())
+        err = gdn::launch_chunk_tc(a, s);
+    else
+        err = gdn::launch_chunk_simt(a, dtype, s);
+    return cuda_status(err);
+}
+
+gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
+                           const float *alpha, const float *beta, const float *S,
+                           void *o, float *S_new,
+                           int B, int Hqk, int Hv, int dk, int dv,
+                           gdn_dtype dtype, void *stream)
+{
+    if (B < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_heads(Hqk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    if ((long long)B * Hv > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !S || !o || !S_new) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, beta, S, o, S_new};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_INVALID_ARG;
+    gdn::DecodeArgs a{q, k, v, alpha, beta, S, o, S_new, B, Hqk, Hv};
+    return cuda_status(gdn::launch_decode(a, dtype, static_cast<cudaStream_t>(stream)));
+}
+
+const char *gdn_status_string(gdn_status status)
+{
+    switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    }
+    return "GDN_UNKNOWN_STATUS";
+}
+
+int gdn_last_cuda_error(void) { return g_last_cuda_error; }
+
+int gdn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// Internal declarations shared by the kernels and the C-ABI layer of libgdn.so.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+constexpr int kHeadDim = 128;   // dk == dv == 128: the head size of the model (section 2.1)
+constexpr int kChunk = 64;      // tokens per chunk of the chunkwise form
+
+// Kernel arguments of the chunked prefill (plain pointers; shapes validated by the caller).
+struct ChunkArgs {
+    const void *q, *k, *v;
+    const float *alpha, *beta, *S0;
+    void *o;
+    float *S_final;
+    int B, T, Hqk, Hv;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *alpha, *beta, *S;
+    void *o;
+    float *S_new;
+    int B, Hqk, Hv;
+};
+
+// Launchers: enqueue on `stream`, return the launch's cudaError_t.
+cudaError_t launch_decode(const DecodeArgs &a, gdn_dtype dtype, cudaStream_t stream);
+cudaError_t launch_chunk_simt(const ChunkArgs &a, gdn_dtype dtype, cudaStream_t stream);
+cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
+bool chunk_tc_available();
+
+// Element conversions used by the kernels.
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// log(alpha) with the documented clamp, so alpha == 0 stays finite.
+__device__ __forceinline__ float clamped_log(float alpha) {
+    return fmaxf(logf(alpha), -87.0f);
+}
+
+}  // namespace gdn

@@ -1,0 +1,111 @@
+"""Host-side checks of libgdn.so that need no GPU: the library loads, exports every
+entry point include/gdn.h declares, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_recurrence_07_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for header in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not header.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", header)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?\w+\s*\**\s*(gdn_\w+)\s*\(", text, flags=re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(binding.LIBRARY_PATH):
+        from linear_attention_recurrence_07_b200 import build
+        build.build()
+    return binding.library()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("gdn_chunk_fwd", "gdn_decode_step", "gdn_status_string", "gdn_last_cuda_error",
+              "gdn_version"):
+        assert n in names, names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"libgdn.so does not export {name}"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.gdn_status_string(0) == b"GDN_OK"
+    assert lib.gdn_status_string(1) == b"GDN_ERR_INVALID_ARG"
+    assert lib.gdn_status_string(2) == b"GDN_ERR_UNSUPPORTED"
+    assert lib.gdn_status_string(3) == b"GDN_ERR_CUDA"
+    assert lib.gdn_version() >= 100
+    assert lib.gdn_last_cuda_error() == 0
+
+
+FAKE = ctypes.c_void_p(0x1000)        # aligned, never dereferenced: checks reject first
+MISALIGNED = ctypes.c_void_p(0x1004)
+
+
+def chunk(lib, B=1, T=64, Hqk=1, Hv=1, dk=128, dv=128, C=64, dtype=1, ptr=FAKE, o=FAKE):
+    return lib.gdn_chunk_fwd(ptr, FAKE, FAKE, FAKE, FAKE, None, o, None,
+                             B, T, Hqk, Hv, dk, dv, C, dtype, None)
+
+
+def decode(lib, B=1, Hqk=1, Hv=1, dk=128, dv=128, dtype=1, ptr=FAKE):
+    return lib.gdn_decode_step(ptr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               B, Hqk, Hv, dk, dv, dtype, None)
+
+
+def test_chunk_argument_checks(lib):
+    assert chunk(lib, B=-1) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, T=-5) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, Hqk=0) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, Hv=0) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, Hqk=2, Hv=3) == binding.GDN_ERR_UNSUPPORTED
+    assert chunk(lib, dk=64) == binding.GDN_ERR_UNSUPPORTED
+    assert chunk(lib, dv=256) == binding.GDN_ERR_UNSUPPORTED
+    assert chunk(lib, C=32) == binding.GDN_ERR_UNSUPPORTED
+    assert chunk(lib, dtype=7) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, ptr=None) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, o=None) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, ptr=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, o=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert chunk(lib, B=70000) == binding.GDN_ERR_UNSUPPORTED
+    # B == 0 is a no-op that succeeds without touching the device
+    assert chunk(lib, B=0) == binding.GDN_OK
+    # T == 0 with no S_final has nothing to do
+    assert chunk(lib, T=0) == binding.GDN_OK
+
+
+def test_decode_argument_checks(lib):
+    assert decode(lib, B=-1) == binding.GDN_ERR_INVALID_ARG
+    assert decode(lib, Hqk=0) == binding.GDN_ERR_INVALID_ARG
+    assert decode(lib, Hqk=16, Hv=40) == binding.GDN_ERR_UNSUPPORTED
+    assert decode(lib, dk=96) == binding.GDN_ERR_UNSUPPORTED
+    assert decode(lib, dtype=-1) == binding.GDN_ERR_INVALID_ARG
+    assert decode(lib, ptr=None) == binding.GDN_ERR_INVALID_ARG
+    assert decode(lib, ptr=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert decode(lib, B=0) == binding.GDN_OK
+
+
+def test_binding_raises_on_bad_tensors():
+    import torch
+    q = torch.zeros(1, 4, 1, 128)
+    with pytest.raises(binding.GdnError, match="CUDA device"):   # host tensors are refused
+        binding.gdn_chunk_fwd(q, q, q, torch.zeros(1, 4, 1), torch.zeros(1, 4, 1), None, q, None)
+    with pytest.raises(binding.GdnError, match="CUDA device"):
+        binding.gdn_decode_step(q[:, 0], q[:, 0], q[:, 0], torch.zeros(1, 1), torch.zeros(1, 1),
+                                torch.zeros(1, 1, 128, 128), q[:, 0], torch.zeros(1, 1, 128, 128))
+    with pytest.raises(binding.GdnError, match="unsupported dtype"):
+        binding.gdn_chunk_fwd(q.to(torch.float16), q.to(torch.float16), q.to(torch.float16),
+                              torch.zeros(1, 4, 1), torch.zeros(1, 4, 1), None,
+                              q.to(torch.float16), None)

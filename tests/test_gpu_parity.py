@@ -1,0 +1,295 @@
+"""GPU parity of libgdn.so against the fp64 CPU oracle, called through the C ABI.
+
+Bar (stated for the method): max|x_gpu - x_ref| <= tau * max|x_ref| over the whole
+tensor, for o and for the final state, with tau = 1e-4 for fp32 inputs and
+tau = 2e-2 for bf16 inputs with an fp32 state.  Inputs come from the seeded
+generators in ``linear_attention_recurrence_07_b200.inputs``; the oracle sees the
+exact values the GPU sees (bf16 upcast exactly to fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_recurrence_07_b200 import binding, inputs
+
+pytestmark = pytest.mark.gpu
+
+TAU_F32 = 1e-4
+TAU_BF16 = 2e-2
+DEV = "cuda"
+
+
+def tau_for(dtype):
+    return TAU_F32 if dtype == torch.float32 else TAU_BF16
+
+
+def rel_err(got, ref):
+    got = got.detach().double().cpu().numpy() if hasattr(got, "detach") else got
+    scale = float(np.abs(ref).max())
+    return float(np.abs(got - ref).max()) / max(scale, 1e-300)
+
+
+def check(got, ref, tau, what):
+    e = rel_err(got, ref)
+    print(f"{what}: max rel err {e:.3e} (tau {tau})")
+    assert e <= tau, f"{what}: max|err| / max|ref| = {e:.3e} > {tau}"
+
+
+def to_dev(d):
+    return {k: (None if v is None else v.to(DEV)) for k, v in d.items()}
+
+
+def run_chunk(d, chunk=64):
+    o, S = binding.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], chunk=chunk)
+    torch.cuda.synchronize()
+    return o, S
+
+
+def oracle_ref(d, h_range=None):
+    return oracle.forward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], h_range=h_range)
+
+
+# ----------------------------------------------------------------------------- prefill
+def test_prefill_small_fp32_workload():
+    """B=1, T=256, Hqk=2, Hv=6, fp32 end to end, tau = 1e-4."""
+    w = inputs.PREFILL_SMALL_FP32
+    d = inputs.workload_inputs(w)
+    o, S = run_chunk(to_dev(d))
+    o_ref, S_ref = oracle_ref(d)
+    check(o, o_ref, TAU_F32, "o")
+    check(S, S_ref, TAU_F32, "S_final")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 100, 191, 256])
+def test_prefill_ragged_lengths(T, dtype):
+    d = inputs.prefill_inputs(2, T, 2, 6, dtype=dtype, s0_std=0.5, seed=100 + T)
+    o, S = run_chunk(to_dev(d))
+    o_ref, S_ref = oracle_ref(d)
+    check(o, o_ref, tau_for(dtype), f"o T={T}")
+    check(S, S_ref, tau_for(dtype), f"S_final T={T}")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_prefill_one_v_head_per_qk_head(dtype):
+    d = inputs.prefill_inputs(3, 130, 3, 3, dtype=dtype, s0_std=0.1, seed=7)
+    o, S = run_chunk(to_dev(d))
+    o_ref, S_ref = oracle_ref(d)
+    check(o, o_ref, tau_for(dtype), "o")
+    check(S, S_ref, tau_for(dtype), "S_final")
+
+
+def test_prefill_strong_and_no_decay():
+    """Gates at the ends of their range: alpha = 1 (no forgetting) on some heads,
+    alpha ~ 1e-30 (near-total forgetting) on others; beta outside (0, 1) too."""
+    d = inputs.prefill_inputs(1, 200, 2, 4, dtype=torch.float32, s0_std=1.0, seed=9)
+    d["alpha"][:, :, 0] = 1.0
+    d["alpha"][:, 50:60, 1] = 1e-30
+    d["beta"][:, :, 2] = 1.5
+    d["beta"][:, :, 3] = 0.0
+    o, S = run_chunk(to_dev(d))
+    o_ref, S_ref = oracle_ref(d)
+    check(o, o_ref, TAU_F32, "o")
+    check(S, S_ref, TAU_F32, "S_final")
+
+
+def test_prefill_model_dims_workload():
+    """B=1, T=4096, Hqk=16, Hv=48, bf16 inputs, fp32 state: every output checked."""
+    w = inputs.PREFILL_4K
+    d = inputs.workload_inputs(w, device=DEV)
+    o, S = run_chunk(d)
+    o_ref, S_ref = oracle_ref(d)
+    check(o, o_ref, TAU_BF16, "o")
+    check(S, S_ref, TAU_BF16, "S_final")
+
+
+def _sub_problem(d, b, h0, h1, Hv, Hqk):
+    """Inputs of sequence b and V heads [h0, h1) (inside one QK group) as a
+    standalone problem with one QK head."""
+    g = Hv // Hqk
+    hq = h0 // g
+    assert (h1 - 1) // g == hq
+    sl = lambda x: x[b:b + 1]  # noqa: E731
+    return dict(q=sl(d["q"])[:, :, hq:hq + 1], k=sl(d["k"])[:, :, hq:hq + 1],
+                v=sl(d["v"])[:, :, h0:h1], alpha=sl(d["alpha"])[:, :, h0:h1],
+                beta=sl(d["beta"])[:, :, h0:h1],
+                S0=None if d["S0"] is None else sl(d["S0"])[:, h0:h1])
+
+
+def test_prefill_batched_workload_sampled():
+    """B=8, T=8192, nonzero S0: the full launch on the GPU; the oracle checks the
+    first and last sequence on the first and last QK group (all their tokens)."""
+    w = inputs.PREFILL_BATCH8_8K
+    d = inputs.workload_inputs(w, device=DEV)
+    o, S = run_chunk(d)
+    for b, (h0, h1) in [(0, (0, 3)), (7, (45, 48)), (3, (21, 24))]:
+        o_ref, S_ref = oracle_ref(_sub_problem(d, b, h0, h1, w.Hv, w.Hqk))
+        check(o[b:b + 1, :, h0:h1], o_ref, TAU_BF16, f"o b={b} h={h0}:{h1}")
+        check(S[b:b + 1, h0:h1], S_ref, TAU_BF16, f"S_final b={b} h={h0}:{h1}")
+
+
+@pytest.mark.timeout(1800)
+def test_prefill_long_context_workload_sampled():
+    """B=1, T=262144 with long-memory gates: the full launch on the GPU; the oracle
+    follows two V heads (first and last) through all 262,144 tokens, which also
+    measures the drift of the fp32 state carried across 4096 chunks."""
+    w = inputs.PREFILL_256K
+    d = inputs.workload_inputs(w, device=DEV)
+    o, S = run_chunk(d)
+    for h in (0, 47):
+        o_ref, S_ref = oracle_ref(_sub_problem(d, 0, h, h + 1, w.Hv, w.Hqk))
+        check(o[:, :, h:h + 1], o_ref, TAU_BF16, f"o h={h}")
+        check(S[:, h:h + 1], S_ref, TAU_BF16, f"S_final h={h}")
+
+
+def test_prefill_empty_sequence_copies_state():
+    d = to_dev(inputs.prefill_inputs(2, 0, 2, 4, s0_std=1.0, seed=3))
+    o, S = run_chunk(d)
+    assert o.shape[1] == 0
+    assert torch.equal(S, d["S0"])
+    # and without S0 the final state is zero
+    d["S0"] = None
+    _, S = run_chunk(d)
+    assert torch.count_nonzero(S) == 0
+
+
+def test_prefill_in_place_state():
+    d = to_dev(inputs.prefill_inputs(2, 100, 2, 4, s0_std=0.3, seed=4))
+    o_ref, S_ref = run_chunk(d)
+    S = d["S0"].clone()
+    o = torch.empty_like(o_ref)
+    binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S, o, S)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+    assert torch.equal(S, S_ref)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_prefill_split_invariance(dtype):
+    """T1 tokens, then T2 tokens from the saved state, equals one call over T1+T2."""
+    d = to_dev(inputs.prefill_inputs(2, 300, 2, 6, dtype=dtype, s0_std=0.2, seed=5))
+    o, S = run_chunk(d)
+    T1 = 130
+    first = {k: (v[:, :T1].contiguous() if k != "S0" else v) for k, v in d.items()}
+    second = {k: (v[:, T1:].contiguous() if k != "S0" else v) for k, v in d.items()}
+    o1, S1 = run_chunk(first)
+    second["S0"] = S1
+    o2, S2 = run_chunk(second)
+    scale_o = o.abs().max().item()
+    tol = 1e-5 if dtype == torch.float32 else 1e-2
+    assert (torch.cat([o1, o2], 1).float() - o.float()).abs().max().item() <= tol * scale_o
+    assert (S2 - S).abs().max().item() <= tol * S.abs().max().item()
+
+
+def test_prefill_column_permutation_equivariance():
+    d = to_dev(inputs.prefill_inputs(1, 96, 1, 2, dtype=torch.float32, s0_std=0.2, seed=6))
+    perm = torch.randperm(128, generator=torch.Generator().manual_seed(0)).to(DEV)
+    o, S = run_chunk(d)
+    dp = dict(d)
+    dp["v"] = d["v"][..., perm].contiguous()
+    dp["S0"] = d["S0"][..., perm].contiguous()
+    o_p, S_p = run_chunk(dp)
+    assert (o_p - o[..., perm]).abs().max().item() <= 1e-6 * o.abs().max().item()
+    assert (S_p - S[..., perm]).abs().max().item() <= 1e-6 * S.abs().max().item()
+
+
+def test_prefill_rejects_misaligned_pointer():
+    d = to_dev(inputs.prefill_inputs(1, 8, 1, 1, dtype=torch.float32, seed=8))
+    flat = torch.empty(d["q"].numel() + 1, device=DEV)
+    q_off = flat[1:].view_as(d["q"])            # contiguous but 4 bytes off alignment
+    q_off.copy_(d["q"])
+    with pytest.raises(binding.GdnError, match="INVALID_ARG"):
+        binding.chunk_fwd(q_off, d["k"], d["v"], d["alpha"], d["beta"], None)
+
+
+# ----------------------------------------------------------------------------- decode
+def decode_run(w, steps, B=None, dtype=None):
+    """Runs `steps` decode steps on the GPU (state in place) and returns the per-step
+    outputs, the final state and the host copies of every step's inputs."""
+    B = B if B is not None else w.B
+    S = inputs.decode_state(w, device=DEV, B=B)
+    S0 = S.clone()
+    outs, ins = [], []
+    for s in range(steps):
+        x = inputs.decode_inputs(w, s, device=DEV, B=B)
+        if dtype is not None:
+            x = {k: (v.to(dtype) if v.dtype == torch.bfloat16 else v) for k, v in x.items()}
+        outs.append(binding.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S))
+        ins.append(x)
+    torch.cuda.synchronize()
+    return torch.stack(outs, 1), S, S0, ins
+
+
+def stacked(ins, key, seqs):
+    return torch.stack([x[key][seqs] for x in ins], 1)
+
+
+def test_decode_workload_all_sequences_first_steps():
+    """B=256, Hqk=16, Hv=48: 8 steps, every sequence and head against the oracle
+    run as one 8-token recurrence per (sequence, head)."""
+    w = inputs.DECODE_B256
+    o, S, S0, ins = decode_run(w, 8)
+    seqs = slice(None)
+    o_ref, S_ref = oracle.forward(stacked(ins, "q", seqs), stacked(ins, "k", seqs),
+                                  stacked(ins, "v", seqs), stacked(ins, "alpha", seqs),
+                                  stacked(ins, "beta", seqs), S0)
+    check(o, o_ref, TAU_BF16, "o")
+    check(S, S_ref, TAU_BF16, "S")
+
+
+@pytest.mark.timeout(1800)
+def test_decode_workload_1000_steps_sampled():
+    """The full 1000 decode steps at B=256; the oracle follows 8 sequences (all 48
+    heads) through all steps with its own fp64 state."""
+    w = inputs.DECODE_B256
+    o, S, S0, ins = decode_run(w, w.decode_steps)
+    seqs = torch.tensor([0, 1, 63, 100, 128, 200, 254, 255], device=DEV)
+    o_ref, S_ref = oracle.forward(stacked(ins, "q", seqs), stacked(ins, "k", seqs),
+                                  stacked(ins, "v", seqs), stacked(ins, "alpha", seqs),
+                                  stacked(ins, "beta", seqs), S0[seqs])
+    check(o[seqs], o_ref, TAU_BF16, "o")
+    check(S[seqs], S_ref, TAU_BF16, "S")
+
+
+def test_decode_fp32():
+    w = inputs.DECODE_B256
+    o, S, S0, ins = decode_run(w, 5, B=4, dtype=torch.float32)
+    seqs = slice(None)
+    o_ref, S_ref = oracle.forward(stacked(ins, "q", seqs), stacked(ins, "k", seqs),
+                                  stacked(ins, "v", seqs), stacked(ins, "alpha", seqs),
+                                  stacked(ins, "beta", seqs), S0)
+    check(o, o_ref, TAU_F32, "o")
+    check(S, S_ref, TAU_F32, "S")
+
+
+def test_decode_steps_equal_one_prefill():
+    """T decode calls reproduce one gdn_chunk_fwd over the same T tokens."""
+    d = to_dev(inputs.prefill_inputs(2, 70, 2, 6, dtype=torch.float32, s0_std=0.3, seed=11))
+    o_c, S_c = run_chunk(d)
+    S = d["S0"].clone()
+    outs = []
+    for t in range(70):
+        outs.append(binding.decode_step(d["q"][:, t].contiguous(), d["k"][:, t].contiguous(),
+                                        d["v"][:, t].contiguous(), d["alpha"][:, t].contiguous(),
+                                        d["beta"][:, t].contiguous(), S))
+    o_d = torch.stack(outs, 1)
+    torch.cuda.synchronize()
+    assert (o_d - o_c).abs().max().item() <= 1e-5 * o_c.abs().max().item()
+    assert (S - S_c).abs().max().item() <= 1e-5 * S_c.abs().max().item()
+
+
+def test_decode_out_of_place_leaves_input_state():
+    w = inputs.DECODE_B256
+    S = inputs.decode_state(w, device=DEV, B=3)
+    S_keep = S.clone()
+    x = inputs.decode_inputs(w, 0, device=DEV, B=3)
+    S_new = torch.empty_like(S)
+    o = torch.empty_like(x["v"])
+    binding.gdn_decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S, o, S_new)
+    S_in = S.clone()
+    o2 = binding.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S_in)
+    torch.cuda.synchronize()
+    assert torch.equal(S, S_keep)
+    assert torch.equal(S_new, S_in)
+    assert torch.equal(o, o2)
