@@ -122,7 +122,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -133,24 +133,27 @@ class ClockSampler:
                 self.proc.kill()
             self.thread.join(timeout=5)
 
-    def summary(self):
+    def summary(self, windows):
+        """Clock statistics over the samples that arrived inside the timed windows
+        (list of (t0, t1) perf_counter pairs)."""
         rows = []
-        for line in self.lines:
+        for ts, line in self.lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) != len(self.FIELDS):
                 continue
             try:
-                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:]))
+                rows.append((ts, float(parts[0]), float(parts[1]), parts[4:]))
             except ValueError:
                 continue
         if not rows:
             return None
-        loaded = [r for r in rows if r[2] >= 50] or rows
-        reasons = sorted({name for r in loaded for name, val in zip(self.REASONS, r[3])
+        inside = [r for r in rows if any(t0 <= r[0] <= t1 for t0, t1 in windows)]
+        use = inside or rows
+        reasons = sorted({name for r in use for name, val in zip(self.REASONS, r[3])
                           if val.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in loaded),
-                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows), "samples_under_load": len([r for r in rows if r[2] >= 50])}
+        return {"sm_mhz": statistics.median(r[1] for r in use),
+                "sm_max_mhz": max(r[2] for r in rows), "reasons": reasons,
+                "samples": len(rows), "samples_in_timed_region": len(inside)}
 
 
 # ----------------------------------------------------------------------------- dist
@@ -176,13 +179,19 @@ def barrier(world):
     torch.cuda.synchronize()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
+    """Largest value of x over all ranks (the job's elapsed time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank_per_step, steps, world, max_total_ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return world * units_per_rank_per_step * steps / (max_total_ms * 1e-3)
 
 
 # ----------------------------------------------------------------------------- timing
@@ -210,12 +219,13 @@ def time_prefill(w, steps, warmup, world, rank):
         step()
         ev[i][1].record(stream)
     barrier(world)
-    wall = time.perf_counter() - wall0
+    wall1 = time.perf_counter()
+    wall = wall1 - wall0
     times = [a.elapsed_time(b) for a, b in ev]            # ms, per launch
     total_ms = max_over_ranks(sum(times), world)
     return {"total_ms": total_ms, "per_launch_ms": sum(times) / steps,
             "median_ms": statistics.median(times), "wall_s": wall, "launches": steps,
-            "o_checksum": float(o.float().abs().sum().item())}
+            "window": (wall0, wall1)}
 
 
 def time_prefill_e2e(w, steps, warmup, world):
@@ -269,14 +279,17 @@ def time_decode(w, steps, warmup, world, pool=16):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(steps)]
     barrier(world)
+    wall0 = time.perf_counter()
     for i in range(steps):
         ev[i][0].record(stream)
         step(i)
         ev[i][1].record(stream)
     barrier(world)
+    wall1 = time.perf_counter()
     times = [a.elapsed_time(b) for a, b in ev]
     total_ms = max_over_ranks(sum(times), world)
-    return {"total_ms": total_ms, "per_launch_ms": sum(times) / steps, "launches": steps}
+    return {"total_ms": total_ms, "per_launch_ms": sum(times) / steps, "launches": steps,
+            "window": (wall0, wall1)}
 
 
 # ----------------------------------------------------------------------------- oracle
@@ -361,10 +374,10 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -387,15 +400,16 @@ def main():
     e2e = time_prefill_e2e(w, args.e2e_steps, 3, world)
 
     tokens_per_step = w.B * w.T
-    value = world * tokens_per_step * args.steps / (pre["total_ms"] * 1e-3)
+    value = job_throughput(tokens_per_step, args.steps, world, pre["total_ms"])
     flops_launch = prefill_flops_per_token(w) * tokens_per_step
     bytes_launch = prefill_bytes_per_token(w) * tokens_per_step + w.B * prefill_state_bytes(w)
     t_launch = pre["per_launch_ms"] * 1e-3
     dec_bytes = decode_bytes_per_step(wd)
     t_dec = dec["per_launch_ms"] * 1e-3
-    clk = clocks.summary()
+    clk = clocks.summary([pre["window"], dec["window"]])
 
     if rank != 0:
+        shutdown(world)
         return
     line = {
         "metric": METRIC,
@@ -421,7 +435,7 @@ def main():
                          hbm_frac=bytes_launch / t_launch / 1e9 / peaks["hbm_gbs"]),
         "decode": {
             "metric": "decode steps/s", "workload": wd.name, "B": wd.B,
-            "value": world * args.decode_steps / (dec["total_ms"] * 1e-3), "unit": "steps/s",
+            "value": job_throughput(1, args.decode_steps, world, dec["total_ms"]), "unit": "steps/s",
             "ms_per_step": dec["total_ms"] / args.decode_steps,
             "roofline": dict(roofline("hbm", dec_bytes / t_dec / 1e9, peaks["hbm_gbs"], "GB/s",
                                       kernel_traffic("decode")),
@@ -429,7 +443,7 @@ def main():
                              algorithmic_bytes_per_launch=dec_bytes),
             "gpu_launches": dec["launches"],
         },
-        "e2e": {"value": world * tokens_per_step * args.e2e_steps / (e2e["total_ms"] * 1e-3),
+        "e2e": {"value": job_throughput(tokens_per_step, args.e2e_steps, world, e2e["total_ms"]),
                 "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"]},
         "gpu_launches": pre["launches"],
@@ -441,5 +455,12 @@ def main():
     print(json.dumps(line), flush=True)
 
 
+def shutdown(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 if __name__ == "__main__":
     main()
+    shutdown(int(os.environ.get("WORLD_SIZE", "1")))

@@ -1,0 +1,48 @@
+"""Runs a few launches of one kernel on one workload, for profiler captures.
+
+    python -m linear_attention_recurrence_07_b200.profile_cases prefill [--T 4096] [--launches 3]
+    python -m linear_attention_recurrence_07_b200.profile_cases decode [--B 64] [--launches 5]
+    python -m linear_attention_recurrence_07_b200.profile_cases prefill-fp32 [--T 1024]
+
+Each case builds its seeded inputs on the GPU, runs the entry point `--launches`
+times and synchronizes; it prints nothing but "ok".  Point a profiler at it with
+a kernel filter and a launch skip/count, e.g. skip the first two launches to
+capture a warm one.
+"""
+import argparse
+
+import torch
+
+from . import binding, inputs
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["prefill", "decode", "prefill-fp32"])
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--B", type=int, default=None)
+    ap.add_argument("--launches", type=int, default=3)
+    args = ap.parse_args()
+    if args.case in ("prefill", "prefill-fp32"):
+        w = inputs.PREFILL_4K if args.case == "prefill" else inputs.PREFILL_SMALL_FP32
+        T = args.T or (w.T if args.case == "prefill" else 1024)
+        B = args.B or w.B
+        d = inputs.prefill_inputs(B, T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.log_alpha,
+                                  w.s0_std, w.seed, "cuda")
+        o = torch.empty((B, T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
+        S = torch.empty((B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+        for _ in range(args.launches):
+            binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S)
+    else:
+        w = inputs.DECODE_B256
+        B = args.B or 64
+        S = inputs.decode_state(w, device="cuda", B=B)
+        x = inputs.decode_inputs(w, 0, device="cuda", B=B)
+        for _ in range(args.launches):
+            binding.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S)
+    torch.cuda.synchronize()
+    print("ok")
+
+
+if __name__ == "__main__":
+    main()
