@@ -18,7 +18,7 @@
 //   G    = [K;Q] K^T      (lanes 0-63: K K^T, lanes 64-127: Q K^T)    M=128 N=64  K=128
 //   W^T  = K^T (T diag(beta gamma))^T                                  M=128 N=64  K=64
 //   U^T  = V^T (T diag(beta))^T  -  S^T W^T                            M=128 N=64  K=64+128
-//   O^T  = S^T Q~^T + U^T P^T,  Q~ = diag(gamma) Q,  P = masked Gam o Q K^T
+//   O^T  = diag(gamma) (S^T Q^T) + U^T P^T,  P = masked Gam o Q K^T
 //   S^T <- gamma_{C-1} S^T + U^T K~,  K~ = diag(g) K                   M=128 N=128 K=64
 // The state S^T (128 lanes x 128 fp32 columns) stays in TMEM for the whole
 // sequence; its bf16 copy in shared memory is only an MMA operand.
@@ -29,10 +29,11 @@
 //               group has its inputs ready, state-dependent groups first
 //   warps 2-5   "prep" warpgroup, runs ahead of the state: gates, A and P from
 //               the grams, the triangular solve (fp32 CUDA cores + TF32 warp
-//               MMAs for the block merges), W^T to shared memory, Q~ and K~
+//               MMAs for the block merges), W^T to shared memory and K~
 //   warps 6-9   "chain" warpgroup, the state-dependent path: S^T -> bf16
-//               operand (+ decay of the fp32 state), U^T -> bf16 operand, and
-//               the O epilogue (staged in shared memory, one TMA store)
+//               operand (+ decay of the fp32 state), U^T -> bf16 operand, the
+//               gamma scaling of the S-part of O^T in TMEM, and the O epilogue
+//               (staged in shared memory, one TMA store)
 // The U^T and O^T accumulators are double-buffered, so the prep work of the
 // next chunk never waits for the state-dependent chain of the current one.
 //
@@ -97,12 +98,13 @@ constexpr int LDA = 68;                           // padded row stride (floats)
 constexpr uint32_t OFF_Y = OFF_A + 64 * LDA * 4;  // solve scratch, fp32 [32][LDY]
 constexpr int LDY = 40;
 // per-chunk gate vectors (2 buffers): b (log2 units), gamma, beta, g, beta*gamma,
-// and e32[i] = 2^(b_32 - b_i) for i < 32
+// alpha (as used: 2^(clamped log2 alpha)), and d31[i] = prod_{i<j<=31} alpha_j (i < 32)
 constexpr uint32_t OFF_GATE = OFF_Y + 32 * LDY * 4;
-constexpr int GV_B = 0, GV_GAM = 64, GV_BETA = 128, GV_G = 192, GV_BG = 256, GV_E32 = 320;
-constexpr uint32_t GATE_BUF = 352 * 4;
+constexpr int GV_B = 0, GV_GAM = 64, GV_BETA = 128, GV_G = 192, GV_BG = 256, GV_ALPHA = 320,
+              GV_D31 = 384;
+constexpr uint32_t GATE_BUF = 416 * 4;
 constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_BUF;
-constexpr uint32_t NBAR = 21;
+constexpr uint32_t NBAR = 23;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;    // tmem slot, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // slack for aligning the base
@@ -114,17 +116,19 @@ enum : int {
     B_V_FULL = 4, B_V_EMPTY = 5,
     B_G_FULL = 6,    // grams done
     B_W_FULL = 7,    // W^T, U~^T done
-    B_SOLVE = 8,     // prep: Bw, Bu, P, Q~ written (128)
+    B_SOLVE = 8,     // prep: Bw, Bu, P written (128)
     B_PREP = 9,      // prep: W, K~ written (128)
     B_GATES = 10,    // 2: gates of a chunk written
     B_S_READY = 12,  // chain: S^T bf16 written (128)
-    B_U_FULL = 13,   // U^T and S-part of O done
+    B_U_FULL = 13,   // U^T done
     B_U_READY = 14,  // chain: U^T bf16 of a chunk with even index written (128); odd: B_U_READY1
-    B_S_FULL = 15,   // state update and O done
+    B_S_FULL = 15,   // state update done
     B_O_FREE = 16,   // 2: O accumulator read out (128)
     B_DRAIN = 18,    // final MMA drain
     B_G_FREE = 19,   // prep: grams read out of TMEM (128)
     B_U_READY1 = 20,
+    B_X_FULL = 21,   // S-part of O^T (S^T Q^T) done
+    B_O_FULL = 22,   // O^T complete (after U^T P^T)
 };
 // One U_READY barrier per U^T buffer, so that a parity probe of chunk c - 2's
 // phase can never alias with a later completion on the same barrier.
@@ -137,7 +141,7 @@ constexpr uint32_t ID_U = idesc_bf16(128, 64, false, true, /*neg_b=*/true);
 constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
 constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);
 
-constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2Floor = -87.0f * 1.4426950408889634f;   // log alpha >= -87
 
 struct TcParams {
     const float *alpha, *beta, *S0;
@@ -242,7 +246,7 @@ __device__ __forceinline__ void mma_tf32_step(float *d, const float *X, int ldx,
     const uint32_t a3 = to_tf32(X[(xr0 + g + 8) * ldx + xc0 + t + 4]);
     const uint32_t b0 = to_tf32(Y[(yr0 + t) * ldy + yc0 + g]);
     const uint32_t b1 = to_tf32(Y[(yr0 + t + 4) * ldy + yc0 + g]);
-    asm volatile(
+    asm(   // not volatile: lets the compiler hoist the fragment loads of later steps
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -455,7 +459,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // ======================================================== MMA issuer
         // Issues, as soon as their inputs are ready, in this priority order:
         //   YS(c): O^T += U^T P^T, S^T += U^T K~     needs U^T bf16 of chunk c
-        //   UO(c): U^T += S^T (-W)^T, O^T = S^T Q~^T  needs S^T bf16 and prep of c
+        //   UO(c): U^T += S^T (-W)^T, O^T = S^T Q^T   needs S^T bf16 and prep of c
         //   WU(c): W^T, U~^T                          needs the solve of c
         //   G(c):  [K;Q] K^T                          needs the K/Q tiles of c
         if (lane == 0) {
@@ -468,15 +472,17 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int c = nys, s = c & 1;
                     tc_fence_after();
                     const uint32_t col_o = COL_O + s * 64;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16(tmem + col_o, smem_desc_sw128(sbase + OFF_U + k * 32, 16, 1024),
-                                 smem_desc_sw128(sbase + OFF_P + s * TILE + k * 32, 16, 1024), ID_O, true);
+                    // the state update first: the next chunk waits for it
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         mma_bf16(tmem + COL_S, smem_desc_sw128(sbase + OFF_U + k * 32, 16, 1024),
                                  smem_desc_sw128(sbase + OFF_KT + k * 2048, TILE, 1024), ID_S, true);
                     mma_commit(&bar[B_S_FULL]);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tmem + col_o, smem_desc_sw128(sbase + OFF_U + k * 32, 16, 1024),
+                                 smem_desc_sw128(sbase + OFF_P + s * TILE + k * 32, 16, 1024), ID_O, true);
+                    mma_commit(&bar[B_O_FULL]);
                     GDN_TRACE_AT(c, 5, true);
                     ++nys;
                     issued = true;
@@ -494,13 +500,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         mma_bf16(tmem + col_u, smem_desc_sw128(sbase + OFF_S + koff, 16, 1024),
                                  smem_desc_sw128(sbase + OFF_W + k * 2048, 2 * TILE, 1024), ID_U, true);
                     }
+                    mma_commit(&bar[B_U_FULL]);
+                    // S-part of O with the unscaled Q; the chain applies gamma_r afterwards
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t koff = (k >> 2) * 2 * TILE + (k & 3) * 32;
                         mma_bf16(tmem + col_o, smem_desc_sw128(sbase + OFF_S + koff, 16, 1024),
                                  smem_desc_sw128(st + TILE + koff, 16, 1024), ID_O, k > 0);
                     }
-                    mma_commit(&bar[B_U_FULL]);
+                    mma_commit(&bar[B_X_FULL]);
                     mma_commit(&bar[B_KQ_EMPTY + s]);
                     GDN_TRACE_AT(c, 2, true);
                     ++nuo;
@@ -545,7 +553,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 if (issued) {
                     idle_since = clock64();
                 } else {
-                    __nanosleep(256);
+                    __nanosleep(64);
                     if (clock64() - idle_since > (1ll << 32)) {
                         *abort_flag = 1;
                         atomicOr(&g_tc_error, 1u);
@@ -581,7 +589,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // ---- gates (warp 2): b in log2 units, gamma, beta, g, beta gamma, e32;
             //      padded rows carry alpha = 1, beta = 0 (neutral)
             if (warp == 2) {
-                const float la0 = clamped_log(nx_a0) * kLog2e, la1 = clamped_log(nx_a1) * kLog2e;
+                // log2 alpha, clamped at -87 / ln 2 (alpha = 0 stays finite)
+                const float la0 = fmaxf(fast_log2(nx_a0), kLog2Floor);
+                const float la1 = fmaxf(fast_log2(nx_a1), kLog2Floor);
                 const float be0 = nx_b0, be1 = nx_b1;
                 if (c + 1 < nchunks) load_gates(p, b, h, T, c + 1, lane, nx_a0, nx_a1, nx_b0, nx_b1);
                 float incl = la0 + la1;
@@ -592,7 +602,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
                 const float b0 = incl - la1, b1 = incl;
                 const float blast = __shfl_sync(0xffffffffu, incl, 31);
-                const float b32 = __shfl_sync(0xffffffffu, b0, 16);      // b at token 32
+                const float b31 = __shfl_sync(0xffffffffu, b1, 15);      // b at token 31
                 const float g0 = fast_exp2(b0), g1 = fast_exp2(b1);
                 gv[GV_B + 2 * lane] = b0;
                 gv[GV_B + 2 * lane + 1] = b1;
@@ -604,18 +614,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 gv[GV_G + 2 * lane + 1] = fast_exp2(blast - b1);
                 gv[GV_BG + 2 * lane] = be0 * g0;
                 gv[GV_BG + 2 * lane + 1] = be1 * g1;
+                gv[GV_ALPHA + 2 * lane] = fast_exp2(la0);
+                gv[GV_ALPHA + 2 * lane + 1] = fast_exp2(la1);
                 if (lane < 16) {   // tokens 2*lane, 2*lane+1 < 32
-                    gv[GV_E32 + 2 * lane] = fast_exp2(b32 - b0);
-                    gv[GV_E32 + 2 * lane + 1] = fast_exp2(b32 - b1);
+                    gv[GV_D31 + 2 * lane] = fast_exp2(b31 - b0);
+                    gv[GV_D31 + 2 * lane + 1] = fast_exp2(b31 - b1);
                 }
             }
             named_sync(1, 128);
             if (pt == 0) mbar_arrive(&bar[B_GATES + s]);
             // ---- grams -> A (rows 0-63, fp32) and P (rows 64-127, bf16 operand).
-            //      Decay factors use the anchor token 32: for i < 32 <= r,
-            //      2^(b_r - b_i) = 2^(b_r - b_32) 2^(b_32 - b_i), both factors <= 1.
-            // (P buffer s is free again: the previous prep iteration waited for the
-            //  state update of chunk c - 2, the last reader of that buffer.)
+            //      Decay factors Gam[r][x] = prod_{x<j<=r} alpha_j are running products
+            //      along the row (no special-function work): descending from x = r,
+            //      Gam[r][x-1] = Gam[r][x] alpha_x.  Rows r >= 32 continue into columns
+            //      x < 32 through the table d31[x] = Gam[31][x]: Gam[r][x] = Gam[r][31] d31[x].
+            //      (P buffer s is free again: the previous prep iteration waited for
+            //      the last reader of that buffer, the O update of chunk c - 2.)
             ok = ctl.wait(B_KQ_FULL + s, (c >> 1) & 1) && ctl.wait(B_G_FULL, c & 1);
             ok = named_and(1, 128, ok);   // same decision in the whole warpgroup
             if (!ok) break;
@@ -623,40 +637,41 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             GDN_TRACE_AT(c, 10, pt == 0);
             {
                 const int r = row & 63;
-                const float br = gv[GV_B + r];
-                const float scale = row < 64 ? gv[GV_BETA + r] : 1.f;
-                const bool low = r < 32;                 // warp-uniform
-                const float er = low ? 1.f : fast_exp2(br - gv[GV_B + 32]);
+                const bool is_a = row < 64;                // A rows: strict lower; P rows: i <= r
+                const bool low = r < 32;                   // warp-uniform
                 float g0[32], g1[32];
                 tmem_ld32(t_row + COL_G, g0);
                 tmem_ld32(t_row + COL_G + 32, g1);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&bar[B_G_FREE]);
-                // columns 0-31
+                float run = is_a ? gv[GV_BETA + r] : 1.f;   // row scale folded into the product
                 if (low) {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        const bool keep = row < 64 ? x < r : x <= r;
-                        g0[x] = keep ? scale * fast_exp2(br - gv[GV_B + x]) * g0[x] : 0.f;
+                    for (int x = 31; x >= 0; --x) {
+                        const bool on = x <= r;
+                        const bool keep = is_a ? x < r : on;
+                        const float val = run * g0[x];
+                        g0[x] = keep ? val : 0.f;
+                        run = on ? run * gv[GV_ALPHA + x] : run;
                     }
-                } else {
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) g0[x] = scale * er * gv[GV_E32 + x] * g0[x];
-                }
-                // columns 32-63 (all zero for rows below 32)
-                if (low) {
 #pragma unroll
                     for (int x = 0; x < 32; ++x) g1[x] = 0.f;
                 } else {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
+                    for (int x = 31; x >= 0; --x) {
                         const int i = 32 + x;
-                        const bool keep = row < 64 ? i < r : i <= r;
-                        g1[x] = keep ? scale * fast_exp2(br - gv[GV_B + i]) * g1[x] : 0.f;
+                        const bool on = i <= r;
+                        const bool keep = is_a ? i < r : on;
+                        const float val = run * g1[x];
+                        g1[x] = keep ? val : 0.f;
+                        run = on ? run * gv[GV_ALPHA + i] : run;
                     }
+                    // run = scale * Gam[r][31]
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) g0[x] = run * gv[GV_D31 + x] * g0[x];
                 }
-                if (row < 64) {
+                if (is_a) {
                     float4 *dst = reinterpret_cast<float4 *>(sA + r * LDA);
 #pragma unroll
                     for (int x = 0; x < 8; ++x) dst[x] = make_float4(g0[4 * x], g0[4 * x + 1], g0[4 * x + 2], g0[4 * x + 3]);
@@ -666,12 +681,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     store_half_row_bf16(sm + OFF_P + s * TILE, r, 0, g0);
                     store_half_row_bf16(sm + OFF_P + s * TILE, r, 1, g1);
                 }
-            }
-            // Q~ = diag(gamma) Q, in place in the stage (the grams have consumed Q)
-            {
-                const int i = pt >> 1, half = pt & 1;
-                unsigned char *qt = sm + OFF_KQ + s * KQ_STAGE + (1 + 2 * half) * TILE;
-                scale_row_bf16(qt, qt, i, gv[GV_GAM + i]);
             }
             named_sync(1, 128);
             GDN_TRACE_AT(c, 11, pt == 0);
@@ -702,7 +711,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // ---- W^T -> W [d][r] (MN-major B) ; K~ = diag(g) K.  The single-buffered
             //      W and K~ must no longer be read by the previous chunk's MMAs.
             ok = ctl.wait(B_W_FULL, c & 1) && (c < 1 || ctl.wait(B_U_FULL, (c - 1) & 1)) &&
-                 (c < 1 || ctl.wait(B_S_FULL, (c - 1) & 1));
+                 (c < 1 || ctl.wait(B_O_FULL, (c - 1) & 1));   // also frees P of chunk c-1
             ok = named_and(1, 128, ok);
             if (!ok) break;
             tc_fence_after();
@@ -774,7 +783,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             GDN_TRACE_AT(c, 18, leader);
             // O epilogue of the previous chunk: O^T (lane j) -> bf16 tile [r][j] in the
             // U^T buffer (idle from the state update of c-1 to the U^T of c) -> TMA store
+            if (c > 0) ok = named_and(2, 128, ctl.wait(B_O_FULL, (c - 1) & 1));
+            if (!ok) break;
             if (c > 0) {
+                tc_fence_after();
                 const int cp = c - 1;
                 const uint32_t col_o = COL_O + (cp & 1) * 64;
                 unsigned char *ot = sm + OFF_U + (j >> 6) * TILE;
@@ -814,13 +826,31 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tmem_wait_ld();
                 store_row_bf16(sm + OFF_U, j, u);
             }
+            // O^T S-part: column r times gamma_r (Q~ = diag(gamma) Q applied here)
+            ok = named_and(2, 128, ctl.wait(B_X_FULL, c & 1));
+            if (!ok) break;
+            tc_fence_after();
+            {
+                const float *gam = reinterpret_cast<const float *>(sm + OFF_GATE + s * GATE_BUF) + GV_GAM;
+                const uint32_t col_o = COL_O + s * 64;
+#pragma unroll 1
+                for (int r0 = 0; r0 < C; r0 += 32) {
+                    float xv[32];
+                    tmem_ld32(t_row + col_o + r0, xv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) xv[x] *= gam[r0 + x];
+                    tmem_st32(t_row + col_o + r0, xv);
+                }
+                tmem_wait_st();
+            }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bar[u_ready(c)]);
             GDN_TRACE_AT(c, 21, leader);
         }
         if (ok && nchunks > 0) {
-            ok = named_and(2, 128, ctl.wait(B_S_FULL, (nchunks - 1) & 1));
+            ok = named_and(2, 128, ctl.wait(B_O_FULL, (nchunks - 1) & 1));
             if (ok) {
                 tc_fence_after();
                 const int cp = nchunks - 1;

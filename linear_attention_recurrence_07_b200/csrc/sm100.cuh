@@ -55,6 +55,12 @@ __device__ __forceinline__ float fast_exp2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// log2(x) on the special-function unit (max relative error about 2^-22).
+__device__ __forceinline__ float fast_log2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 // Waits for the phase with the given parity to complete.  Gives up after
 // `limit_cycles` SM clocks and returns false instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
