@@ -80,15 +80,16 @@ def load_peaks():
 
 def kernel_traffic(kernel):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current source of that kernel (else None)."""
+    current sources of that kernel (all files it is built from; else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             entry = json.load(f)[kernel]
-        src = os.path.join(ROOT, entry["source"])
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
-        if sha != entry["source_sha256_16"]:
+        h = hashlib.sha256()
+        for src in entry["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != entry["sources_sha256_16"]:
             return None
         return float(entry["bytes_per_launch"])
     except (OSError, KeyError, ValueError):
@@ -380,6 +381,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto",
+                    help="prefill kernel to time (default: the library's own choice)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -393,6 +396,8 @@ def main():
     peaks, peak_src = load_peaks()
     w = inputs.PREFILL_4K
     wd = inputs.DECODE_B256
+    binding.set_prefill_kernel(args.prefill_kernel)
+    kernel = binding.prefill_kernel_for(w.B, w.Hv, w.dtype)
 
     with ClockSampler(local) as clocks:
         pre = time_prefill(w, args.steps, args.warmup, world, rank)
@@ -426,10 +431,11 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "Hqk": w.Hqk, "Hv": w.Hv,
                    "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "state": "fp32",
+                   "prefill_kernel": kernel,
                    "l2": "flushed before every timed step (256 MiB write)",
                    "parallelism": f"dp{world} (independent sequences per GPU)"},
         "roofline": dict(roofline("tensor", flops_launch / t_launch / 1e12, peaks["bf16_tflops"],
-                                  "TFLOP/s", kernel_traffic("prefill")),
+                                  "TFLOP/s", kernel_traffic("prefill_" + kernel)),
                          peak_source=f"{peak_src} bf16 burst",
                          algorithmic_flops_per_launch=flops_launch,
                          hbm_frac=bytes_launch / t_launch / 1e9 / peaks["hbm_gbs"]),

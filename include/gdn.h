@@ -103,6 +103,46 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            int B, int Hqk, int Hv, int dk, int dv,
                            gdn_dtype dtype, void *stream);
 
+/*
+ * Prefill kernel selection (library-specific: the page describes the method,
+ * not how its evaluation is split over the GPU).
+ *
+ *   GDN_PREFILL_AUTO        default: GDN_BF16 runs on the tensor cores
+ *                           (GDN_PREFILL_TC in this version), GDN_F32 on the
+ *                           CUDA-core kernel
+ *   GDN_PREFILL_SIMT        CUDA-core chunk kernel, both dtypes
+ *   GDN_PREFILL_TC          tensor cores, one CTA per (sequence, V head)
+ *   GDN_PREFILL_TC_CLUSTER  tensor cores, a cluster of two CTAs per
+ *                           (sequence, V head): one carries the state, the
+ *                           other prepares the chunks' WY factors
+ * All variants compute the same function (to the dtype's rounding); the two TC
+ * variants return identical bits.  The TC variants take GDN_BF16 only: with
+ * another choice gdn_chunk_fwd returns GDN_ERR_UNSUPPORTED, as it does when
+ * the tensor-map encoder is missing.
+ *
+ * gdn_set_prefill_kernel sets the choice for every later gdn_chunk_fwd call of
+ * the process (all threads and devices); it returns GDN_ERR_INVALID_ARG for a
+ * value outside the enum.  gdn_get_prefill_kernel returns the current choice.
+ */
+typedef enum {
+    GDN_PREFILL_AUTO = 0,
+    GDN_PREFILL_SIMT = 1,
+    GDN_PREFILL_TC = 2,
+    GDN_PREFILL_TC_CLUSTER = 3
+} gdn_prefill_kernel;
+
+gdn_status gdn_set_prefill_kernel(gdn_prefill_kernel kernel);
+gdn_prefill_kernel gdn_get_prefill_kernel(void);
+
+/*
+ * The kernel (a gdn_prefill_kernel value, never GDN_PREFILL_AUTO) that
+ * gdn_chunk_fwd runs for B sequences of Hv V heads in `dtype` under the current
+ * choice, on the calling thread's current CUDA device; -1 if that call would
+ * return GDN_ERR_UNSUPPORTED (a forced TC kernel with GDN_F32) or the arguments
+ * are invalid.  No kernel is launched.
+ */
+int gdn_prefill_kernel_for(int B, int Hv, gdn_dtype dtype);
+
 /* Static, NUL-terminated name of a status code. */
 const char *gdn_status_string(gdn_status status);
 

@@ -6,6 +6,7 @@ the C entry points.  All computation happens in the library's CUDA kernels.
 PyTorch is used for device memory and streams.  If the shared library is
 missing, every call raises ``GdnError``: there is no fallback.
 """
+import contextlib
 import ctypes
 import os
 
@@ -17,6 +18,8 @@ LIBRARY_PATH = os.path.join(_PKG, "libgdn.so")
 GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA = 0, 1, 2, 3
 GDN_F32, GDN_BF16 = 0, 1
 _DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
+# gdn_prefill_kernel values
+PREFILL_KERNELS = {"auto": 0, "simt": 1, "tc": 2, "tc_cluster": 3}
 
 
 class GdnError(RuntimeError):
@@ -51,6 +54,12 @@ def library():
         lib.gdn_last_cuda_error.restype = I
         lib.gdn_version.argtypes = []
         lib.gdn_version.restype = I
+        lib.gdn_set_prefill_kernel.argtypes = [I]
+        lib.gdn_set_prefill_kernel.restype = I
+        lib.gdn_get_prefill_kernel.argtypes = []
+        lib.gdn_get_prefill_kernel.restype = I
+        lib.gdn_prefill_kernel_for.argtypes = [I, I, I]
+        lib.gdn_prefill_kernel_for.restype = I
         _lib = lib
     return _lib
 
@@ -138,6 +147,42 @@ def gdn_decode_step(q, k, v, alpha, beta, S, o, S_new, stream=None):
                                      _ptr(o), _ptr(S_new), B, Hqk, Hv, dk, dv,
                                      _DTYPES[q.dtype], _stream_handle(stream, dev)),
            "gdn_decode_step")
+
+
+def set_prefill_kernel(name):
+    """Selects the kernel of every later prefill call in this process (C entry point
+    ``gdn_set_prefill_kernel``): one of ``PREFILL_KERNELS``."""
+    if name not in PREFILL_KERNELS:
+        raise GdnError(f"unknown prefill kernel {name!r}; one of {sorted(PREFILL_KERNELS)}")
+    _check(library().gdn_set_prefill_kernel(PREFILL_KERNELS[name]), "gdn_set_prefill_kernel")
+
+
+def get_prefill_kernel():
+    """The current prefill kernel choice, as a key of ``PREFILL_KERNELS``."""
+    code = library().gdn_get_prefill_kernel()
+    return {v: k for k, v in PREFILL_KERNELS.items()}[code]
+
+
+def prefill_kernel_for(B, Hv, dtype):
+    """The kernel a prefill of B sequences x Hv V heads in ``dtype`` (a torch dtype)
+    runs under the current choice (C entry point ``gdn_prefill_kernel_for``)."""
+    code = library().gdn_prefill_kernel_for(B, Hv, _DTYPES[dtype])
+    if code < 0:
+        raise GdnError(f"no prefill kernel takes B={B}, Hv={Hv}, {dtype} under the current choice",
+                       GDN_ERR_UNSUPPORTED)
+    return {v: k for k, v in PREFILL_KERNELS.items()}[code]
+
+
+@contextlib.contextmanager
+def prefill_kernel(name):
+    """Context manager: ``name`` is the prefill kernel inside the block, the previous
+    choice is restored after it."""
+    prev = get_prefill_kernel()
+    set_prefill_kernel(name)
+    try:
+        yield
+    finally:
+        set_prefill_kernel(prev)
 
 
 def chunk_fwd(q, k, v, alpha, beta, S0=None, chunk=64, stream=None):

@@ -40,39 +40,13 @@
 // Every wait is bounded.  On a timeout the CTA raises a device error flag, the
 // other roles see a shared abort flag and stop, in-flight copies and MMAs are
 // drained (again with a bound) and TMEM is freed before returning.
-#include <cuda.h>
-
-#include "gdn_internal.cuh"
-#include "sm100.cuh"
+#include "tc_common.cuh"
 
 namespace gdn {
 
-__device__ unsigned int g_tc_error = 0;   // set when a bounded wait gave up
-
-// Optional event trace (build with -DGDN_TRACE): block (0, 0) records %globaltimer
-// at fixed points of every role for the first kTraceChunks chunks.
-#ifdef GDN_TRACE
-constexpr int kTraceChunks = 16, kTraceSlots = 32;
-__device__ unsigned long long g_trace[kTraceChunks][kTraceSlots];
-__device__ __forceinline__ void trace(int c, int slot, bool leader) {
-    if (leader && blockIdx.x == 0 && blockIdx.y == 0 && c < kTraceChunks) {
-        unsigned long long t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        g_trace[c][slot] = t;
-    }
-}
-#define GDN_TRACE_AT(c, slot, leader) trace((c), (slot), (leader))
-#else
-#define GDN_TRACE_AT(c, slot, leader) ((void)0)
-#endif
-
 namespace {
 
-using namespace sm100;
-
-constexpr int C = kChunk;          // 64
 constexpr int NT = 320;            // 10 warps
-constexpr uint32_t TILE = 8192;    // one 64 x 64 bf16 tile, 128B-swizzled
 
 // TMEM columns (fp32 accumulators over 128 lanes)
 constexpr uint32_t COL_S = 0;      // S^T: 128 columns
@@ -94,15 +68,8 @@ constexpr uint32_t OFF_W = OFF_BU + TILE;         // W stored [d][r] (MN-major B
 constexpr uint32_t OFF_S = OFF_W + 2 * TILE;      // S^T bf16 [j][d], two 64-column halves
 constexpr uint32_t OFF_U = OFF_S + 4 * TILE;      // U^T bf16 [j][i]; between chunks: O staging [r][j]
 constexpr uint32_t OFF_A = OFF_U + 2 * TILE;      // A, then T = (I + A)^-1, fp32 [64][LDA]
-constexpr int LDA = 68;                           // padded row stride (floats)
 constexpr uint32_t OFF_Y = OFF_A + 64 * LDA * 4;  // solve scratch, fp32 [32][LDY]
-constexpr int LDY = 40;
-// per-chunk gate vectors (2 buffers): b (log2 units), gamma, beta, g, beta*gamma,
-// alpha (as used: 2^(clamped log2 alpha)), and d31[i] = prod_{i<j<=31} alpha_j (i < 32)
-constexpr uint32_t OFF_GATE = OFF_Y + 32 * LDY * 4;
-constexpr int GV_B = 0, GV_GAM = 64, GV_BETA = 128, GV_G = 192, GV_BG = 256, GV_ALPHA = 320,
-              GV_D31 = 384;
-constexpr uint32_t GATE_BUF = 416 * 4;
+constexpr uint32_t OFF_GATE = OFF_Y + 32 * LDY * 4;  // 2 buffers of gate vectors
 constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_BUF;
 constexpr uint32_t NBAR = 23;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;    // tmem slot, abort flag
@@ -133,253 +100,6 @@ enum : int {
 // One U_READY barrier per U^T buffer, so that a parity probe of chunk c - 2's
 // phase can never alias with a later completion on the same barrier.
 __host__ __device__ constexpr int u_ready(int c) { return (c & 1) ? B_U_READY1 : B_U_READY; }
-
-constexpr uint32_t ID_G = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_W = idesc_bf16(128, 64, true, false);
-constexpr uint32_t ID_UT = idesc_bf16(128, 64, true, false);
-constexpr uint32_t ID_U = idesc_bf16(128, 64, false, true, /*neg_b=*/true);
-constexpr uint32_t ID_O = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_S = idesc_bf16(128, 128, false, true);
-
-constexpr float kLog2Floor = -87.0f * 1.4426950408889634f;   // log alpha >= -87
-
-struct TcParams {
-    const float *alpha, *beta, *S0;
-    float *S_final;
-    int T, Hqk, Hv;
-};
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t *>(&h);
-}
-
-// 64 fp32 values (one row) -> bf16 row `row` of a 128B-swizzled tile.
-__device__ __forceinline__ void store_row_bf16(unsigned char *tile, uint32_t row, const float *x) {
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        uint4 v;
-        v.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
-        v.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
-        v.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
-        v.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-        *reinterpret_cast<uint4 *>(tile + sw128_chunk(row, c)) = v;
-    }
-}
-
-// 32 fp32 values -> bf16 elements 32*half .. 32*half+31 of row `row` (4 chunks).
-__device__ __forceinline__ void store_half_row_bf16(unsigned char *tile, uint32_t row, int half,
-                                                    const float *x) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        uint4 v;
-        v.x = pack_bf16x2(x[8 * c + 0], x[8 * c + 1]);
-        v.y = pack_bf16x2(x[8 * c + 2], x[8 * c + 3]);
-        v.z = pack_bf16x2(x[8 * c + 4], x[8 * c + 5]);
-        v.w = pack_bf16x2(x[8 * c + 6], x[8 * c + 7]);
-        *reinterpret_cast<uint4 *>(tile + sw128_chunk(row, 4 * half + c)) = v;
-    }
-}
-
-// Scales row `row` (64 bf16, swizzled) of a tile in place / into another tile.
-__device__ __forceinline__ void scale_row_bf16(const unsigned char *src, unsigned char *dst,
-                                               uint32_t row, float s) {
-#pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-        const uint32_t off = sw128_chunk(row, ch);
-        uint4 v = *reinterpret_cast<const uint4 *>(src + off);
-        __nv_bfloat162 *hv = reinterpret_cast<__nv_bfloat162 *>(&v);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(hv[e]);
-            hv[e] = __floats2bfloat162_rn(f.x * s, f.y * s);
-        }
-        *reinterpret_cast<uint4 *>(dst + off) = v;
-    }
-}
-
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-// Named barrier that also returns the AND of `v` over the participating threads.
-__device__ __forceinline__ bool named_and(int id, int nthreads, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 q, %1, 0;\n\t"
-        "bar.red.and.pred p, %2, %3, q;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(r) : "r"((uint32_t)v), "r"(id), "r"(nthreads) : "memory");
-    return r != 0;
-}
-// Non-blocking probe of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(done) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return done != 0;
-}
-
-// ---------------------------------------------------------------- triangular solve
-// T = (I + A)^-1 for the 64 x 64 strictly lower A in sA (row stride LDA), in place,
-// by the 128 threads of one warpgroup (named barrier `bid`).  Blocked: 8 x 8
-// diagonal blocks by substitution, then merges 8 -> 16 on CUDA cores and
-// 16 -> 32 -> 64 with warp-level TF32 tensor-core products, using
-// T_ba = -T_bb (A_ba T_aa) for the block below the diagonal of each merge.
-// (The merges are 16- and 32-wide products: too small for a tcgen05 tile and
-// its TMEM round trip, so they run as register-resident warp MMAs.)
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-// d (16 x 8 fp32 fragment) += X[xr0.., xc0..xc0+8) * Y[yr0..yr0+8, yc0..yc0+8)
-__device__ __forceinline__ void mma_tf32_step(float *d, const float *X, int ldx, int xr0, int xc0,
-                                              const float *Y, int ldy, int yr0, int yc0, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    const uint32_t a0 = to_tf32(X[(xr0 + g) * ldx + xc0 + t]);
-    const uint32_t a1 = to_tf32(X[(xr0 + g + 8) * ldx + xc0 + t]);
-    const uint32_t a2 = to_tf32(X[(xr0 + g) * ldx + xc0 + t + 4]);
-    const uint32_t a3 = to_tf32(X[(xr0 + g + 8) * ldx + xc0 + t + 4]);
-    const uint32_t b0 = to_tf32(Y[(yr0 + t) * ldy + yc0 + g]);
-    const uint32_t b1 = to_tf32(Y[(yr0 + t + 4) * ldy + yc0 + g]);
-    asm(   // not volatile: lets the compiler hoist the fragment loads of later steps
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
-        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void store_frag(float *D, int ldd, int r0, int c0, const float *d,
-                                           float s, int lane) {
-    const int g = lane >> 2, t = lane & 3;
-    D[(r0 + g) * ldd + c0 + 2 * t] = s * d[0];
-    D[(r0 + g) * ldd + c0 + 2 * t + 1] = s * d[1];
-    D[(r0 + g + 8) * ldd + c0 + 2 * t] = s * d[2];
-    D[(r0 + g + 8) * ldd + c0 + 2 * t + 1] = s * d[3];
-}
-
-__device__ void unit_lower_inverse(float *sA, float *sY, int t, int bid) {
-    const int warp = t >> 5, lane = t & 31;
-    // 8 x 8 diagonal blocks: thread (block kb, column cl), right-looking substitution
-    if (t < 64) {
-        const int kb = t >> 3, cl = t & 7;
-        float x[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) x[r] = (r == cl) ? 1.f : 0.f;
-#pragma unroll
-        for (int r = 0; r < 7; ++r) {
-            const float xr = x[r];
-#pragma unroll
-            for (int q = r + 1; q < 8; ++q) x[q] = fmaf(-sA[(8 * kb + q) * LDA + 8 * kb + r], xr, x[q]);
-        }
-        named_sync(bid, 128);
-#pragma unroll
-        for (int r = 0; r < 8; ++r) sA[(8 * kb + r) * LDA + 8 * kb + cl] = x[r];
-    } else {
-        named_sync(bid, 128);
-    }
-    named_sync(bid, 128);
-    // 8 -> 16 inside each 16 x 16 diagonal block: thread (block k, row r, 2 columns)
-    {
-        const int k = t >> 5, r = (t >> 2) & 7, c0 = (t & 3) * 2;
-        const int ra = 16 * k, rb = 16 * k + 8;
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float av = sA[(rb + r) * LDA + ra + i];
-            y0 = fmaf(av, sA[(ra + i) * LDA + ra + c0], y0);
-            y1 = fmaf(av, sA[(ra + i) * LDA + ra + c0 + 1], y1);
-        }
-        sY[k * 64 + r * 8 + c0] = y0;
-        sY[k * 64 + r * 8 + c0 + 1] = y1;
-        named_sync(bid, 128);
-        float z0 = 0.f, z1 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float tv = sA[(rb + r) * LDA + rb + i];
-            z0 = fmaf(-tv, sY[k * 64 + i * 8 + c0], z0);
-            z1 = fmaf(-tv, sY[k * 64 + i * 8 + c0 + 1], z1);
-        }
-        sA[(rb + r) * LDA + ra + c0] = z0;
-        sA[(rb + r) * LDA + ra + c0 + 1] = z1;
-    }
-    named_sync(bid, 128);
-    // 16 -> 32 for the blocks (16-31, 0-15) and (48-63, 32-47): warp -> (block, 8-column tile)
-    {
-        const int blk = warp >> 1, nt = warp & 1;
-        const int a = 32 * blk, bb = a + 16;
-        float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-            mma_tf32_step(d, sA, LDA, bb, a + 8 * ks, sA, LDA, a + 8 * ks, a + 8 * nt, lane);
-        store_frag(sY + blk * 16 * LDY, LDY, 0, 8 * nt, d, 1.f, lane);
-        named_sync(bid, 128);
-        float e[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 2; ++ks)
-            mma_tf32_step(e, sA, LDA, bb, bb + 8 * ks, sY + blk * 16 * LDY, LDY, 8 * ks, 8 * nt, lane);
-        store_frag(sA, LDA, bb, a + 8 * nt, e, -1.f, lane);
-    }
-    named_sync(bid, 128);
-    // 32 -> 64 for the block (32-63, 0-31): warp -> (16-row tile, two 8-column tiles)
-    {
-        const int mt = warp >> 1, n0 = 2 * (warp & 1);
-        float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            mma_tf32_step(d0, sA, LDA, 32 + 16 * mt, 8 * ks, sA, LDA, 8 * ks, 8 * n0, lane);
-            mma_tf32_step(d1, sA, LDA, 32 + 16 * mt, 8 * ks, sA, LDA, 8 * ks, 8 * (n0 + 1), lane);
-        }
-        store_frag(sY, LDY, 16 * mt, 8 * n0, d0, 1.f, lane);
-        store_frag(sY, LDY, 16 * mt, 8 * (n0 + 1), d1, 1.f, lane);
-        named_sync(bid, 128);
-        float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            mma_tf32_step(e0, sA, LDA, 32 + 16 * mt, 32 + 8 * ks, sY, LDY, 8 * ks, 8 * n0, lane);
-            mma_tf32_step(e1, sA, LDA, 32 + 16 * mt, 32 + 8 * ks, sY, LDY, 8 * ks, 8 * (n0 + 1), lane);
-        }
-        store_frag(sA, LDA, 32 + 16 * mt, 8 * n0, e0, -1.f, lane);
-        store_frag(sA, LDA, 32 + 16 * mt, 8 * (n0 + 1), e1, -1.f, lane);
-    }
-    named_sync(bid, 128);
-}
-
-// alpha, beta of tokens 2*lane, 2*lane+1 of chunk cn (alpha = 1, beta = 0 past the end)
-__device__ __forceinline__ void load_gates(const TcParams &p, int b, int h, int T, int cn, int lane,
-                                           float &a0, float &a1, float &b0, float &b1) {
-    const int tn = cn * C, Ln = min(C, T - tn);
-    const int r = 2 * lane;
-    const size_t gi = ((size_t)b * T + tn + r) * p.Hv + h;
-    a0 = r < Ln ? p.alpha[gi] : 1.f;
-    b0 = r < Ln ? p.beta[gi] : 0.f;
-    a1 = r + 1 < Ln ? p.alpha[gi + p.Hv] : 1.f;
-    b1 = r + 1 < Ln ? p.beta[gi + p.Hv] : 0.f;
-}
-
-struct Ctl {
-    uint64_t *bar;
-    volatile int *abort_flag;
-    // Bounded wait that also gives up as soon as another role aborted.  The
-    // thread sleeps in the barrier unit between checks, so waiting roles do not
-    // take issue slots from the working ones.
-    __device__ __forceinline__ bool wait(int i, uint32_t parity) const {
-        if (mbar_try_wait(&bar[i], parity)) return true;
-        const long long t0 = clock64();
-        for (;;) {
-            if (mbar_try_wait_suspend(&bar[i], parity, 20000)) return true;
-            if (*abort_flag) return false;
-            if (clock64() - t0 > (1ll << 32)) {
-                *abort_flag = 1;
-                atomicOr(&g_tc_error, 1u);
-                return false;
-            }
-        }
-    }
-};
 
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
@@ -589,37 +309,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // ---- gates (warp 2): b in log2 units, gamma, beta, g, beta gamma, e32;
             //      padded rows carry alpha = 1, beta = 0 (neutral)
             if (warp == 2) {
-                // log2 alpha, clamped at -87 / ln 2 (alpha = 0 stays finite)
-                const float la0 = fmaxf(fast_log2(nx_a0), kLog2Floor);
-                const float la1 = fmaxf(fast_log2(nx_a1), kLog2Floor);
-                const float be0 = nx_b0, be1 = nx_b1;
+                const float a0 = nx_a0, a1 = nx_a1, be0 = nx_b0, be1 = nx_b1;
                 if (c + 1 < nchunks) load_gates(p, b, h, T, c + 1, lane, nx_a0, nx_a1, nx_b0, nx_b1);
-                float incl = la0 + la1;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += y;
-                }
-                const float b0 = incl - la1, b1 = incl;
-                const float blast = __shfl_sync(0xffffffffu, incl, 31);
-                const float b31 = __shfl_sync(0xffffffffu, b1, 15);      // b at token 31
-                const float g0 = fast_exp2(b0), g1 = fast_exp2(b1);
-                gv[GV_B + 2 * lane] = b0;
-                gv[GV_B + 2 * lane + 1] = b1;
-                gv[GV_GAM + 2 * lane] = g0;
-                gv[GV_GAM + 2 * lane + 1] = g1;
-                gv[GV_BETA + 2 * lane] = be0;
-                gv[GV_BETA + 2 * lane + 1] = be1;
-                gv[GV_G + 2 * lane] = fast_exp2(blast - b0);
-                gv[GV_G + 2 * lane + 1] = fast_exp2(blast - b1);
-                gv[GV_BG + 2 * lane] = be0 * g0;
-                gv[GV_BG + 2 * lane + 1] = be1 * g1;
-                gv[GV_ALPHA + 2 * lane] = fast_exp2(la0);
-                gv[GV_ALPHA + 2 * lane + 1] = fast_exp2(la1);
-                if (lane < 16) {   // tokens 2*lane, 2*lane+1 < 32
-                    gv[GV_D31 + 2 * lane] = fast_exp2(b31 - b0);
-                    gv[GV_D31 + 2 * lane + 1] = fast_exp2(b31 - b1);
-                }
+                compute_gates(gv, a0, a1, be0, be1, lane);
             }
             named_sync(1, 128);
             if (pt == 0) mbar_arrive(&bar[B_GATES + s]);
@@ -636,75 +328,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc_fence_after();
             GDN_TRACE_AT(c, 10, pt == 0);
             {
-                const int r = row & 63;
-                const bool is_a = row < 64;                // A rows: strict lower; P rows: i <= r
-                const bool low = r < 32;                   // warp-uniform
                 float g0[32], g1[32];
                 tmem_ld32(t_row + COL_G, g0);
                 tmem_ld32(t_row + COL_G + 32, g1);
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&bar[B_G_FREE]);
-                float run = is_a ? gv[GV_BETA + r] : 1.f;   // row scale folded into the product
-                if (low) {
-#pragma unroll
-                    for (int x = 31; x >= 0; --x) {
-                        const bool on = x <= r;
-                        const bool keep = is_a ? x < r : on;
-                        const float val = run * g0[x];
-                        g0[x] = keep ? val : 0.f;
-                        run = on ? run * gv[GV_ALPHA + x] : run;
-                    }
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) g1[x] = 0.f;
-                } else {
-#pragma unroll
-                    for (int x = 31; x >= 0; --x) {
-                        const int i = 32 + x;
-                        const bool on = i <= r;
-                        const bool keep = is_a ? i < r : on;
-                        const float val = run * g1[x];
-                        g1[x] = keep ? val : 0.f;
-                        run = on ? run * gv[GV_ALPHA + i] : run;
-                    }
-                    // run = scale * Gam[r][31]
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) g0[x] = run * gv[GV_D31 + x] * g0[x];
-                }
-                if (is_a) {
-                    float4 *dst = reinterpret_cast<float4 *>(sA + r * LDA);
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) dst[x] = make_float4(g0[4 * x], g0[4 * x + 1], g0[4 * x + 2], g0[4 * x + 3]);
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) dst[8 + x] = make_float4(g1[4 * x], g1[4 * x + 1], g1[4 * x + 2], g1[4 * x + 3]);
-                } else {
-                    store_half_row_bf16(sm + OFF_P + s * TILE, r, 0, g0);
-                    store_half_row_bf16(sm + OFF_P + s * TILE, r, 1, g1);
-                }
+                ap_row(gv, row, g0, g1, sA, sm + OFF_P + s * TILE);
             }
             named_sync(1, 128);
             GDN_TRACE_AT(c, 11, pt == 0);
             // ---- T = (I + A)^-1, then Bw = T diag(beta gamma) (threads 0-63, row pt)
             //      and Bu = T diag(beta) (threads 64-127, row pt - 64) as bf16 operands
             unit_lower_inverse(sA, sY, pt, 1);
-            {
-                const int r = pt & 63;
-                unsigned char *dst = sm + (pt < 64 ? OFF_BW : OFF_BU);
-                const float *colscale = gv + (pt < 64 ? GV_BG : GV_BETA);
-#pragma unroll 1
-                for (int hf = 0; hf < 2; ++hf) {
-                    const float4 *trow = reinterpret_cast<const float4 *>(sA + r * LDA + 32 * hf);
-                    const float4 *cs = reinterpret_cast<const float4 *>(colscale + 32 * hf);
-                    float v[32];
-#pragma unroll
-                    for (int x = 0; x < 8; ++x) {
-                        const float4 x4 = trow[x], c4 = cs[x];
-                        v[4 * x] = x4.x * c4.x; v[4 * x + 1] = x4.y * c4.y;
-                        v[4 * x + 2] = x4.z * c4.z; v[4 * x + 3] = x4.w * c4.w;
-                    }
-                    store_half_row_bf16(dst, r, hf, v);
-                }
-            }
+            write_bw_bu(gv, sA, pt, sm + OFF_BW, sm + OFF_BU);
             fence_proxy_async_smem();
             mbar_arrive(&bar[B_SOLVE]);
             GDN_TRACE_AT(c, 12, pt == 0);
@@ -896,40 +533,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
-}
-
-// ------------------------------------------------------------------ host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
-    return fn;
-}
-
-// 4-D map over a [B, T, H, 128] bf16 tensor; box = 64 head-dim x 1 head x 64 tokens x 1.
-bool make_map(CUtensorMap *map, const void *base, int B, int T, int H)
-{
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    const cuuint64_t dims[4] = {(cuuint64_t)kHeadDim, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    const cuuint64_t strides[3] = {(cuuint64_t)kHeadDim * 2, (cuuint64_t)H * kHeadDim * 2,
-                                   (cuuint64_t)T * H * kHeadDim * 2};
-    const cuuint32_t box[4] = {64, 1, (cuuint32_t)C, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
-              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace

@@ -34,6 +34,8 @@ cudaError_t launch_decode(const DecodeArgs &a, gdn_dtype dtype, cudaStream_t str
 cudaError_t launch_chunk_simt(const ChunkArgs &a, gdn_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 bool chunk_tc_available();
+cudaError_t launch_chunk_tc_cluster(const ChunkArgs &a, cudaStream_t stream);
+bool chunk_tc_cluster_fits(int B, int Hv);   // all B * Hv clusters resident at once
 
 // Element conversions used by the kernels.
 __device__ __forceinline__ float to_f32(float x) { return x; }

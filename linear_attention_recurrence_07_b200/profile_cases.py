@@ -1,6 +1,7 @@
 """Runs a few launches of one kernel on one workload, for profiler captures.
 
     python -m linear_attention_recurrence_07_b200.profile_cases prefill [--T 4096] [--launches 3]
+                                                                [--kernel tc|tc_cluster|simt]
     python -m linear_attention_recurrence_07_b200.profile_cases decode [--B 64] [--launches 5]
     python -m linear_attention_recurrence_07_b200.profile_cases prefill-fp32 [--T 1024]
 
@@ -22,7 +23,9 @@ def main():
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto")
     args = ap.parse_args()
+    binding.set_prefill_kernel(args.kernel)
     if args.case in ("prefill", "prefill-fp32"):
         w = inputs.PREFILL_4K if args.case == "prefill" else inputs.PREFILL_SMALL_FP32
         T = args.T or (w.T if args.case == "prefill" else 1024)

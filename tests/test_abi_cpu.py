@@ -33,7 +33,8 @@ def lib():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("gdn_chunk_fwd", "gdn_decode_step", "gdn_status_string", "gdn_last_cuda_error",
-              "gdn_version"):
+              "gdn_version", "gdn_set_prefill_kernel", "gdn_get_prefill_kernel",
+              "gdn_prefill_kernel_for"):
         assert n in names, names
 
 
@@ -109,3 +110,38 @@ def test_binding_raises_on_bad_tensors():
         binding.gdn_chunk_fwd(q.to(torch.float16), q.to(torch.float16), q.to(torch.float16),
                               torch.zeros(1, 4, 1), torch.zeros(1, 4, 1), None,
                               q.to(torch.float16), None)
+
+
+def test_prefill_kernel_selection(lib):
+    assert lib.gdn_get_prefill_kernel() == binding.PREFILL_KERNELS["auto"]
+    for name, code in binding.PREFILL_KERNELS.items():
+        with binding.prefill_kernel(name):
+            assert lib.gdn_get_prefill_kernel() == code
+            assert binding.get_prefill_kernel() == name
+        assert binding.get_prefill_kernel() == "auto"
+    assert lib.gdn_set_prefill_kernel(4) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_set_prefill_kernel(-1) == binding.GDN_ERR_INVALID_ARG
+    assert binding.get_prefill_kernel() == "auto"
+    with pytest.raises(binding.GdnError, match="unknown prefill kernel"):
+        binding.set_prefill_kernel("wgmma")
+    # the tensor-core kernels take bf16 only: fp32 with a forced TC kernel is refused
+    # on the host, before any launch
+    for name in ("tc", "tc_cluster"):
+        with binding.prefill_kernel(name):
+            assert chunk(lib, dtype=0) == binding.GDN_ERR_UNSUPPORTED
+            assert chunk(lib, dtype=0, T=0) == binding.GDN_OK   # nothing to launch
+
+
+def test_prefill_kernel_for_without_device_work(lib):
+    import torch
+    # fp32 never needs the device to decide
+    assert binding.prefill_kernel_for(1, 48, torch.float32) == "simt"
+    with binding.prefill_kernel("simt"):
+        assert binding.prefill_kernel_for(4, 48, torch.bfloat16) == "simt"
+    for name in ("tc", "tc_cluster"):
+        with binding.prefill_kernel(name):
+            with pytest.raises(binding.GdnError, match="no prefill kernel"):
+                binding.prefill_kernel_for(1, 48, torch.float32)
+    assert lib.gdn_prefill_kernel_for(-1, 48, 1) == -1
+    assert lib.gdn_prefill_kernel_for(1, 0, 1) == -1
+    assert lib.gdn_prefill_kernel_for(1, 48, 5) == -1

@@ -40,8 +40,19 @@ def to_dev(d):
     return {k: (None if v is None else v.to(DEV)) for k, v in d.items()}
 
 
-def run_chunk(d, chunk=64):
-    o, S = binding.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], chunk=chunk)
+# Prefill kernels a bf16 input can run on; fp32 inputs always take "simt".
+BF16_KERNELS = ["tc", "tc_cluster", "simt"]
+TC_KERNELS = ["tc", "tc_cluster"]
+
+
+def kernels_for(dtype):
+    return BF16_KERNELS if dtype == torch.bfloat16 else ["simt"]
+
+
+def run_chunk(d, chunk=64, kernel="auto"):
+    with binding.prefill_kernel(kernel):
+        o, S = binding.chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"],
+                                 chunk=chunk)
     torch.cuda.synchronize()
     return o, S
 
@@ -62,22 +73,56 @@ def test_prefill_small_fp32_workload():
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
-@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 100, 191, 256])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 100, 191, 256, 385])
 def test_prefill_ragged_lengths(T, dtype):
+    """1 to 7 chunks with ragged tails: the cluster kernel's two helpers get 0..4
+    chunks each and reuse their receive slots from the third chunk on."""
     d = inputs.prefill_inputs(2, T, 2, 6, dtype=dtype, s0_std=0.5, seed=100 + T)
-    o, S = run_chunk(to_dev(d))
     o_ref, S_ref = oracle_ref(d)
-    check(o, o_ref, tau_for(dtype), f"o T={T}")
-    check(S, S_ref, tau_for(dtype), f"S_final T={T}")
+    dd = to_dev(d)
+    for kernel in kernels_for(dtype):
+        o, S = run_chunk(dd, kernel=kernel)
+        check(o, o_ref, tau_for(dtype), f"{kernel} o T={T}")
+        check(S, S_ref, tau_for(dtype), f"{kernel} S_final T={T}")
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
 def test_prefill_one_v_head_per_qk_head(dtype):
     d = inputs.prefill_inputs(3, 130, 3, 3, dtype=dtype, s0_std=0.1, seed=7)
-    o, S = run_chunk(to_dev(d))
     o_ref, S_ref = oracle_ref(d)
-    check(o, o_ref, tau_for(dtype), "o")
-    check(S, S_ref, tau_for(dtype), "S_final")
+    dd = to_dev(d)
+    for kernel in kernels_for(dtype):
+        o, S = run_chunk(dd, kernel=kernel)
+        check(o, o_ref, tau_for(dtype), f"{kernel} o")
+        check(S, S_ref, tau_for(dtype), f"{kernel} S_final")
+
+
+@pytest.mark.parametrize("kernel", TC_KERNELS)
+def test_prefill_tc_kernels_beyond_one_wave(kernel):
+    """More (sequence, V head) pairs than the GPU holds at once (B=7, Hv=48: 336
+    CTAs, 1008 in clusters): later waves reuse SMs and TMEM of finished ones."""
+    d = to_dev(inputs.prefill_inputs(7, 130, 16, 48, dtype=torch.bfloat16, s0_std=0.1, seed=11))
+    o, S = run_chunk(d, kernel=kernel)
+    o_a, S_a = run_chunk(d, kernel="simt")
+    for b, (h0, h1) in [(0, (0, 3)), (6, (45, 48))]:
+        o_ref, S_ref = oracle_ref({k: (None if v is None else v.cpu()) for k, v in
+                                   _sub_problem(d, b, h0, h1, 48, 16).items()})
+        check(o[b:b + 1, :, h0:h1], o_ref, TAU_BF16, f"{kernel} o b={b} h={h0}:{h1}")
+        check(S[b:b + 1, h0:h1], S_ref, TAU_BF16, f"{kernel} S_final b={b} h={h0}:{h1}")
+    # every pair against the CUDA-core kernel (same inputs, a different evaluation)
+    assert (o.float() - o_a.float()).abs().max().item() <= TAU_BF16 * o_a.float().abs().max().item()
+    assert (S - S_a).abs().max().item() <= TAU_BF16 * S_a.abs().max().item()
+
+
+@pytest.mark.parametrize("B,T,Hqk,Hv,seed", [(1, 385, 2, 6, 21), (2, 4096, 16, 48, 22)])
+def test_prefill_tc_kernels_agree_bitwise(B, T, Hqk, Hv, seed):
+    """The cluster kernel spreads the one-CTA kernel's arithmetic over two CTAs with
+    the same operand values and rounding points: both return the same bits."""
+    d = to_dev(inputs.prefill_inputs(B, T, Hqk, Hv, dtype=torch.bfloat16, s0_std=0.3, seed=seed))
+    o1, S1 = run_chunk(d, kernel="tc")
+    o2, S2 = run_chunk(d, kernel="tc_cluster")
+    assert torch.equal(o1, o2), (o1.float() - o2.float()).abs().max().item()
+    assert torch.equal(S1, S2), (S1 - S2).abs().max().item()
 
 
 def test_prefill_strong_and_no_decay():
@@ -95,13 +140,15 @@ def test_prefill_strong_and_no_decay():
 
 
 def test_prefill_model_dims_workload():
-    """B=1, T=4096, Hqk=16, Hv=48, bf16 inputs, fp32 state: every output checked."""
+    """B=1, T=4096, Hqk=16, Hv=48, bf16 inputs, fp32 state: every output checked,
+    for the default kernel choice and each tensor-core kernel."""
     w = inputs.PREFILL_4K
     d = inputs.workload_inputs(w, device=DEV)
-    o, S = run_chunk(d)
     o_ref, S_ref = oracle_ref(d)
-    check(o, o_ref, TAU_BF16, "o")
-    check(S, S_ref, TAU_BF16, "S_final")
+    for kernel in ["auto"] + TC_KERNELS:
+        o, S = run_chunk(d, kernel=kernel)
+        check(o, o_ref, TAU_BF16, f"{kernel} o")
+        check(S, S_ref, TAU_BF16, f"{kernel} S_final")
 
 
 def _sub_problem(d, b, h0, h1, Hv, Hqk):
@@ -122,11 +169,12 @@ def test_prefill_batched_workload_sampled():
     first and last sequence on the first and last QK group (all their tokens)."""
     w = inputs.PREFILL_BATCH8_8K
     d = inputs.workload_inputs(w, device=DEV)
-    o, S = run_chunk(d)
+    outs = {kernel: run_chunk(d, kernel=kernel) for kernel in ["auto", "tc_cluster"]}
     for b, (h0, h1) in [(0, (0, 3)), (7, (45, 48)), (3, (21, 24))]:
         o_ref, S_ref = oracle_ref(_sub_problem(d, b, h0, h1, w.Hv, w.Hqk))
-        check(o[b:b + 1, :, h0:h1], o_ref, TAU_BF16, f"o b={b} h={h0}:{h1}")
-        check(S[b:b + 1, h0:h1], S_ref, TAU_BF16, f"S_final b={b} h={h0}:{h1}")
+        for kernel, (o, S) in outs.items():
+            check(o[b:b + 1, :, h0:h1], o_ref, TAU_BF16, f"{kernel} o b={b} h={h0}:{h1}")
+            check(S[b:b + 1, h0:h1], S_ref, TAU_BF16, f"{kernel} S_final b={b} h={h0}:{h1}")
 
 
 @pytest.mark.timeout(1800)
@@ -136,11 +184,12 @@ def test_prefill_long_context_workload_sampled():
     measures the drift of the fp32 state carried across 4096 chunks."""
     w = inputs.PREFILL_256K
     d = inputs.workload_inputs(w, device=DEV)
-    o, S = run_chunk(d)
+    outs = {kernel: run_chunk(d, kernel=kernel) for kernel in TC_KERNELS}
     for h in (0, 47):
         o_ref, S_ref = oracle_ref(_sub_problem(d, 0, h, h + 1, w.Hv, w.Hqk))
-        check(o[:, :, h:h + 1], o_ref, TAU_BF16, f"o h={h}")
-        check(S[:, h:h + 1], S_ref, TAU_BF16, f"S_final h={h}")
+        for kernel, (o, S) in outs.items():
+            check(o[:, :, h:h + 1], o_ref, TAU_BF16, f"{kernel} o h={h}")
+            check(S[:, h:h + 1], S_ref, TAU_BF16, f"{kernel} S_final h={h}")
 
 
 def test_prefill_empty_sequence_copies_state():
@@ -165,17 +214,19 @@ def test_prefill_in_place_state():
     assert torch.equal(S, S_ref)
 
 
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
-def test_prefill_split_invariance(dtype):
+@pytest.mark.parametrize("dtype,kernel", [(torch.bfloat16, "tc"), (torch.bfloat16, "tc_cluster"),
+                                          (torch.float32, "simt")],
+                         ids=["bf16-tc", "bf16-tc_cluster", "fp32-simt"])
+def test_prefill_split_invariance(dtype, kernel):
     """T1 tokens, then T2 tokens from the saved state, equals one call over T1+T2."""
     d = to_dev(inputs.prefill_inputs(2, 300, 2, 6, dtype=dtype, s0_std=0.2, seed=5))
-    o, S = run_chunk(d)
+    o, S = run_chunk(d, kernel=kernel)
     T1 = 130
     first = {k: (v[:, :T1].contiguous() if k != "S0" else v) for k, v in d.items()}
     second = {k: (v[:, T1:].contiguous() if k != "S0" else v) for k, v in d.items()}
-    o1, S1 = run_chunk(first)
+    o1, S1 = run_chunk(first, kernel=kernel)
     second["S0"] = S1
-    o2, S2 = run_chunk(second)
+    o2, S2 = run_chunk(second, kernel=kernel)
     scale_o = o.abs().max().item()
     tol = 1e-5 if dtype == torch.float32 else 1e-2
     assert (torch.cat([o1, o2], 1).float() - o.float()).abs().max().item() <= tol * scale_o
