@@ -84,7 +84,7 @@ static_assert(SEND_PV % 16 == 0 && SLOT % 1024 == 0 && WG_BYTES % 1024 == 0 && S
               "bulk copies move 16-byte multiples between 1024-aligned tiles");
 
 // TMEM columns
-constexpr uint32_t COL_S = 0, COL_U = 128, COL_O = 256, COL_W = 384;   // main (2 U, 2 O buffers)
+constexpr uint32_t COL_S = 0, COL_U = 128, COL_O = 256, COL_W = 384;   // main (2 U, 2 O, 2 W buffers)
 constexpr uint32_t MAIN_TMEM = 512;
 constexpr uint32_t HELP_TMEM = 128;                                     // helper: G of each prep WG
 
@@ -277,8 +277,9 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
             // Issues, as soon as their inputs are ready, in this priority order:
             //   YS(c): S^T += U^T K~                         needs bf16 U^T of chunk c
             //   UO(c): U^T += S^T (-W)^T, O^T = S^T Q^T      needs bf16 S^T and W of c
-            //   YO(c): O^T += U^T P^T                        needs the scaled S-part of O^T
             //   WU(c): W^T = K^T Bw^T, U~^T = V^T Bu^T        needs Bu, Bw^T of c
+            //   YO(c): O^T += U^T P^T                        needs the scaled S-part of O^T
+            // W^T and U^T have two TMEM buffers each, by chunk parity.
             if (lane == 0) {
                 int nwu = 0, nuo = 0, nys = 0, nyo = 0;
                 long long idle_since = clock64();
@@ -325,6 +326,27 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                         GDN_TRACE_CL(c, 1, true);
                         ++nuo;
                         issued = true;
+                    } else if (nwu < nchunks &&
+                               mbar_test(&bar[B_BW_READY + nwu % NSLOT], (nwu / NSLOT) & 1) &&
+                               mbar_test(&bar[B_V_FULL], nwu & 1) &&
+                               (nwu < 2 || mbar_test(&bar[B_FIN + (nwu - 2) % NSLOT], ((nwu - 2) / NSLOT) & 1)) &&
+                               (nwu < 2 || mbar_test(&bar[B_UB + (nwu & 1)], ((nwu >> 1) - 1) & 1))) {
+                        const int c = nwu, s = c & 1;
+                        const uint32_t slot = sbase + OFF_SLOT + (c % NSLOT) * SLOT;
+                        tc_fence_after();
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(tmem + COL_W + s * 64, smem_desc_sw128(slot + SL_K + k * 2048, TILE, 1024),
+                                     smem_desc_sw128(slot + SL_BWT + k * 2048, 16, 1024), ID_WT, k > 0);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            mma_bf16(tmem + COL_U + s * 64, smem_desc_sw128(sbase + OFF_V + k * 2048, TILE, 1024),
+                                     smem_desc_sw128(slot + SL_X + k * 32, 16, 1024), ID_UT, k > 0);
+                        mma_commit(&bar[B_W_FULL]);
+                        mma_commit(&bar[B_V_EMPTY]);
+                        GDN_TRACE_CL(c, 0, true);
+                        ++nwu;
+                        issued = true;
                     } else if (nyo < nys && mbar_test(&bar[B_O_READY + (nyo & 1)], (nyo >> 1) & 1)) {
                         const int c = nyo, s = c & 1;
                         const uint32_t slot = sbase + OFF_SLOT + (c % NSLOT) * SLOT;
@@ -336,27 +358,6 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                         mma_commit(&bar[B_O_FULL + s]);
                         GDN_TRACE_CL(c, 3, true);
                         ++nyo;
-                        issued = true;
-                    } else if (nwu < nchunks &&
-                               mbar_test(&bar[B_BW_READY + nwu % NSLOT], (nwu / NSLOT) & 1) &&
-                               mbar_test(&bar[B_V_FULL], nwu & 1) &&
-                               (nwu < 1 || mbar_test(&bar[B_FIN + (nwu - 1) % NSLOT], ((nwu - 1) / NSLOT) & 1)) &&
-                               (nwu < 2 || mbar_test(&bar[B_UB + (nwu & 1)], ((nwu >> 1) - 1) & 1))) {
-                        const int c = nwu, s = c & 1;
-                        const uint32_t slot = sbase + OFF_SLOT + (c % NSLOT) * SLOT;
-                        tc_fence_after();
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_bf16(tmem + COL_W, smem_desc_sw128(slot + SL_K + k * 2048, TILE, 1024),
-                                     smem_desc_sw128(slot + SL_BWT + k * 2048, 16, 1024), ID_WT, k > 0);
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            mma_bf16(tmem + COL_U + s * 64, smem_desc_sw128(sbase + OFF_V + k * 2048, TILE, 1024),
-                                     smem_desc_sw128(slot + SL_X + k * 32, 16, 1024), ID_UT, k > 0);
-                        mma_commit(&bar[B_W_FULL]);
-                        mma_commit(&bar[B_V_EMPTY]);
-                        GDN_TRACE_CL(c, 0, true);
-                        ++nwu;
                         issued = true;
                     }
                     if (issued) {
@@ -558,17 +559,20 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                 GDN_TRACE_CL(c, 11, leader);
                 {
                     float w0[32], w1[32];
-                    tmem_ld32(t_row + COL_W, w0);
-                    tmem_ld32(t_row + COL_W + 32, w1);
+                    tmem_ld32(t_row + COL_W + (c & 1) * 64, w0);
+                    tmem_ld32(t_row + COL_W + (c & 1) * 64 + 32, w1);
                     tmem_wait_ld();
+                    GDN_TRACE_CL(c, 4, leader);
                     store_half_row_bf16(slot + SL_W, lrow, 0, w0);
                     store_half_row_bf16(slot + SL_W, lrow, 1, w1);
                 }
+                GDN_TRACE_CL(c, 15, leader);
                 {
                     const int i = pt >> 1, half = pt & 1;
                     const float gi = reinterpret_cast<const float *>(slot + SL_VEC)[64 + i];
                     scale_row_bf16(slot + SL_K + half * TILE, slot + SL_K + half * TILE, i, gi);
                 }
+                GDN_TRACE_CL(c, 24, leader);
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bar[B_FIN + sl]);
