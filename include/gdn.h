@@ -86,6 +86,31 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
                          gdn_dtype dtype, void *stream);
 
 /*
+ * gdn_chunk_fwd_varlen -- prefill of N sequences of different lengths packed
+ * back to back (continuous batching of prompts of any lengths in one call).
+ *
+ * Defines: gdn_chunk_fwd applied to each sequence on its own.  Use: continuous
+ * batching in serving ("通义千问Qwen3.8-Flash-Next开源：四大架构升级与部署优化全解析",
+ * section "性能表现与开源生态支持").
+ *
+ * In:  q, k [T_total, Hqk, dk]; v [T_total, Hv, dv]; alpha, beta [T_total, Hv];
+ *      cu_seqlens [N + 1] int32 (device): sequence n is token rows
+ *      cu_seqlens[n] .. cu_seqlens[n+1] - 1 (cu_seqlens[0] = 0, nondecreasing,
+ *      cu_seqlens[N] = T_total; offsets are clamped into [0, T_total], so a
+ *      malformed table gives wrong results, never an out-of-bounds access);
+ *      S0 [N, Hv, dk, dv] or NULL (zeros).
+ * Out: o [T_total, Hv, dv]; S_final [N, Hv, dk, dv] or NULL (may be S0).  An
+ *      empty sequence copies its S0 (or zeros) to S_final.
+ * Sizes, dtypes, alignment and kernel choice as for gdn_chunk_fwd, with
+ *      N in place of B (N <= 65535); cu_seqlens must be 4-byte aligned.
+ */
+gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                                const float *alpha, const float *beta, const float *S0,
+                                void *o, float *S_final, const int *cu_seqlens,
+                                int N, int T_total, int Hqk, int Hv, int dk, int dv, int chunk,
+                                gdn_dtype dtype, void *stream);
+
+/*
  * gdn_decode_step -- one token for each of B sequences (autoregressive decode).
  *
  * Defines: the first form of the update in section 2.1 "Gated DeltaNet",
@@ -102,6 +127,56 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
                            void *o, float *S_new,
                            int B, int Hqk, int Hv, int dk, int dv,
                            gdn_dtype dtype, void *stream);
+
+/*
+ * gdn_decode_tokens -- n tokens per sequence in one call (multi-token decode and
+ * verification of speculative drafts), with the state after every token kept
+ * for rollback.
+ *
+ * Defines: the update of gdn_decode_step applied to tokens 0 .. n-1 in order.
+ * Use: "Qwen3.8-Flash-Next 技术总结 -- Qwen4 架构的探路者", section 2.5 (MTP):
+ * the multi-token prediction head drafts several tokens per step for
+ * speculative decoding, and the backbone checks them in one pass.  If only
+ * the first m drafts are accepted, the state to continue from is S_steps[:, m-1].
+ *
+ * In:  q, k [B, n, Hqk, dk]; v [B, n, Hv, dv]; alpha, beta [B, n, Hv];
+ *      S [B, Hv, dk, dv].
+ * Out: o [B, n, Hv, dv], o_t read after token t's update;
+ *      S_new [B, Hv, dk, dv], the state after token n-1 (may be S itself);
+ *      S_steps [B, n, Hv, dk, dv] or NULL, the state after every token
+ *      (it must not overlap S or S_new).
+ * Sizes: B >= 0, 1 <= n <= 64 (n > 64: GDN_ERR_UNSUPPORTED), heads as for
+ *      gdn_decode_step.  n == 1 with S_steps == NULL is gdn_decode_step.
+ */
+gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta, const float *S,
+                             void *o, float *S_new, float *S_steps,
+                             int B, int n, int Hqk, int Hv, int dk, int dv,
+                             gdn_dtype dtype, void *stream);
+
+/*
+ * gdn_decode_step_slots -- one decode token for B sequences whose states live
+ * in a shared pool, updated in place (continuous batching: the sequences of a
+ * step are any subset of the pool, in any order).
+ *
+ * Defines: the update of gdn_decode_step, with sequence b's state at
+ * state_pool[slots[b]].  Use: continuous batching in serving
+ * ("通义千问Qwen3.8-Flash-Next开源：四大架构升级与部署优化全解析", section
+ * "性能表现与开源生态支持").
+ *
+ * In:  q, k [B, Hqk, dk]; v [B, Hv, dv]; alpha, beta [B, Hv];
+ *      slots [B] int32 (device); state_pool [n_slots, Hv, dk, dv] fp32.
+ * Out: o [B, Hv, dv]; state_pool[slots[b]] updated in place.
+ * A slot outside [0, n_slots) marks a padding entry: sequence b is skipped, its
+ * o row is left as it was and no state changes.  Two entries with the same slot
+ * race (undefined result).  slots must be 4-byte aligned; the other pointers
+ * 16-byte aligned.
+ */
+gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v,
+                                 const float *alpha, const float *beta,
+                                 float *state_pool, const int *slots, void *o,
+                                 int B, int n_slots, int Hqk, int Hv, int dk, int dv,
+                                 gdn_dtype dtype, void *stream);
 
 /*
  * Prefill kernel selection (library-specific: the page describes the method,

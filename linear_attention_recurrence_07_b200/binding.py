@@ -48,6 +48,15 @@ def library():
         lib.gdn_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
                                         I, I, I, I, I, I, vp]
         lib.gdn_decode_step.restype = I
+        lib.gdn_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp,
+                                             I, I, I, I, I, I, I, I, vp]
+        lib.gdn_chunk_fwd_varlen.restype = I
+        lib.gdn_decode_tokens.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp,
+                                          I, I, I, I, I, I, I, vp]
+        lib.gdn_decode_tokens.restype = I
+        lib.gdn_decode_step_slots.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp,
+                                              I, I, I, I, I, I, I, vp]
+        lib.gdn_decode_step_slots.restype = I
         lib.gdn_status_string.argtypes = [I]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_last_cuda_error.argtypes = []
@@ -183,6 +192,81 @@ def prefill_kernel(name):
         yield
     finally:
         set_prefill_kernel(prev)
+
+
+def gdn_chunk_fwd_varlen(q, k, v, alpha, beta, S0, o, S_final, cu_seqlens, chunk=64,
+                         stream=None):
+    """Prefill of N packed sequences (C entry point ``gdn_chunk_fwd_varlen``).  q, k
+    [T_total, Hqk, dk] and v, o [T_total, Hv, dv] (float32 or bfloat16); alpha,
+    beta [T_total, Hv] float32; cu_seqlens [N + 1] int32; S0, S_final
+    [N, Hv, dk, dv] float32 or None."""
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    N = cu_seqlens.shape[0] - 1
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (T, Hv, dv), q.dtype),
+                               ("o", o, (T, Hv, dv), q.dtype),
+                               ("alpha", alpha, (T, Hv), torch.float32),
+                               ("beta", beta, (T, Hv), torch.float32),
+                               ("cu_seqlens", cu_seqlens, (N + 1,), torch.int32)):
+        _expect(t, name, shape, dt, dev)
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None:
+            _expect(t, name, (N, Hv, dk, dv), torch.float32, dev)
+    _check(library().gdn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                          _ptr(S0), _ptr(o), _ptr(S_final), _ptr(cu_seqlens),
+                                          N, T, Hqk, Hv, dk, dv, chunk, _DTYPES[q.dtype],
+                                          _stream_handle(stream, dev)),
+           "gdn_chunk_fwd_varlen")
+
+
+def gdn_decode_tokens(q, k, v, alpha, beta, S, o, S_new, S_steps=None, stream=None):
+    """n decode tokens per sequence (C entry point ``gdn_decode_tokens``); writes o,
+    S_new (may be S itself) and, if given, S_steps.  q, k [B, n, Hqk, dk]; v, o
+    [B, n, Hv, dv]; alpha, beta [B, n, Hv] float32; S, S_new [B, Hv, dk, dv]
+    float32; S_steps [B, n, Hv, dk, dv] float32 or None."""
+    B, n, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, n, Hv, dv), q.dtype),
+                               ("o", o, (B, n, Hv, dv), q.dtype),
+                               ("alpha", alpha, (B, n, Hv), torch.float32),
+                               ("beta", beta, (B, n, Hv), torch.float32),
+                               ("S", S, (B, Hv, dk, dv), torch.float32),
+                               ("S_new", S_new, (B, Hv, dk, dv), torch.float32)):
+        _expect(t, name, shape, dt, dev)
+    if S_steps is not None:
+        _expect(S_steps, "S_steps", (B, n, Hv, dk, dv), torch.float32, dev)
+    _check(library().gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+                                       _ptr(o), _ptr(S_new), _ptr(S_steps), B, n, Hqk, Hv, dk, dv,
+                                       _DTYPES[q.dtype], _stream_handle(stream, dev)),
+           "gdn_decode_tokens")
+
+
+def gdn_decode_step_slots(q, k, v, alpha, beta, state_pool, slots, o, stream=None):
+    """One decode token per sequence with states in a pool (C entry point
+    ``gdn_decode_step_slots``): state_pool[slots[b]] is updated in place.  q, k
+    [B, Hqk, dk]; v, o [B, Hv, dv]; alpha, beta [B, Hv] float32; state_pool
+    [n_slots, Hv, dk, dv] float32; slots [B] int32."""
+    B, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    n_slots = state_pool.shape[0]
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, Hv, dv), q.dtype),
+                               ("o", o, (B, Hv, dv), q.dtype),
+                               ("alpha", alpha, (B, Hv), torch.float32),
+                               ("beta", beta, (B, Hv), torch.float32),
+                               ("state_pool", state_pool, (n_slots, Hv, dk, dv), torch.float32),
+                               ("slots", slots, (B,), torch.int32)):
+        _expect(t, name, shape, dt, dev)
+    _check(library().gdn_decode_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                           _ptr(state_pool), _ptr(slots), _ptr(o), B, n_slots,
+                                           Hqk, Hv, dk, dv, _DTYPES[q.dtype],
+                                           _stream_handle(stream, dev)),
+           "gdn_decode_step_slots")
 
 
 def chunk_fwd(q, k, v, alpha, beta, S0=None, chunk=64, stream=None):

@@ -8,6 +8,7 @@
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+constexpr int kMaxDecodeTokens = 64;   // gdn_decode_tokens: tokens per call
 std::atomic<int> g_prefill_kernel{GDN_PREFILL_AUTO};   // process-wide prefill kernel choice
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -48,15 +49,13 @@ int resolve_prefill_kernel(int B, int Hv, gdn_dtype dtype)
     return kind;
 }
 
-}  // namespace
-
-extern "C" {
-
-gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
-                         const float *alpha, const float *beta, const float *S0,
-                         void *o, float *S_final,
-                         int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
-                         gdn_dtype dtype, void *stream)
+// Shared by the two prefill entry points: B sequences of T tokens each, or, with
+// cu_seqlens, B packed sequences in T token rows.
+gdn_status chunk_fwd_common(const void *q, const void *k, const void *v,
+                            const float *alpha, const float *beta, const float *S0,
+                            void *o, float *S_final, const int *cu_seqlens,
+                            int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                            gdn_dtype dtype, void *stream)
 {
     if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
@@ -67,7 +66,7 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
     if (B == 0) return GDN_OK;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t state_bytes = (size_t)B * Hv * dk * dv * sizeof(float);
-    if (T == 0) {
+    if (T == 0) {   // every sequence is empty: the state passes through
         if (!S_final) return GDN_OK;
         if (!aligned16(S_final) || (S0 && !aligned16(S0))) return GDN_ERR_INVALID_ARG;
         if (S0 == S_final) return GDN_OK;
@@ -80,6 +79,7 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
         if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
 
     gdn::ChunkArgs a{q, k, v, alpha, beta, S0, o, S_final, B, T, Hqk, Hv};
+    a.cu_seqlens = cu_seqlens;
     const int kind = resolve_prefill_kernel(B, Hv, dtype);
     if (kind < 0) return GDN_ERR_UNSUPPORTED;
     cudaError_t err;
@@ -89,6 +89,32 @@ gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
     default: err = gdn::launch_chunk_simt(a, dtype, s); break;
     }
     return cuda_status(err);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_chunk_fwd(const void *q, const void *k, const void *v,
+                         const float *alpha, const float *beta, const float *S0,
+                         void *o, float *S_final,
+                         int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                         gdn_dtype dtype, void *stream)
+{
+    return chunk_fwd_common(q, k, v, alpha, beta, S0, o, S_final, nullptr, B, T, Hqk, Hv, dk, dv,
+                            chunk, dtype, stream);
+}
+
+gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
+                                const float *alpha, const float *beta, const float *S0,
+                                void *o, float *S_final, const int *cu_seqlens,
+                                int N, int T_total, int Hqk, int Hv, int dk, int dv, int chunk,
+                                gdn_dtype dtype, void *stream)
+{
+    if (N > 0 && T_total > 0 && (!cu_seqlens || (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u)))
+        return GDN_ERR_INVALID_ARG;
+    return chunk_fwd_common(q, k, v, alpha, beta, S0, o, S_final, cu_seqlens, N, T_total, Hqk, Hv,
+                            dk, dv, chunk, dtype, stream);
 }
 
 gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
@@ -128,6 +154,53 @@ int gdn_prefill_kernel_for(int B, int Hv, gdn_dtype dtype)
 {
     if (B < 0 || Hv <= 0 || (dtype != GDN_F32 && dtype != GDN_BF16)) return -1;
     return resolve_prefill_kernel(B, Hv, dtype);
+}
+
+gdn_status gdn_decode_tokens(const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta, const float *S,
+                             void *o, float *S_new, float *S_steps,
+                             int B, int n, int Hqk, int Hv, int dk, int dv,
+                             gdn_dtype dtype, void *stream)
+{
+    if (B < 0 || n < 1) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_heads(Hqk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (n > kMaxDecodeTokens) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if ((long long)B * Hv > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !S || !o || !S_new) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, beta, S, o, S_new, S_steps};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    gdn::DecodeArgs a{q, k, v, alpha, beta, S, o, S_new, B, Hqk, Hv};
+    a.ntok = n;
+    a.S_steps = S_steps;
+    return cuda_status(gdn::launch_decode(a, dtype, static_cast<cudaStream_t>(stream)));
+}
+
+gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v,
+                                 const float *alpha, const float *beta,
+                                 float *state_pool, const int *slots, void *o,
+                                 int B, int n_slots, int Hqk, int Hv, int dk, int dv,
+                                 gdn_dtype dtype, void *stream)
+{
+    if (B < 0 || n_slots < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_heads(Hqk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (B == 0) return GDN_OK;
+    if ((long long)B * Hv > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !slots || !o || (n_slots > 0 && !state_pool))
+        return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, beta, state_pool, o};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(slots) & 3u) return GDN_ERR_INVALID_ARG;
+    gdn::DecodeArgs a{q, k, v, alpha, beta, state_pool, o, state_pool, B, Hqk, Hv};
+    a.slots = slots;
+    a.n_slots = n_slots;
+    return cuda_status(gdn::launch_decode(a, dtype, static_cast<cudaStream_t>(stream)));
 }
 
 const char *gdn_status_string(gdn_status status)

@@ -45,7 +45,8 @@ template <typename T>
 __global__ void __launch_bounds__(NT, 1)
 chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                   const float *__restrict__ alpha, const float *__restrict__ beta,
-                  const float *S0, T *__restrict__ o, float *S_final, int Tlen, int Hqk, int Hv)
+                  const float *S0, T *__restrict__ o, float *S_final, int Tlen, int Hqk, int Hv,
+                  const int *__restrict__ cu_seqlens)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
@@ -56,6 +57,14 @@ chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     const int hq = h / (Hv / Hqk);
     const int j_base = slice * DVS;
     const int tid = threadIdx.x;
+    // token rows of this sequence: [bt * Tlen + tb, ... + Lseq) of the token arrays
+    int tb = 0, Lseq = Tlen, bt = b;
+    if (cu_seqlens) {   // packed sequences; offsets clamped into [0, Tlen]
+        const int s0 = min(max(cu_seqlens[b], 0), Tlen);
+        tb = s0;
+        Lseq = min(max(cu_seqlens[b + 1], s0), Tlen) - s0;
+        bt = 0;
+    }
 
     // ---- initial state slice
     const size_t s_off = ((size_t)b * Hv + h) * D * kHeadDim;
@@ -69,8 +78,8 @@ chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     const int c0 = (tid % 16) * 4;     // 4 columns
     const int d0 = (tid / 16) * 8;     // 8 state rows of the 128 x 64 state update
 
-    for (int t0 = 0; t0 < Tlen; t0 += C) {
-        const int L = min(C, Tlen - t0);
+    for (int t0 = 0; t0 < Lseq; t0 += C) {
+        const int L = min(C, Lseq - t0);
         __syncthreads();  // previous chunk fully consumed
 
         // ---- load the chunk (transposed K, Q; V slice), padding rows >= L
@@ -78,7 +87,7 @@ chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
             const int r = e / D, d = e % D;
             float kv = 0.f, qv = 0.f;
             if (r < L) {
-                const size_t off = (((size_t)b * Tlen + t0 + r) * Hqk + hq) * D + d;
+                const size_t off = (((size_t)bt * Tlen + tb + t0 + r) * Hqk + hq) * D + d;
                 kv = to_f32(k[off]);
                 qv = to_f32(q[off]);
             }
@@ -87,7 +96,7 @@ chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
         }
         for (int e = tid; e < C * DVS; e += NT) {
             const int r = e / DVS, j = e % DVS;
-            sm.U[r][j] = r < L ? to_f32(v[(((size_t)b * Tlen + t0 + r) * Hv + h) * kHeadDim + j_base + j]) : 0.f;
+            sm.U[r][j] = r < L ? to_f32(v[(((size_t)bt * Tlen + tb + t0 + r) * Hv + h) * kHeadDim + j_base + j]) : 0.f;
         }
         if (tid < 32) {  // gates and the chunk-local cumulative log decay (warp scan)
             const int lane = tid;
@@ -95,7 +104,7 @@ chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 const int r = 2 * lane + x;
-                const size_t g = ((size_t)b * Tlen + t0 + r) * Hv + h;
+                const size_t g = ((size_t)bt * Tlen + tb + t0 + r) * Hv + h;
                 la[x] = r < L ? clamped_log(alpha[g]) : 0.f;
                 be[x] = r < L ? beta[g] : 0.f;
             }
@@ -226,7 +235,7 @@ chunk_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
             for (int x = 0; x < 4; ++x) {
                 const int r = r0 + x;
                 if (r < L) {
-                    T *dst = o + (((size_t)b * Tlen + t0 + r) * Hv + h) * kHeadDim + j_base + c0;
+                    T *dst = o + (((size_t)bt * Tlen + tb + t0 + r) * Hv + h) * kHeadDim + j_base + c0;
 #pragma unroll
                     for (int y = 0; y < 4; ++y) dst[y] = from_f32<T>(acc[x][y]);
                 }
@@ -278,7 +287,7 @@ cudaError_t launch_typed(const ChunkArgs &a, cudaStream_t stream)
     const dim3 grid((unsigned)(a.Hv * (kHeadDim / DVS)), (unsigned)a.B);
     chunk_simt_kernel<T><<<grid, NT, smem, stream>>>(
         (const T *)a.q, (const T *)a.k, (const T *)a.v, a.alpha, a.beta, a.S0, (T *)a.o,
-        a.S_final, a.T, a.Hqk, a.Hv);
+        a.S_final, a.T, a.Hqk, a.Hv, a.cu_seqlens);
     return cudaGetLastError();
 }
 

@@ -118,8 +118,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x, b = blockIdx.y;
     const int hq = h / (p.Hv / p.Hqk);
-    const int T = p.T;
-    const int nchunks = (T + C - 1) / C;
+    const SeqSpan sq = seq_span(p, b);           // this sequence's token rows
+    const int nchunks = (sq.L + C - 1) / C;
     const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
@@ -151,21 +151,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             bool ok = true;
             int issued_kq0 = -1, issued_kq1 = -1, issued_v = -1;
             for (int c = 0; c < nchunks && ok; ++c) {
-                const int s = c & 1, t0 = c * C;
+                const int s = c & 1, t0 = sq.tb + c * C;
                 if (c >= 2) ok = ctl.wait(B_KQ_EMPTY + s, ((c >> 1) - 1) & 1);
                 if (!ok) break;
                 unsigned char *st = sm + OFF_KQ + s * KQ_STAGE;
                 mbar_arrive_expect_tx(&bar[B_KQ_FULL + s], KQ_STAGE);
-                tma_load_4d(st + 0 * TILE, &tm_k, &bar[B_KQ_FULL + s], 0, hq, t0, b);
-                tma_load_4d(st + 1 * TILE, &tm_q, &bar[B_KQ_FULL + s], 0, hq, t0, b);
-                tma_load_4d(st + 2 * TILE, &tm_k, &bar[B_KQ_FULL + s], 64, hq, t0, b);
-                tma_load_4d(st + 3 * TILE, &tm_q, &bar[B_KQ_FULL + s], 64, hq, t0, b);
+                tma_load_4d(st + 0 * TILE, &tm_k, &bar[B_KQ_FULL + s], 0, hq, t0, sq.bt);
+                tma_load_4d(st + 1 * TILE, &tm_q, &bar[B_KQ_FULL + s], 0, hq, t0, sq.bt);
+                tma_load_4d(st + 2 * TILE, &tm_k, &bar[B_KQ_FULL + s], 64, hq, t0, sq.bt);
+                tma_load_4d(st + 3 * TILE, &tm_q, &bar[B_KQ_FULL + s], 64, hq, t0, sq.bt);
                 if (s) issued_kq1 = c; else issued_kq0 = c;
                 if (c >= 1) ok = ctl.wait(B_V_EMPTY, (c - 1) & 1);
                 if (!ok) break;
                 mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * TILE);
-                tma_load_4d(sm + OFF_V, &tm_v, &bar[B_V_FULL], 0, h, t0, b);
-                tma_load_4d(sm + OFF_V + TILE, &tm_v, &bar[B_V_FULL], 64, h, t0, b);
+                tma_load_4d(sm + OFF_V, &tm_v, &bar[B_V_FULL], 0, h, t0, sq.bt);
+                tma_load_4d(sm + OFF_V + TILE, &tm_v, &bar[B_V_FULL], 64, h, t0, sq.bt);
                 issued_v = c;
             }
             if (*abort_flag) {
@@ -297,7 +297,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         // gate prefetch (warp 2): alpha, beta of the next chunk are in flight while
         // the current chunk is prepared
         float nx_a0 = 1.f, nx_a1 = 1.f, nx_b0 = 0.f, nx_b1 = 0.f;
-        if (warp == 2 && nchunks > 0) load_gates(p, b, h, T, 0, lane, nx_a0, nx_a1, nx_b0, nx_b1);
+        if (warp == 2 && nchunks > 0) load_gates(p, sq, h, 0, lane, nx_a0, nx_a1, nx_b0, nx_b1);
         for (int c = 0; c < nchunks && ok; ++c) {
             const int s = c & 1;
             float *gv = reinterpret_cast<float *>(sm + OFF_GATE + s * GATE_BUF);
@@ -310,7 +310,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             //      padded rows carry alpha = 1, beta = 0 (neutral)
             if (warp == 2) {
                 const float a0 = nx_a0, a1 = nx_a1, be0 = nx_b0, be1 = nx_b1;
-                if (c + 1 < nchunks) load_gates(p, b, h, T, c + 1, lane, nx_a0, nx_a1, nx_b0, nx_b1);
+                if (c + 1 < nchunks) load_gates(p, sq, h, c + 1, lane, nx_a0, nx_a1, nx_b0, nx_b1);
                 compute_gates(gv, a0, a1, be0, be1, lane);
             }
             named_sync(1, 128);
@@ -390,6 +390,28 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             tmem_wait_st();
         }
+        // Staged O^T of chunk cp (bf16 tile [r][j] at OFF_U) -> o: one TMA store,
+        // except for the last chunk of a packed sequence that ends inside it,
+        // whose rows past the end belong to the next sequence: its rows are
+        // stored one by one (rows past the array's end are clipped by the TMA).
+        auto store_staged_o = [&](int cp, bool wait_read) {
+            const int rows = min(C, sq.L - cp * C);
+            if (p.cu_seqlens && rows < C) {
+                const size_t row_stride = (size_t)p.Hv * kHeadDim;
+                const unsigned char *ot = sm + OFF_U + (j >> 6) * TILE;
+                __nv_bfloat16 *dst = p.o + ((size_t)sq.bt * p.T + sq.tb + (size_t)cp * C) * row_stride +
+                                     (size_t)h * kHeadDim + j;
+#pragma unroll 1
+                for (int r = 0; r < rows; ++r)
+                    dst[(size_t)r * row_stride] =
+                        *reinterpret_cast<const __nv_bfloat16 *>(ot + sw128_offset(r, j & 63));
+            } else if (leader) {
+                tma_store_4d(&tm_o, sm + OFF_U, 0, h, sq.tb + cp * C, sq.bt);
+                tma_store_4d(&tm_o, sm + OFF_U + TILE, 64, h, sq.tb + cp * C, sq.bt);
+                bulk_commit_group();
+                if (wait_read) bulk_wait_group_read0();
+            }
+        };
         for (int c = 0; c < nchunks && ok; ++c) {
             const int s = c & 1;
             GDN_TRACE_AT(c, 16, leader);
@@ -442,12 +464,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 mbar_arrive(&bar[B_O_FREE + (cp & 1)]);
                 fence_proxy_async_smem();
                 named_sync(2, 128);
-                if (leader) {
-                    tma_store_4d(&tm_o, sm + OFF_U, 0, h, cp * C, b);
-                    tma_store_4d(&tm_o, sm + OFF_U + TILE, 64, h, cp * C, b);
-                    bulk_commit_group();
-                    bulk_wait_group_read0();   // staging must be read before U^T reuses it
-                }
+                store_staged_o(cp, true);      // staging must be read before U^T reuses it
             }
             GDN_TRACE_AT(c, 19, leader);
             // U^T -> bf16 operand
@@ -506,11 +523,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
                 fence_proxy_async_smem();
                 named_sync(2, 128);
-                if (leader) {
-                    tma_store_4d(&tm_o, sm + OFF_U, 0, h, cp * C, b);
-                    tma_store_4d(&tm_o, sm + OFF_U + TILE, 64, h, cp * C, b);
-                    bulk_commit_group();
-                }
+                store_staged_o(cp, false);
             }
         }
         if (ok && p.S_final) {
@@ -551,14 +564,16 @@ extern "C" int gdn_trace_read(unsigned long long *host, int n)
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
 {
     CUtensorMap tk, tq, tv, to;
-    if (!make_map(&tk, a.k, a.B, a.T, a.Hqk) || !make_map(&tq, a.q, a.B, a.T, a.Hqk) ||
-        !make_map(&tv, a.v, a.B, a.T, a.Hv) || !make_map(&to, a.o, a.B, a.T, a.Hv))
+    const int rows_b = a.cu_seqlens ? 1 : a.B;   // batch rows of the token arrays
+    if (!make_map(&tk, a.k, rows_b, a.T, a.Hqk) || !make_map(&tq, a.q, rows_b, a.T, a.Hqk) ||
+        !make_map(&tv, a.v, rows_b, a.T, a.Hv) || !make_map(&to, a.o, rows_b, a.T, a.Hv))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(chunk_tc_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
-    TcParams p{a.alpha, a.beta, a.S0, a.S_final, a.T, a.Hqk, a.Hv};
+    TcParams p{a.alpha, a.beta, a.S0, a.S_final, a.T, a.Hqk, a.Hv,
+               static_cast<__nv_bfloat16 *>(a.o), a.cu_seqlens};
     chunk_tc_kernel<<<dim3((unsigned)a.Hv, (unsigned)a.B), NT, SMEM_BYTES, stream>>>(tk, tq, tv, to, p);
     return cudaGetLastError();
 }

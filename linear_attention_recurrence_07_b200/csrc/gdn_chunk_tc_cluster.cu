@@ -218,8 +218,8 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
     const uint32_t rank = cluster_rank();
     const int h = blockIdx.x / CLUSTER, b = blockIdx.y;
     const int hq = h / (p.Hv / p.Hqk);
-    const int T = p.T;
-    const int nchunks = (T + C - 1) / C;
+    const SeqSpan sq = seq_span(p, b);           // this sequence's token rows
+    const int nchunks = (sq.L + C - 1) / C;
     const uint32_t sbase = smem_u32(sm);
     const bool is_main = (rank == 0);
     const uint32_t tmem_cols = is_main ? MAIN_TMEM : HELP_TMEM;
@@ -250,19 +250,19 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                 bool ok = true;
                 int issued_q0 = -1, issued_q1 = -1, issued_v = -1;
                 for (int c = 0; c < nchunks && ok; ++c) {
-                    const int s = c & 1, t0 = c * C;
+                    const int s = c & 1, t0 = sq.tb + c * C;
                     if (c >= 2) ok = ctl.wait(B_Q_EMPTY + s, ((c >> 1) - 1) & 1);
                     if (!ok) break;
                     unsigned char *qd = sm + OFF_Q + s * Q_STAGE;
                     mbar_arrive_expect_tx(&bar[B_Q_FULL + s], Q_STAGE);
-                    tma_load_4d(qd, &tm_q, &bar[B_Q_FULL + s], 0, hq, t0, b);
-                    tma_load_4d(qd + TILE, &tm_q, &bar[B_Q_FULL + s], 64, hq, t0, b);
+                    tma_load_4d(qd, &tm_q, &bar[B_Q_FULL + s], 0, hq, t0, sq.bt);
+                    tma_load_4d(qd + TILE, &tm_q, &bar[B_Q_FULL + s], 64, hq, t0, sq.bt);
                     if (s) issued_q1 = c; else issued_q0 = c;
                     if (c >= 1) ok = ctl.wait(B_V_EMPTY, (c - 1) & 1);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * TILE);
-                    tma_load_4d(sm + OFF_V, &tm_v, &bar[B_V_FULL], 0, h, t0, b);
-                    tma_load_4d(sm + OFF_V + TILE, &tm_v, &bar[B_V_FULL], 64, h, t0, b);
+                    tma_load_4d(sm + OFF_V, &tm_v, &bar[B_V_FULL], 0, h, t0, sq.bt);
+                    tma_load_4d(sm + OFF_V + TILE, &tm_v, &bar[B_V_FULL], 64, h, t0, sq.bt);
                     issued_v = c;
                 }
                 if (*abort_flag) {
@@ -470,8 +470,8 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                 mbar_arrive(&bar[B_O_READY + s]);
                 GDN_TRACE_CL(c, 10, leader);
             }
-            if (ok && nchunks > 0) {
-                ok = named_and(2, 128, ctl.wait(B_S_FULL, (nchunks - 1) & 1));
+            if (ok && nchunks > 0) ok = named_and(2, 128, ctl.wait(B_S_FULL, (nchunks - 1) & 1));
+            {   // an empty sequence passes S0 (in TMEM since the start) through
                 if (ok && p.S_final) {
                     tc_fence_after();
                     float *dst = p.S_final + ((size_t)b * p.Hv + h) * kHeadDim * kHeadDim;
@@ -513,8 +513,8 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                 const int sl = cn % NSLOT;
                 unsigned char *kd = sm + OFF_SLOT + sl * SLOT + SL_K;
                 mbar_arrive_expect_tx(&bar[B_RECV + sl], K_BYTES);
-                tma_load_4d(kd, &tm_k, &bar[B_RECV + sl], 0, hq, cn * C, b);
-                tma_load_4d(kd + TILE, &tm_k, &bar[B_RECV + sl], 64, hq, cn * C, b);
+                tma_load_4d(kd, &tm_k, &bar[B_RECV + sl], 0, hq, sq.tb + cn * C, sq.bt);
+                tma_load_4d(kd + TILE, &tm_k, &bar[B_RECV + sl], 64, hq, sq.tb + cn * C, sq.bt);
                 issued_k = cn + 1;
             };
             // Chunk cp is done once its O MMAs complete: every MMA reading its slot
@@ -530,9 +530,9 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                     remote_arrive(map_to_rank(smem_u32(&bar[B_SLOT_FREE + sl]), 1));
                 }
                 const uint32_t col_o = COL_O + (cp & 1) * 64;
-                const int rows = min(C, T - cp * C);
+                const int rows = min(C, sq.L - cp * C);
                 const size_t row_stride = (size_t)p.Hv * kHeadDim;
-                __nv_bfloat16 *dst = p.o + ((size_t)b * T + (size_t)cp * C) * row_stride +
+                __nv_bfloat16 *dst = p.o + ((size_t)sq.bt * p.T + sq.tb + (size_t)cp * C) * row_stride +
                                      (size_t)h * kHeadDim + lrow;
                 float ov[64];
                 tmem_ld32(t_row + col_o, ov);
@@ -597,15 +597,15 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
                 bool ok = true;
                 int issued = 0;
                 for (int c = 0; c < nchunks && ok; ++c) {
-                    const int st = c % NSTAGE, n = c / NSTAGE, t0 = c * C;
+                    const int st = c % NSTAGE, n = c / NSTAGE, t0 = sq.tb + c * C;
                     if (n >= 1) ok = ctl.wait(B_KQ_EMPTY + st, (n - 1) & 1);
                     if (!ok) break;
                     unsigned char *dst = sm + H_OFF_KQ + st * KQ_STAGE;
                     mbar_arrive_expect_tx(&bar[B_KQ_FULL + st], KQ_STAGE);
-                    tma_load_4d(dst + 0 * TILE, &tm_k, &bar[B_KQ_FULL + st], 0, hq, t0, b);
-                    tma_load_4d(dst + 1 * TILE, &tm_q, &bar[B_KQ_FULL + st], 0, hq, t0, b);
-                    tma_load_4d(dst + 2 * TILE, &tm_k, &bar[B_KQ_FULL + st], 64, hq, t0, b);
-                    tma_load_4d(dst + 3 * TILE, &tm_q, &bar[B_KQ_FULL + st], 64, hq, t0, b);
+                    tma_load_4d(dst + 0 * TILE, &tm_k, &bar[B_KQ_FULL + st], 0, hq, t0, sq.bt);
+                    tma_load_4d(dst + 1 * TILE, &tm_q, &bar[B_KQ_FULL + st], 0, hq, t0, sq.bt);
+                    tma_load_4d(dst + 2 * TILE, &tm_k, &bar[B_KQ_FULL + st], 64, hq, t0, sq.bt);
+                    tma_load_4d(dst + 3 * TILE, &tm_q, &bar[B_KQ_FULL + st], 64, hq, t0, sq.bt);
                     issued = c + 1;
                     GDN_TRACE_CL(c, 22, true);
                 }
@@ -659,12 +659,12 @@ chunk_tc_cluster_kernel(const __grid_constant__ CUtensorMap tm_k,
             bool ok = true;
             float nx_a0 = 1.f, nx_a1 = 1.f, nx_b0 = 0.f, nx_b1 = 0.f;
             if (warp == lead_warp && wg < nchunks)
-                load_gates(p, b, h, T, wg, lane, nx_a0, nx_a1, nx_b0, nx_b1);
+                load_gates(p, sq, h, wg, lane, nx_a0, nx_a1, nx_b0, nx_b1);
             for (int c = wg, n = 0; c < nchunks && ok; c += 2, ++n) {
                 GDN_TRACE_CL(c, 16, pt == 0);
                 if (warp == lead_warp) {
                     const float a0 = nx_a0, a1 = nx_a1, be0 = nx_b0, be1 = nx_b1;
-                    if (c + 2 < nchunks) load_gates(p, b, h, T, c + 2, lane, nx_a0, nx_a1, nx_b0, nx_b1);
+                    if (c + 2 < nchunks) load_gates(p, sq, h, c + 2, lane, nx_a0, nx_a1, nx_b0, nx_b1);
                     compute_gates(gv, a0, a1, be0, be1, lane);
                 }
                 if (pt == 0) bulk_wait_group_read0();   // the previous chunk's copies read the staging
@@ -781,15 +781,16 @@ bool chunk_tc_cluster_fits(int B, int Hv)
 cudaError_t launch_chunk_tc_cluster(const ChunkArgs &a, cudaStream_t stream)
 {
     CUtensorMap tk, tq, tv;
-    if (!make_map(&tk, a.k, a.B, a.T, a.Hqk) || !make_map(&tq, a.q, a.B, a.T, a.Hqk) ||
-        !make_map(&tv, a.v, a.B, a.T, a.Hv))
+    const int rows_b = a.cu_seqlens ? 1 : a.B;   // batch rows of the token arrays
+    if (!make_map(&tk, a.k, rows_b, a.T, a.Hqk) || !make_map(&tq, a.q, rows_b, a.T, a.Hqk) ||
+        !make_map(&tv, a.v, rows_b, a.T, a.Hv))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(chunk_tc_cluster_kernel,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     TcParams p{a.alpha, a.beta, a.S0, a.S_final, a.T, a.Hqk, a.Hv,
-               static_cast<__nv_bfloat16 *>(a.o)};
+               static_cast<__nv_bfloat16 *>(a.o), a.cu_seqlens};
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = cluster_config(a.B, a.Hv, stream, attr);
     err = cudaLaunchKernelEx(&cfg, chunk_tc_cluster_kernel, tk, tq, tv, p);

@@ -19,6 +19,9 @@ struct ChunkArgs {
     void *o;
     float *S_final;
     int B, T, Hqk, Hv;
+    // Packed sequences: B sequences at token rows cu_seqlens[b] .. cu_seqlens[b+1]
+    // of token arrays with one batch row of T tokens; null for [B, T, ...] arrays.
+    const int *cu_seqlens = nullptr;
 };
 
 struct DecodeArgs {
@@ -27,6 +30,10 @@ struct DecodeArgs {
     void *o;
     float *S_new;
     int B, Hqk, Hv;
+    int ntok = 1;                // tokens per sequence
+    float *S_steps = nullptr;    // state after each token, or null
+    const int *slots = nullptr;  // pool index of each sequence's state, or null
+    int n_slots = 0;
 };
 
 // Launchers: enqueue on `stream`, return the launch's cudaError_t.

@@ -69,8 +69,20 @@ struct TcParams {
     const float *alpha, *beta, *S0;
     float *S_final;
     int T, Hqk, Hv;
-    __nv_bfloat16 *o;   // output, for kernels that store it without a tensor map
+    __nv_bfloat16 *o;   // output, for stores without a tensor map
+    const int *cu_seqlens;   // packed sequences (see ChunkArgs), or null
 };
+
+// Token rows of sequence b: rows tb .. tb + L of batch row bt of the token arrays.
+struct SeqSpan {
+    int tb, L, bt;
+};
+__device__ __forceinline__ SeqSpan seq_span(const TcParams &p, int b) {
+    if (!p.cu_seqlens) return SeqSpan{0, p.T, b};
+    const int s0 = min(max(p.cu_seqlens[b], 0), p.T);   // clamped into [0, T]
+    const int s1 = min(max(p.cu_seqlens[b + 1], s0), p.T);
+    return SeqSpan{s0, s1 - s0, 0};
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
@@ -271,12 +283,13 @@ __device__ void unit_lower_inverse(float *sA, float *sY, int t, int bid) {
     named_sync(bid, 128);
 }
 
-// alpha, beta of tokens 2*lane, 2*lane+1 of chunk cn (alpha = 1, beta = 0 past the end)
-__device__ __forceinline__ void load_gates(const TcParams &p, int b, int h, int T, int cn, int lane,
+// alpha, beta of tokens 2*lane, 2*lane+1 of chunk cn of the sequence (alpha = 1,
+// beta = 0 past its end: those rows then add nothing to the state)
+__device__ __forceinline__ void load_gates(const TcParams &p, const SeqSpan &sq, int h, int cn, int lane,
                                            float &a0, float &a1, float &b0, float &b1) {
-    const int tn = cn * C, Ln = min(C, T - tn);
+    const int tn = cn * C, Ln = min(C, sq.L - tn);
     const int r = 2 * lane;
-    const size_t gi = ((size_t)b * T + tn + r) * p.Hv + h;
+    const size_t gi = ((size_t)sq.bt * p.T + sq.tb + tn + r) * p.Hv + h;
     a0 = r < Ln ? p.alpha[gi] : 1.f;
     b0 = r < Ln ? p.beta[gi] : 0.f;
     a1 = r + 1 < Ln ? p.alpha[gi + p.Hv] : 1.f;

@@ -43,7 +43,7 @@ class Workload:
         return self.B * self.T
 
 
-# The five workloads the library is checked and measured on.
+# The workloads the library is checked and measured on.
 PREFILL_SMALL_FP32 = Workload("gdn_prefill_small_fp32", B=1, T=256, Hqk=2, Hv=6,
                               dtype=torch.float32, seed=20260)
 PREFILL_4K = Workload("gdn_prefill_B1_T4096", B=1, T=4096, Hqk=16, Hv=48, seed=20261)
@@ -53,9 +53,18 @@ PREFILL_256K = Workload("gdn_prefill_B1_T262144", B=1, T=262144, Hqk=16, Hv=48,
                         log_alpha=(-0.02, -0.0005), seed=20263)
 DECODE_B256 = Workload("gdn_decode_B256", B=256, T=1, Hqk=16, Hv=48, s0_std=0.02,
                        seed=20264, decode_steps=1000)
+# Multi-token decode (draft verification): 4 tokens for each of 256 sequences, with
+# the state after every token kept.
+VERIFY_B256_N4 = Workload("gdn_verify_B256_n4", B=256, T=4, Hqk=16, Hv=48, s0_std=0.02,
+                          seed=20265)
+
+# Packed prefill of 24 sequences of mixed lengths (64 .. 8192 tokens, seeded),
+# continuous batching of prompts; extra: lengths drawn by varlen_lengths.
+PREFILL_VARLEN = Workload("gdn_prefill_varlen_N24", B=24, T=0, Hqk=16, Hv=48, s0_std=0.02,
+                          seed=20266, extra={"lo": 64, "hi": 8192})
 
 WORKLOADS = {w.name: w for w in (PREFILL_SMALL_FP32, PREFILL_4K, PREFILL_BATCH8_8K,
-                                  PREFILL_256K, DECODE_B256)}
+                                  PREFILL_256K, DECODE_B256, VERIFY_B256_N4, PREFILL_VARLEN)}
 
 
 def _generator(device, seed: int) -> torch.Generator:
@@ -115,3 +124,34 @@ def decode_inputs(w: Workload, step: int, device="cpu", B: Optional[int] = None)
     return dict(q=d["q"][:, 0].contiguous(), k=d["k"][:, 0].contiguous(),
                 v=d["v"][:, 0].contiguous(), alpha=d["alpha"][:, 0].contiguous(),
                 beta=d["beta"][:, 0].contiguous())
+
+
+def varlen_lengths(n: int, lo: int, hi: int, seed: int):
+    """n sequence lengths, uniform integers in [lo, hi] (seeded, CPU generator)."""
+    g = torch.Generator().manual_seed(seed)
+    return torch.randint(lo, hi + 1, (n,), generator=g).tolist()
+
+
+def varlen_inputs(lengths, Hqk: int, Hv: int, dk: int = 128, dv: int = 128,
+                  dtype=torch.bfloat16, log_alpha=(-0.1, -0.001), s0_std: float = 0.0,
+                  seed: int = 0, device="cpu"):
+    """Packed prefill inputs: q, k [T_total, Hqk, dk], v [T_total, Hv, dv], alpha,
+    beta [T_total, Hv], S0 [N, Hv, dk, dv] or None, cu_seqlens [N + 1] int32, for
+    sequences of the given lengths laid out back to back."""
+    T = int(sum(lengths))
+    d = prefill_inputs(1, max(T, 1), Hqk, Hv, dk, dv, dtype, log_alpha, 0.0, seed, device)
+    out = {key: d[key][0, :T].contiguous() for key in ("q", "k", "v", "alpha", "beta")}
+    g = _generator(device, seed + 1)
+    out["S0"] = (torch.randn((len(lengths), Hv, dk, dv), generator=g, device=device,
+                             dtype=torch.float32) * s0_std) if s0_std > 0 else None
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(torch.tensor(lengths, dtype=torch.int64), 0).to(torch.int32)
+    out["cu_seqlens"] = cu.to(device)
+    return out
+
+
+def varlen_workload_inputs(w: Workload, device="cpu"):
+    """Inputs of a packed-prefill workload (lengths from w.extra, seeded)."""
+    lengths = varlen_lengths(w.B, w.extra["lo"], w.extra["hi"], w.seed)
+    return varlen_inputs(lengths, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.log_alpha, w.s0_std,
+                         w.seed, device)

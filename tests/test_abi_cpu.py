@@ -34,7 +34,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("gdn_chunk_fwd", "gdn_decode_step", "gdn_status_string", "gdn_last_cuda_error",
               "gdn_version", "gdn_set_prefill_kernel", "gdn_get_prefill_kernel",
-              "gdn_prefill_kernel_for"):
+              "gdn_prefill_kernel_for", "gdn_decode_tokens", "gdn_decode_step_slots",
+              "gdn_chunk_fwd_varlen"):
         assert n in names, names
 
 
@@ -145,3 +146,52 @@ def test_prefill_kernel_for_without_device_work(lib):
     assert lib.gdn_prefill_kernel_for(-1, 48, 1) == -1
     assert lib.gdn_prefill_kernel_for(1, 0, 1) == -1
     assert lib.gdn_prefill_kernel_for(1, 48, 5) == -1
+
+
+def test_decode_tokens_argument_checks(lib):
+    def call(B=1, n=2, Hqk=1, Hv=1, dk=128, dv=128, dtype=1, ptr=FAKE, S_new=FAKE, steps=None):
+        return lib.gdn_decode_tokens(ptr, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, S_new, steps,
+                                     B, n, Hqk, Hv, dk, dv, dtype, None)
+    assert call(n=0) == binding.GDN_ERR_INVALID_ARG
+    assert call(n=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(n=65) == binding.GDN_ERR_UNSUPPORTED
+    assert call(B=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(Hqk=2, Hv=3) == binding.GDN_ERR_UNSUPPORTED
+    assert call(dk=64) == binding.GDN_ERR_UNSUPPORTED
+    assert call(dtype=3) == binding.GDN_ERR_INVALID_ARG
+    assert call(ptr=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(S_new=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(ptr=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert call(steps=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert call(B=0) == binding.GDN_OK
+
+
+def test_decode_slots_argument_checks(lib):
+    def call(B=1, n_slots=4, Hqk=1, Hv=1, dk=128, dv=128, dtype=1, pool=FAKE, slots=FAKE, ptr=FAKE):
+        return lib.gdn_decode_step_slots(ptr, FAKE, FAKE, FAKE, FAKE, pool, slots, FAKE,
+                                         B, n_slots, Hqk, Hv, dk, dv, dtype, None)
+    assert call(n_slots=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(B=-2) == binding.GDN_ERR_INVALID_ARG
+    assert call(slots=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(pool=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(slots=ctypes.c_void_p(0x1002)) == binding.GDN_ERR_INVALID_ARG
+    assert call(pool=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert call(Hqk=4, Hv=6) == binding.GDN_ERR_UNSUPPORTED
+    assert call(dtype=9) == binding.GDN_ERR_INVALID_ARG
+    assert call(B=0) == binding.GDN_OK
+
+
+def test_chunk_varlen_argument_checks(lib):
+    def call(N=2, T=64, Hqk=1, Hv=1, dk=128, dv=128, C=64, dtype=1, cu=FAKE, ptr=FAKE):
+        return lib.gdn_chunk_fwd_varlen(ptr, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, cu,
+                                        N, T, Hqk, Hv, dk, dv, C, dtype, None)
+    assert call(cu=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(cu=ctypes.c_void_p(0x1002)) == binding.GDN_ERR_INVALID_ARG
+    assert call(N=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(T=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(N=70000) == binding.GDN_ERR_UNSUPPORTED
+    assert call(C=16) == binding.GDN_ERR_UNSUPPORTED
+    assert call(Hqk=2, Hv=3) == binding.GDN_ERR_UNSUPPORTED
+    assert call(ptr=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert call(N=0) == binding.GDN_OK
+    assert call(T=0) == binding.GDN_OK          # every sequence empty, no S_final: nothing to do

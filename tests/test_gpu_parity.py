@@ -344,3 +344,170 @@ def test_decode_out_of_place_leaves_input_state():
     assert torch.equal(S, S_keep)
     assert torch.equal(S_new, S_in)
     assert torch.equal(o, o2)
+
+
+# ----------------------------------------------------------------------------- multi-token decode
+def decode_tokens_run(d, with_steps=True):
+    B, n, Hqk, dk = d["q"].shape
+    Hv = d["v"].shape[2]
+    o = torch.empty_like(d["v"])
+    S_new = torch.empty_like(d["S0"])
+    steps = torch.empty((B, n, Hv, dk, dk), dtype=torch.float32, device=DEV) if with_steps else None
+    binding.gdn_decode_tokens(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S_new, steps)
+    torch.cuda.synchronize()
+    return o, S_new, steps
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+@pytest.mark.parametrize("n", [1, 2, 5, 8])
+def test_decode_tokens_against_oracle(n, dtype):
+    """n tokens per call: outputs, the final state and the state after every token
+    (for rollback) against the oracle run over the first t+1 tokens."""
+    d = inputs.prefill_inputs(3, n, 2, 6, dtype=dtype, s0_std=0.05, seed=300 + n)
+    o, S_new, steps = decode_tokens_run(to_dev(d))
+    o_ref, S_ref = oracle_ref(d)
+    check(o, o_ref, tau_for(dtype), f"o n={n}")
+    check(S_new, S_ref, tau_for(dtype), f"S_new n={n}")
+    for t in range(n):
+        pre = {k: (v if k == "S0" else v[:, :t + 1]) for k, v in d.items()}
+        _, S_t = oracle_ref(pre)
+        check(steps[:, t], S_t, tau_for(dtype), f"S_steps[{t}] n={n}")
+
+
+def test_decode_tokens_one_token_is_decode_step():
+    w = inputs.DECODE_B256
+    S = inputs.decode_state(w, device=DEV, B=5)
+    x = inputs.decode_inputs(w, 0, device=DEV, B=5)
+    o1 = torch.empty_like(x["v"])
+    S1 = torch.empty_like(S)
+    binding.gdn_decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S, o1, S1)
+    o2 = torch.empty_like(x["v"])[:, None].contiguous()
+    S2 = torch.empty_like(S)
+    binding.gdn_decode_tokens(x["q"][:, None].contiguous(), x["k"][:, None].contiguous(),
+                              x["v"][:, None].contiguous(), x["alpha"][:, None].contiguous(),
+                              x["beta"][:, None].contiguous(), S, o2, S2)
+    torch.cuda.synchronize()
+    assert torch.equal(o2[:, 0], o1)
+    assert torch.equal(S2, S1)
+
+
+def test_decode_tokens_in_place_and_workload_sampled():
+    """B=256, n=4 at model dims, state updated in place; 6 sequences (all heads)
+    against the oracle, and the in-place result equal to the out-of-place one."""
+    w = inputs.VERIFY_B256_N4
+    d = to_dev(inputs.workload_inputs(w))
+    o, S_new, steps = decode_tokens_run(d)
+    S_in = d["S0"].clone()
+    o2 = torch.empty_like(o)
+    binding.gdn_decode_tokens(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S_in, o2, S_in)
+    torch.cuda.synchronize()
+    assert torch.equal(o2, o) and torch.equal(S_in, S_new)
+    assert torch.equal(steps[:, -1], S_new)
+    seqs = [0, 1, 77, 128, 254, 255]
+    sub = {k: v[seqs].cpu() for k, v in d.items()}
+    o_ref, S_ref = oracle_ref(sub)
+    check(o[seqs], o_ref, TAU_BF16, "o")
+    check(S_new[seqs], S_ref, TAU_BF16, "S_new")
+
+
+# ----------------------------------------------------------------------------- slot-indexed decode
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_decode_slots_against_oracle(dtype):
+    """States gathered from a pool by slot; padding entries (-1, out of range) are
+    skipped; pool rows that no sequence names are left untouched."""
+    w = inputs.DECODE_B256
+    n_slots, B = 10, 6
+    pool = inputs.decode_state(w, device=DEV, B=n_slots)
+    pool0 = pool.clone()
+    x = inputs.decode_inputs(w, 3, device=DEV, B=B)
+    if dtype == torch.float32:
+        x = {k: v.float() for k, v in x.items()}
+    slots = torch.tensor([3, -1, 7, 0, 12, 5], dtype=torch.int32, device=DEV)
+    o = torch.full_like(x["v"], 7.0)
+    binding.gdn_decode_step_slots(x["q"], x["k"], x["v"], x["alpha"], x["beta"], pool, slots, o)
+    torch.cuda.synchronize()
+    live = [0, 2, 3, 5]
+    sl = [3, 7, 0, 5]
+    o_ref, S_ref = oracle.decode_step(*(x[k][live].cpu() for k in ("q", "k", "v", "alpha", "beta")),
+                                      pool0[sl].cpu())
+    check(o[live], o_ref, tau_for(dtype), "o")
+    check(pool[sl], S_ref, tau_for(dtype), "pool")
+    assert torch.all(o[[1, 4]] == 7.0)                       # padding rows untouched
+    untouched = [i for i in range(n_slots) if i not in sl]
+    assert torch.equal(pool[untouched], pool0[untouched])
+    # the same as gdn_decode_step on the gathered states
+    S_g = pool0[sl].clone()
+    o_g = binding.decode_step(*(x[k][live] for k in ("q", "k", "v", "alpha", "beta")), S_g)
+    torch.cuda.synchronize()
+    assert torch.equal(o_g, o[live]) and torch.equal(S_g, pool[sl])
+
+
+# ----------------------------------------------------------------------------- packed (varlen) prefill
+def run_varlen(d, kernel="auto"):
+    T, Hv, dv = d["v"].shape
+    N = d["cu_seqlens"].shape[0] - 1
+    o = torch.empty_like(d["v"])
+    S = torch.empty((N, Hv, d["q"].shape[2], dv), dtype=torch.float32, device=DEV)
+    with binding.prefill_kernel(kernel):
+        binding.gdn_chunk_fwd_varlen(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S,
+                                     d["cu_seqlens"])
+    torch.cuda.synchronize()
+    return o, S
+
+
+def varlen_oracle(d, n):
+    """The oracle on sequence n of packed inputs d (host tensors), as a B=1 problem."""
+    cu = d["cu_seqlens"].tolist()
+    a, b = cu[n], cu[n + 1]
+    sub = dict(q=d["q"][None, a:b], k=d["k"][None, a:b], v=d["v"][None, a:b],
+               alpha=d["alpha"][None, a:b], beta=d["beta"][None, a:b],
+               S0=None if d["S0"] is None else d["S0"][n:n + 1])
+    return oracle_ref(sub)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
+def test_prefill_varlen_against_oracle(dtype):
+    """Sequences of 0, 1, 63, 64, 65, 130, 7 and 200 tokens packed back to back:
+    every sequence against the oracle, for every kernel that takes the dtype.
+    Rows of the next sequence share a chunk with a sequence's tail."""
+    lengths = [0, 1, 63, 64, 65, 130, 7, 200]
+    d = inputs.varlen_inputs(lengths, 2, 6, dtype=dtype, s0_std=0.3, seed=41)
+    dd = to_dev(d)
+    refs = [varlen_oracle(d, n) for n in range(len(lengths))]
+    cu = d["cu_seqlens"].tolist()
+    for kernel in kernels_for(dtype):
+        o, S = run_varlen(dd, kernel)
+        for n, (o_ref, S_ref) in enumerate(refs):
+            if lengths[n]:
+                check(o[cu[n]:cu[n + 1]][None], o_ref, tau_for(dtype), f"{kernel} o seq {n}")
+            check(S[n:n + 1], S_ref, tau_for(dtype), f"{kernel} S_final seq {n}")
+        assert torch.equal(S[0], dd["S0"][0])          # empty sequence: the state passes through
+
+
+@pytest.mark.parametrize("kernel", BF16_KERNELS)
+def test_prefill_varlen_equal_lengths_is_batched(kernel):
+    """Equal lengths packed back to back give the bits of the [B, T] call."""
+    B, T = 3, 200
+    d = to_dev(inputs.prefill_inputs(B, T, 2, 6, dtype=torch.bfloat16, s0_std=0.2, seed=43))
+    o_b, S_b = run_chunk(d, kernel=kernel)
+    packed = {k: (v if k == "S0" else v.reshape(B * T, *v.shape[2:]).contiguous()) for k, v in d.items()}
+    packed["cu_seqlens"] = torch.arange(0, (B + 1) * T, T, dtype=torch.int32, device=DEV)
+    o_v, S_v = run_varlen(packed, kernel)
+    assert torch.equal(o_v.reshape(B, T, *o_v.shape[1:]), o_b)
+    assert torch.equal(S_v, S_b)
+
+
+def test_prefill_varlen_workload_sampled():
+    """24 sequences of 64 .. 8192 tokens (91,038 in all), 16/48 heads: the full
+    launch on the GPU; the oracle checks 3 sequences on one QK group each."""
+    w = inputs.PREFILL_VARLEN
+    d = inputs.varlen_workload_inputs(w, device=DEV)
+    o, S = run_varlen(d)
+    cu = d["cu_seqlens"].tolist()
+    for n, (h0, h1) in [(0, (0, 3)), (13, (21, 24)), (23, (45, 48))]:
+        a, b = cu[n], cu[n + 1]
+        sub = dict(q=d["q"][None, a:b], k=d["k"][None, a:b], v=d["v"][None, a:b],
+                   alpha=d["alpha"][None, a:b], beta=d["beta"][None, a:b], S0=d["S0"][n:n + 1])
+        o_ref, S_ref = oracle_ref({k: v.cpu() for k, v in _sub_problem(sub, 0, h0, h1, w.Hv, w.Hqk).items()})
+        check(o[a:b, h0:h1][None], o_ref, TAU_BF16, f"o seq {n} h={h0}:{h1}")
+        check(S[n:n + 1, h0:h1], S_ref, TAU_BF16, f"S_final seq {n} h={h0}:{h1}")
