@@ -67,6 +67,15 @@ def decode_bytes_per_step(w, elt=2):
     return state + tok
 
 
+def verify_bytes_per_call(w, elt=2):
+    """Multi-token decode with per-token states: the state read once, written after
+    each of the n tokens (S_steps) and once more as the final state, plus the n
+    tokens' q, k, v, o, alpha, beta."""
+    state = w.B * w.Hv * w.dk * w.dv * 4
+    tok = w.B * w.T * (2 * w.Hqk * w.dk * elt + 2 * w.Hv * w.dv * elt + 2 * w.Hv * 4)
+    return (2 + w.T) * state + tok
+
+
 # ----------------------------------------------------------------------------- env
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -293,6 +302,57 @@ def time_decode(w, steps, warmup, world, pool=16):
             "window": (wall0, wall1)}
 
 
+def time_calls(call, steps, warmup, world):
+    """CUDA-event time of `steps` calls of call(i) on the current stream, after
+    `warmup` untimed ones; the inputs are larger than L2, so no flush."""
+    stream = torch.cuda.current_stream()
+    for i in range(warmup):
+        call(i)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    barrier(world)
+    wall0 = time.perf_counter()
+    for i in range(steps):
+        ev[i][0].record(stream)
+        call(i)
+        ev[i][1].record(stream)
+    barrier(world)
+    wall1 = time.perf_counter()
+    times = [a.elapsed_time(b) for a, b in ev]
+    return {"total_ms": max_over_ranks(sum(times), world), "per_launch_ms": sum(times) / steps,
+            "launches": steps, "window": (wall0, wall1)}
+
+
+def time_verify(w, steps, warmup, world):
+    """gdn_decode_tokens: n draft tokens for each of B sequences, state in place,
+    the state after every token written to S_steps."""
+    d = inputs.workload_inputs(w, device="cuda")
+    S = d["S0"]
+    o = torch.empty((w.B, w.T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
+    steps_buf = torch.empty((w.B, w.T, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+
+    def call(i):
+        binding.gdn_decode_tokens(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S, o, S, steps_buf)
+
+    return time_calls(call, steps, warmup, world)
+
+
+def time_varlen(w, steps, warmup, world):
+    """gdn_chunk_fwd_varlen over the packed sequences of w (inputs > L2)."""
+    d = inputs.varlen_workload_inputs(w, device="cuda")
+    N = w.B
+    o = torch.empty_like(d["v"])
+    S = torch.empty((N, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+
+    def call(i):
+        binding.gdn_chunk_fwd_varlen(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S,
+                                     d["cu_seqlens"])
+
+    r = time_calls(call, steps, warmup, world)
+    r["tokens"] = int(d["q"].shape[0])
+    return r
+
+
 # ----------------------------------------------------------------------------- oracle
 def oracle_prefill_sample(w, min_seconds=10.0, max_seconds=30.0):
     """Times the fp64 oracle on the prefill workload (all heads), repeating whole
@@ -380,6 +440,8 @@ def main():
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--verify-steps", type=int, default=50)
+    ap.add_argument("--varlen-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto",
                     help="prefill kernel to time (default: the library's own choice)")
@@ -402,6 +464,10 @@ def main():
     with ClockSampler(local) as clocks:
         pre = time_prefill(w, args.steps, args.warmup, world, rank)
         dec = time_decode(wd, args.decode_steps, args.warmup, world)
+    wv, wl = inputs.VERIFY_B256_N4, inputs.PREFILL_VARLEN
+    with ClockSampler(local) as clocks2:
+        ver = time_verify(wv, args.verify_steps, args.warmup, world)
+        vl = time_varlen(wl, args.varlen_steps, args.warmup, world)
     e2e = time_prefill_e2e(w, args.e2e_steps, 3, world)
 
     tokens_per_step = w.B * w.T
@@ -448,6 +514,32 @@ def main():
                              peak_source=f"{peak_src} copy bandwidth",
                              algorithmic_bytes_per_launch=dec_bytes),
             "gpu_launches": dec["launches"],
+        },
+        "verify": {
+            "metric": "draft-verify tokens/s (gdn_decode_tokens, per-token states kept)",
+            "workload": wv.name, "B": wv.B, "tokens_per_sequence": wv.T,
+            "value": job_throughput(wv.B * wv.T, args.verify_steps, world, ver["total_ms"]),
+            "unit": "tokens/s", "ms_per_call": ver["total_ms"] / args.verify_steps,
+            "roofline": dict(roofline("hbm", verify_bytes_per_call(wv) / (ver["per_launch_ms"] * 1e-3) / 1e9,
+                                      peaks["hbm_gbs"], "GB/s", None),
+                             peak_source=f"{peak_src} copy bandwidth",
+                             algorithmic_bytes_per_launch=verify_bytes_per_call(wv)),
+            "gpu_launches": ver["launches"],
+        },
+        "varlen_prefill": {
+            "metric": "packed-prefill tokens/s (gdn_chunk_fwd_varlen)",
+            "workload": wl.name, "sequences": wl.B, "tokens": vl["tokens"],
+            "prefill_kernel": binding.prefill_kernel_for(wl.B, wl.Hv, wl.dtype),
+            "value": job_throughput(vl["tokens"], args.varlen_steps, world, vl["total_ms"]),
+            "unit": "tokens/s", "ms_per_call": vl["total_ms"] / args.varlen_steps,
+            "roofline": dict(roofline("tensor", prefill_flops_per_token(wl) * vl["tokens"]
+                                      / (vl["per_launch_ms"] * 1e-3) / 1e12,
+                                      peaks["bf16_tflops"], "TFLOP/s", None),
+                             peak_source=f"{peak_src} bf16 burst",
+                             hbm_frac=(prefill_bytes_per_token(wl) * vl["tokens"] + wl.B * prefill_state_bytes(wl))
+                             / (vl["per_launch_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"]),
+            "gpu_launches": vl["launches"],
+            "clocks": clocks2.summary([ver["window"], vl["window"]]),
         },
         "e2e": {"value": job_throughput(tokens_per_step, args.e2e_steps, world, e2e["total_ms"]),
                 "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],

@@ -31,7 +31,9 @@ __device__ __forceinline__ void st_stream(float4 *p, float4 v) { __stcs(p, v); }
 // token inputs are [B, n, H, 128] (gates [B, n, Hv]).  Optional: S_steps gets
 // the state after every token ([B, n, Hv, 128, 128]); slots maps sequence b to
 // its state in a pool of n_slots states (a slot outside [0, n_slots) skips b).
-template <typename T>
+// kMulti = false is the one-token form (ntok == 1, S_steps null): the state update
+// and its store are one loop, as the HBM stream wants.
+template <typename T, bool kMulti>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
               const float *__restrict__ alpha, const float *__restrict__ beta,
@@ -60,6 +62,8 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
 #pragma unroll
     for (int m = 0; m < kRowsPerThread; ++m) s[m] = ld_stream(S4 + (warp + 8 * m) * 32 + lane);
 
+    if (!kMulti) ntok = 1;
+    float4 *D4 = reinterpret_cast<float4 *>(S_new + base);
 #pragma unroll 1
     for (int t = 0; t < ntok; ++t) {
         const size_t tok = (size_t)b * ntok + t;            // token row in [B, n, ...]
@@ -112,7 +116,8 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
             o[v_off + 2] = from_f32<T>(fmaf(kq, u.z, a * r.z));
             o[v_off + 3] = from_f32<T>(fmaf(kq, u.w, a * r.w));
         }
-        float4 *P4 = S_steps ? reinterpret_cast<float4 *>(S_steps + gi * kHeadDim * kHeadDim) : nullptr;
+        float4 *P4 = (kMulti && S_steps) ? reinterpret_cast<float4 *>(S_steps + gi * kHeadDim * kHeadDim)
+                                         : nullptr;
 #pragma unroll
         for (int m = 0; m < kRowsPerThread; ++m) {
             const float ki = sk[warp + 8 * m];
@@ -120,29 +125,36 @@ decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restr
             s[m].y = fmaf(a, s[m].y, ki * u.y);
             s[m].z = fmaf(a, s[m].z, ki * u.z);
             s[m].w = fmaf(a, s[m].w, ki * u.w);
-            if (P4) st_stream(P4 + (warp + 8 * m) * 32 + lane, s[m]);
+            if (!kMulti) st_stream(D4 + (warp + 8 * m) * 32 + lane, s[m]);
+            else if (P4) st_stream(P4 + (warp + 8 * m) * 32 + lane, s[m]);
         }
     }
-    float4 *D4 = reinterpret_cast<float4 *>(S_new + base);
+    if (kMulti) {
 #pragma unroll
-    for (int m = 0; m < kRowsPerThread; ++m) st_stream(D4 + (warp + 8 * m) * 32 + lane, s[m]);
+        for (int m = 0; m < kRowsPerThread; ++m) st_stream(D4 + (warp + 8 * m) * 32 + lane, s[m]);
+    }
+}
+
+template <typename T, bool kMulti>
+void launch_typed(const DecodeArgs &a, cudaStream_t stream)
+{
+    const unsigned grid = (unsigned)((size_t)a.B * a.Hv);
+    decode_kernel<T, kMulti><<<grid, kDecodeThreads, 0, stream>>>(
+        (const T *)a.q, (const T *)a.k, (const T *)a.v, a.alpha, a.beta, a.S, (T *)a.o, a.S_new,
+        a.S_steps, a.slots, a.n_slots, a.ntok, a.Hqk, a.Hv);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const DecodeArgs &a, gdn_dtype dtype, cudaStream_t stream)
 {
-    const unsigned grid = (unsigned)((size_t)a.B * a.Hv);
+    const bool multi = a.ntok != 1 || a.S_steps;
     if (dtype == GDN_BF16) {
-        decode_kernel<__nv_bfloat16><<<grid, kDecodeThreads, 0, stream>>>(
-            (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.v,
-            a.alpha, a.beta, a.S, (__nv_bfloat16 *)a.o, a.S_new, a.S_steps, a.slots, a.n_slots,
-            a.ntok, a.Hqk, a.Hv);
+        if (multi) launch_typed<__nv_bfloat16, true>(a, stream);
+        else launch_typed<__nv_bfloat16, false>(a, stream);
     } else {
-        decode_kernel<float><<<grid, kDecodeThreads, 0, stream>>>(
-            (const float *)a.q, (const float *)a.k, (const float *)a.v,
-            a.alpha, a.beta, a.S, (float *)a.o, a.S_new, a.S_steps, a.slots, a.n_slots,
-            a.ntok, a.Hqk, a.Hv);
+        if (multi) launch_typed<float, true>(a, stream);
+        else launch_typed<float, false>(a, stream);
     }
     return cudaGetLastError();
 }
