@@ -205,16 +205,34 @@ def job_throughput(units_per_rank_per_step, steps, world, max_total_ms):
 
 
 # ----------------------------------------------------------------------------- timing
-def time_prefill(w, steps, warmup, world, rank):
+def prefill_call(w, split, stream):
+    """The prefill entry point the bench times: gdn_chunk_fwd_split with the
+    automatic segment count (workspace allocated once), or plain gdn_chunk_fwd."""
+    ws = None
+    if split:
+        need = binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv)
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+
+    def call(d, o, S_final):
+        if split:
+            binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o,
+                                        S_final, segments=0, workspace=ws, stream=stream)
+        else:
+            binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o,
+                                  S_final, stream=stream)
+    return call
+
+
+def time_prefill(w, steps, warmup, world, rank, split=True):
     d = inputs.workload_inputs(w, device="cuda")
     o = torch.empty((w.B, w.T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
     S_final = torch.empty((w.B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
+    call = prefill_call(w, split, stream)
 
     def step():
-        binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S_final,
-                              stream=stream)
+        call(d, o, S_final)
 
     for _ in range(warmup):
         flush.fill_(1)
@@ -238,7 +256,7 @@ def time_prefill(w, steps, warmup, world, rank):
             "window": (wall0, wall1)}
 
 
-def time_prefill_e2e(w, steps, warmup, world):
+def time_prefill_e2e(w, steps, warmup, world, split=True):
     """Same call with inputs from pinned host memory and results read back."""
     host = {k: (None if v is None else v.cpu().pin_memory())
             for k, v in inputs.workload_inputs(w, device="cpu").items()}
@@ -250,13 +268,13 @@ def time_prefill_e2e(w, steps, warmup, world):
     stream = torch.cuda.current_stream()
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = o_h.numel() * o_h.element_size() + S_h.numel() * 4
+    call = prefill_call(w, split, stream)
 
     def step():
         for k_, v in host.items():
             if v is not None:
                 dev[k_].copy_(v, non_blocking=True)
-        binding.gdn_chunk_fwd(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"], dev["S0"],
-                              o, S_final, stream=stream)
+        call(dev, o, S_final)
         o_h.copy_(o, non_blocking=True)
         S_h.copy_(S_final, non_blocking=True)
 
@@ -461,14 +479,16 @@ def main():
     binding.set_prefill_kernel(args.prefill_kernel)
     kernel = binding.prefill_kernel_for(w.B, w.Hv, w.dtype)
 
+    segs = binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv) > 0
     with ClockSampler(local) as clocks:
-        pre = time_prefill(w, args.steps, args.warmup, world, rank)
+        pre = time_prefill(w, args.steps, args.warmup, world, rank, split=segs)
+        plain = time_prefill(w, max(args.steps // 5, 3), args.warmup, world, rank, split=False)
         dec = time_decode(wd, args.decode_steps, args.warmup, world)
     wv, wl = inputs.VERIFY_B256_N4, inputs.PREFILL_VARLEN
     with ClockSampler(local) as clocks2:
         ver = time_verify(wv, args.verify_steps, args.warmup, world)
         vl = time_varlen(wl, args.varlen_steps, args.warmup, world)
-    e2e = time_prefill_e2e(w, args.e2e_steps, 3, world)
+    e2e = time_prefill_e2e(w, args.e2e_steps, 3, world, split=segs)
 
     tokens_per_step = w.B * w.T
     value = job_throughput(tokens_per_step, args.steps, world, pre["total_ms"])
@@ -498,10 +518,15 @@ def main():
         "config": {"workload": w.name, "B": w.B, "T": w.T, "Hqk": w.Hqk, "Hv": w.Hv,
                    "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "state": "fp32",
                    "prefill_kernel": kernel,
+                   "prefill_entry": ("gdn_chunk_fwd_split (segments chosen by the library)" if segs
+                                     else "gdn_chunk_fwd"),
+                   "plain_gdn_chunk_fwd_ms": plain["total_ms"] / max(args.steps // 5, 3),
                    "l2": "flushed before every timed step (256 MiB write)",
                    "parallelism": f"dp{world} (independent sequences per GPU)"},
         "roofline": dict(roofline("tensor", flops_launch / t_launch / 1e12, peaks["bf16_tflops"],
-                                  "TFLOP/s", kernel_traffic("prefill_" + kernel)),
+                                  "TFLOP/s", kernel_traffic("prefill_split" if segs else "prefill_" + kernel)),
+                         timed=("the whole split step: segment launch of the chunk kernel, "
+                                "segment chain, output fix-up" if segs else "the chunk kernel"),
                          peak_source=f"{peak_src} bf16 burst",
                          algorithmic_flops_per_launch=flops_launch,
                          hbm_frac=bytes_launch / t_launch / 1e9 / peaks["hbm_gbs"]),
@@ -544,7 +569,7 @@ def main():
         "e2e": {"value": job_throughput(tokens_per_step, args.e2e_steps, world, e2e["total_ms"]),
                 "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"]},
-        "gpu_launches": pre["launches"],
+        "gpu_launches": pre["launches"] * (3 if segs else 1),
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:

@@ -44,6 +44,8 @@
 #ifndef GDN_H
 #define GDN_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -109,6 +111,42 @@ gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
                                 void *o, float *S_final, const int *cu_seqlens,
                                 int N, int T_total, int Hqk, int Hv, int dk, int dv, int chunk,
                                 gdn_dtype dtype, void *stream);
+
+/*
+ * gdn_chunk_fwd_split -- gdn_chunk_fwd with each sequence cut into segments that
+ * run side by side (long sequences, or few sequences x heads for the GPU).
+ *
+ * Defines: the same function as gdn_chunk_fwd.  The update of section 2.1
+ * "Gated DeltaNet" (page above) is affine in the state, so a segment's end state
+ * is M S_start + D and its outputs are o^0_t + S_start^T r_t.  Here:
+ *   - D and o^0 come from a run from a zero start;
+ *   - M and the rows r_t come from a run from S = I with v = 0;
+ *   - one launch runs these for every segment at once;
+ *   - a short fp32 walk over the segments then gives each S_start, and a
+ *     tensor-core pass adds R S_start to the outputs.
+ * The serial chain is one segment long.  Use: long contexts at small batch
+ * ("Qwen3.8-Flash-Next 技术总结 -- Qwen4 架构的探路者", section 2.1 and the model
+ * card's 262,144-token native context).
+ *
+ * Arguments as gdn_chunk_fwd, plus:
+ *   segments   1..16, or 0 for the most segments whose CTAs all fit on the device
+ *              at once (B*Hv*(2*segments-1) CTAs).  Segments are whole chunks.
+ *   workspace  device scratch of at least gdn_chunk_fwd_split_workspace(...)
+ *              bytes, 256-byte aligned, owned by the caller; its contents on
+ *              entry do not matter, and calls sharing it must not overlap.
+ * Only GDN_BF16 on the tensor cores splits; otherwise, or when one segment
+ * covers the sequence, the call is gdn_chunk_fwd (workspace unused, may be
+ * NULL).  A too small or misaligned workspace returns GDN_ERR_INVALID_ARG.
+ * Rounding differs from gdn_chunk_fwd (outputs of later segments are a sum
+ * of two bf16-rounded terms) within the bf16 tolerance of the method.
+ */
+size_t gdn_chunk_fwd_split_workspace(int B, int T, int Hv, int dk, int dv, int segments);
+gdn_status gdn_chunk_fwd_split(const void *q, const void *k, const void *v,
+                               const float *alpha, const float *beta, const float *S0,
+                               void *o, float *S_final,
+                               int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                               int segments, gdn_dtype dtype, void *workspace,
+                               size_t workspace_bytes, void *stream);
 
 /*
  * gdn_decode_step -- one token for each of B sequences (autoregressive decode).

@@ -51,6 +51,11 @@ def library():
         lib.gdn_chunk_fwd_varlen.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, vp,
                                              I, I, I, I, I, I, I, I, vp]
         lib.gdn_chunk_fwd_varlen.restype = I
+        lib.gdn_chunk_fwd_split_workspace.argtypes = [I, I, I, I, I, I]
+        lib.gdn_chunk_fwd_split_workspace.restype = ctypes.c_size_t
+        lib.gdn_chunk_fwd_split.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
+                                            I, I, I, I, I, I, I, I, I, vp, ctypes.c_size_t, vp]
+        lib.gdn_chunk_fwd_split.restype = I
         lib.gdn_decode_tokens.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp,
                                           I, I, I, I, I, I, I, vp]
         lib.gdn_decode_tokens.restype = I
@@ -192,6 +197,41 @@ def prefill_kernel(name):
         yield
     finally:
         set_prefill_kernel(prev)
+
+
+def split_workspace_bytes(B, T, Hv, segments=0, dk=128, dv=128):
+    """Device scratch bytes gdn_chunk_fwd_split needs (C entry point
+    ``gdn_chunk_fwd_split_workspace``); 0 when no split happens."""
+    return library().gdn_chunk_fwd_split_workspace(B, T, Hv, dk, dv, segments)
+
+
+def gdn_chunk_fwd_split(q, k, v, alpha, beta, S0, o, S_final, segments=0, workspace=None,
+                        chunk=64, stream=None):
+    """Segment-parallel prefill (C entry point ``gdn_chunk_fwd_split``): the same
+    arguments and results as gdn_chunk_fwd.  ``workspace`` is a uint8 CUDA tensor of
+    at least split_workspace_bytes(...) bytes; None allocates one for this call."""
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, T, Hv, dv), q.dtype),
+                               ("o", o, (B, T, Hv, dv), q.dtype),
+                               ("alpha", alpha, (B, T, Hv), torch.float32),
+                               ("beta", beta, (B, T, Hv), torch.float32)):
+        _expect(t, name, shape, dt, dev)
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None:
+            _expect(t, name, (B, Hv, dk, dv), torch.float32, dev)
+    if workspace is None:
+        need = split_workspace_bytes(B, T, Hv, segments, dk, dv)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    elif workspace.device != dev or workspace.dtype != torch.uint8:
+        raise GdnError("workspace must be a uint8 tensor on the inputs' device")
+    _check(library().gdn_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                         _ptr(S0), _ptr(o), _ptr(S_final), B, T, Hqk, Hv, dk, dv,
+                                         chunk, segments, _DTYPES[q.dtype], _ptr(workspace),
+                                         workspace.numel(), _stream_handle(stream, dev)),
+           "gdn_chunk_fwd_split")
 
 
 def gdn_chunk_fwd_varlen(q, k, v, alpha, beta, S0, o, S_final, cu_seqlens, chunk=64,

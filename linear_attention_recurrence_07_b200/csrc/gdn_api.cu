@@ -9,6 +9,7 @@ namespace {
 
 thread_local int g_last_cuda_error = 0;
 constexpr int kMaxDecodeTokens = 64;   // gdn_decode_tokens: tokens per call
+constexpr int kMaxSegments = 16;       // gdn_chunk_fwd_split: segments per sequence
 std::atomic<int> g_prefill_kernel{GDN_PREFILL_AUTO};   // process-wide prefill kernel choice
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -201,6 +202,65 @@ gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v,
     a.slots = slots;
     a.n_slots = n_slots;
     return cuda_status(gdn::launch_decode(a, dtype, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+
+// Most segments whose CTAs (B*Hv*(2S-1): first runs plus transition runs) all fit
+// on the device at once; 1 when even two do not.
+int auto_segments(int B, int Hv)
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 1;
+    }
+    int S = 1;
+    while (S < kMaxSegments && (long long)B * Hv * (2 * (S + 1) - 1) <= sms) ++S;
+    return S;
+}
+
+}  // namespace
+
+size_t gdn_chunk_fwd_split_workspace(int B, int T, int Hv, int dk, int dv, int segments)
+{
+    if (B <= 0 || T <= 0 || Hv <= 0 || dk != gdn::kHeadDim || dv != gdn::kHeadDim) return 0;
+    if (segments == 0) segments = auto_segments(B, Hv);
+    if (segments < 1 || segments > kMaxSegments) return 0;
+    return gdn::chunk_tc_split_workspace(B, T, Hv, segments);
+}
+
+gdn_status gdn_chunk_fwd_split(const void *q, const void *k, const void *v,
+                               const float *alpha, const float *beta, const float *S0,
+                               void *o, float *S_final,
+                               int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                               int segments, gdn_dtype dtype, void *workspace,
+                               size_t workspace_bytes, void *stream)
+{
+    if (segments < 0 || segments > kMaxSegments) return GDN_ERR_INVALID_ARG;
+    if (segments == 0 && B > 0 && Hv > 0) segments = auto_segments(B, Hv);
+    const bool tc = dtype == GDN_BF16 && gdn::chunk_tc_available() &&
+                    g_prefill_kernel.load(std::memory_order_relaxed) != GDN_PREFILL_SIMT;
+    const size_t need = (tc && B > 0 && T > 0 && Hv > 0 && segments > 1)
+                            ? gdn::chunk_tc_split_workspace(B, T, Hv, segments) : 0;
+    if (need == 0 || dk != gdn::kHeadDim || dv != gdn::kHeadDim)   // nothing to split
+        return gdn_chunk_fwd(q, k, v, alpha, beta, S0, o, S_final, B, T, Hqk, Hv, dk, dv, chunk,
+                             dtype, stream);
+    if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_heads(Hqk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if ((long long)B * (2 * segments - 1) > 65535) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, beta, S0, o, S_final};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GDN_ERR_INVALID_ARG;
+    gdn::ChunkArgs a{q, k, v, alpha, beta, S0, o, S_final, B, T, Hqk, Hv};
+    return cuda_status(gdn::launch_chunk_tc_split(a, segments, workspace,
+                                                  static_cast<cudaStream_t>(stream)));
 }
 
 const char *gdn_status_string(gdn_status status)

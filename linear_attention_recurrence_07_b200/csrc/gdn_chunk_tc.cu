@@ -104,7 +104,7 @@ __host__ __device__ constexpr int u_ready(int c) { return (c & 1) ? B_U_READY1 :
 __global__ void __launch_bounds__(NT, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                const TcParams p)
+                const __grid_constant__ CUtensorMap tm_r, const TcParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // Align by offsetting the shared array itself (not via an integer round trip), so
@@ -116,9 +116,40 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const Ctl ctl{bar, abort_flag};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h = blockIdx.x, b = blockIdx.y;
+    const int h = blockIdx.x;
     const int hq = h / (p.Hv / p.Hqk);
-    const SeqSpan sq = seq_span(p, b);           // this sequence's token rows
+    // This CTA's tokens, start state, final state and output (see TcParams).
+    int b = blockIdx.y;
+    SeqSpan sq;
+    bool trans = false;                          // transition run: v = 0, S0 = I
+    const float *s0_src;                         // null: zero start
+    float *sf_dst;                               // null: no final state
+    const CUtensorMap *out_map = &tm_o;
+    int out_t0 = 0;                              // output row = token row - out_t0
+    const size_t hstate = (size_t)kHeadDim * kHeadDim;
+    if (p.seg_len > 0) {
+        int y = blockIdx.y, k;
+        if (y < p.B * p.nseg) {
+            b = y / p.nseg;
+            k = y % p.nseg;
+            s0_src = (k == 0 && p.S0) ? p.S0 + ((size_t)b * p.Hv + h) * hstate : nullptr;
+            sf_dst = p.seg_D + (((size_t)b * p.nseg + k) * p.Hv + h) * hstate;
+        } else {
+            y -= p.B * p.nseg;
+            b = y / (p.nseg - 1);
+            k = 1 + y % (p.nseg - 1);
+            trans = true;
+            s0_src = nullptr;
+            sf_dst = p.seg_M + (((size_t)b * (p.nseg - 1) + k - 1) * p.Hv + h) * hstate;
+            out_map = &tm_r;
+            out_t0 = p.seg_len;
+        }
+        sq = SeqSpan{k * p.seg_len, min(p.seg_len, p.T - k * p.seg_len), b};
+    } else {
+        sq = seq_span(p, b);
+        s0_src = p.S0 ? p.S0 + ((size_t)b * p.Hv + h) * hstate : nullptr;
+        sf_dst = p.S_final ? p.S_final + ((size_t)b * p.Hv + h) * hstate : nullptr;
+    }
     const int nchunks = (sq.L + C - 1) / C;
     const uint32_t sbase = smem_u32(sm);
 
@@ -126,7 +157,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_v);
-        prefetch_tensormap(&tm_o);
+        prefetch_tensormap(out_map);
         for (int i = 0; i < (int)NBAR; ++i) {
             const bool many = (i == B_SOLVE || i == B_PREP || i == B_S_READY || i == B_U_READY ||
                                i == B_U_READY1 || i == B_O_FREE || i == B_O_FREE + 1 ||
@@ -135,6 +166,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
         *abort_flag = 0;
         fence_mbar_init();
+    }
+    if (trans) {   // transition run: v = 0 for every chunk, so the V tile is zero once
+        for (int x = tid; x < 2 * (int)TILE / 16; x += NT)
+            reinterpret_cast<uint4 *>(sm + OFF_V)[x] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, TMEM_COLS);
@@ -163,6 +199,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 if (s) issued_kq1 = c; else issued_kq0 = c;
                 if (c >= 1) ok = ctl.wait(B_V_EMPTY, (c - 1) & 1);
                 if (!ok) break;
+                if (trans) {                 // v = 0: the zero tile stays; only signal it
+                    mbar_arrive(&bar[B_V_FULL]);
+                    continue;
+                }
                 mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * TILE);
                 tma_load_4d(sm + OFF_V, &tm_v, &bar[B_V_FULL], 0, h, t0, sq.bt);
                 tma_load_4d(sm + OFF_V + TILE, &tm_v, &bar[B_V_FULL], 64, h, t0, sq.bt);
@@ -380,12 +420,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         bool ok = true;
         // initial state: S^T[j][d] = S0[d][j]
         {
-            const float *src = p.S0 ? p.S0 + ((size_t)b * p.Hv + h) * kHeadDim * kHeadDim : nullptr;
+            const float *src = s0_src;
 #pragma unroll 1
             for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
                 float v[32];
 #pragma unroll
-                for (int x = 0; x < 32; ++x) v[x] = src ? src[(size_t)(c0 + x) * kHeadDim + j] : 0.f;
+                for (int x = 0; x < 32; ++x)
+                    v[x] = trans ? (c0 + x == j ? 1.f : 0.f) : src ? src[(size_t)(c0 + x) * kHeadDim + j] : 0.f;
                 tmem_st32(t_row + COL_S + c0, v);
             }
             tmem_wait_st();
@@ -406,8 +447,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     dst[(size_t)r * row_stride] =
                         *reinterpret_cast<const __nv_bfloat16 *>(ot + sw128_offset(r, j & 63));
             } else if (leader) {
-                tma_store_4d(&tm_o, sm + OFF_U, 0, h, sq.tb + cp * C, sq.bt);
-                tma_store_4d(&tm_o, sm + OFF_U + TILE, 64, h, sq.tb + cp * C, sq.bt);
+                tma_store_4d(out_map, sm + OFF_U, 0, h, sq.tb + cp * C - out_t0, sq.bt);
+                tma_store_4d(out_map, sm + OFF_U + TILE, 64, h, sq.tb + cp * C - out_t0, sq.bt);
                 bulk_commit_group();
                 if (wait_read) bulk_wait_group_read0();
             }
@@ -526,8 +567,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 store_staged_o(cp, false);
             }
         }
-        if (ok && p.S_final) {
-            float *dst = p.S_final + ((size_t)b * p.Hv + h) * kHeadDim * kHeadDim;
+        if (ok && sf_dst) {
+            float *dst = sf_dst;
 #pragma unroll 1
             for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
                 float v[32];
@@ -574,7 +615,26 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     TcParams p{a.alpha, a.beta, a.S0, a.S_final, a.T, a.Hqk, a.Hv,
                static_cast<__nv_bfloat16 *>(a.o), a.cu_seqlens};
-    chunk_tc_kernel<<<dim3((unsigned)a.Hv, (unsigned)a.B), NT, SMEM_BYTES, stream>>>(tk, tq, tv, to, p);
+    chunk_tc_kernel<<<dim3((unsigned)a.Hv, (unsigned)a.B), NT, SMEM_BYTES, stream>>>(tk, tq, tv, to, to, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, float *segD,
+                                     float *segM, __nv_bfloat16 *R, cudaStream_t stream)
+{
+    CUtensorMap tk, tq, tv, to, tr;
+    if (!make_map(&tk, a.k, a.B, a.T, a.Hqk) || !make_map(&tq, a.q, a.B, a.T, a.Hqk) ||
+        !make_map(&tv, a.v, a.B, a.T, a.Hv) || !make_map(&to, a.o, a.B, a.T, a.Hv) ||
+        !make_map(&tr, R, a.B, a.T - seg_len, a.Hv))
+        return cudaErrorInvalidValue;
+    cudaError_t err = cudaFuncSetAttribute(chunk_tc_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)SMEM_BYTES);
+    if (err != cudaSuccess) return err;
+    TcParams p{a.alpha, a.beta, a.S0, nullptr, a.T, a.Hqk, a.Hv,
+               static_cast<__nv_bfloat16 *>(a.o), nullptr, a.B, seg_len, nseg, segD, segM};
+    const unsigned rows = (unsigned)(a.B * nseg + a.B * (nseg - 1));
+    chunk_tc_kernel<<<dim3((unsigned)a.Hv, rows), NT, SMEM_BYTES, stream>>>(tk, tq, tv, to, tr, p);
     return cudaGetLastError();
 }
 

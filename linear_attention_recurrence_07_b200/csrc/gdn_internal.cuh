@@ -43,6 +43,13 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 bool chunk_tc_available();
 cudaError_t launch_chunk_tc_cluster(const ChunkArgs &a, cudaStream_t stream);
 bool chunk_tc_cluster_fits(int B, int Hv);   // all B * Hv clusters resident at once
+// Segment-parallel prefill (bf16, tensor cores): each sequence in up to `segments`
+// pieces; workspace of chunk_tc_split_workspace bytes (0: no split needed).
+size_t chunk_tc_split_workspace(int B, int T, int Hv, int segments);
+cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *workspace,
+                                  cudaStream_t stream);
+cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, float *segD,
+                                     float *segM, __nv_bfloat16 *R, cudaStream_t stream);
 
 // Element conversions used by the kernels.
 __device__ __forceinline__ float to_f32(float x) { return x; }

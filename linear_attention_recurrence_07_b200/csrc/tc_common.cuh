@@ -71,6 +71,15 @@ struct TcParams {
     int T, Hqk, Hv;
     __nv_bfloat16 *o;   // output, for stores without a tensor map
     const int *cu_seqlens;   // packed sequences (see ChunkArgs), or null
+    // Segment mode (seg_len > 0): each of the B sequences is cut into nseg segments
+    // of seg_len tokens.  CTA rows y < B*nseg run segment y % nseg of sequence
+    // y / nseg from its start state (S0 for the first segment, zero otherwise),
+    // writing o and its final state to seg_D; the B*(nseg-1) rows after them run
+    // segments 1.. from S = I with v = 0, writing their outputs (M_t^T q_t) through
+    // the second output map and their final state (the segment's transition) to
+    // seg_M.
+    int B, seg_len, nseg;
+    float *seg_D, *seg_M;
 };
 
 // Token rows of sequence b: rows tb .. tb + L of batch row bt of the token arrays.

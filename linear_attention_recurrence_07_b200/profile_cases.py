@@ -4,6 +4,7 @@
                                                                 [--kernel tc|tc_cluster|simt]
     python -m linear_attention_recurrence_07_b200.profile_cases decode [--B 64] [--launches 5]
     python -m linear_attention_recurrence_07_b200.profile_cases prefill-fp32 [--T 1024]
+    python -m linear_attention_recurrence_07_b200.profile_cases prefill-split [--segments 0]
 
 Each case builds its seeded inputs on the GPU, runs the entry point `--launches`
 times and synchronizes; it prints nothing but "ok".  Point a profiler at it with
@@ -19,23 +20,32 @@ from . import binding, inputs
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill", "decode", "prefill-fp32"])
+    ap.add_argument("case", choices=["prefill", "decode", "prefill-fp32", "prefill-split"])
+    ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto")
     args = ap.parse_args()
     binding.set_prefill_kernel(args.kernel)
-    if args.case in ("prefill", "prefill-fp32"):
-        w = inputs.PREFILL_4K if args.case == "prefill" else inputs.PREFILL_SMALL_FP32
-        T = args.T or (w.T if args.case == "prefill" else 1024)
+    if args.case in ("prefill", "prefill-fp32", "prefill-split"):
+        w = inputs.PREFILL_SMALL_FP32 if args.case == "prefill-fp32" else inputs.PREFILL_4K
+        T = args.T or (1024 if args.case == "prefill-fp32" else w.T)
         B = args.B or w.B
         d = inputs.prefill_inputs(B, T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.log_alpha,
                                   w.s0_std, w.seed, "cuda")
         o = torch.empty((B, T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
         S = torch.empty((B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+        ws = None
+        if args.case == "prefill-split":
+            need = binding.split_workspace_bytes(B, T, w.Hv, args.segments)
+            ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
         for _ in range(args.launches):
-            binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S)
+            if ws is not None:
+                binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"],
+                                            o, S, segments=args.segments, workspace=ws)
+            else:
+                binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S)
     else:
         w = inputs.DECODE_B256
         B = args.B or 64

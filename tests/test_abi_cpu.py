@@ -35,7 +35,7 @@ def test_header_declares_the_entry_points():
     for n in ("gdn_chunk_fwd", "gdn_decode_step", "gdn_status_string", "gdn_last_cuda_error",
               "gdn_version", "gdn_set_prefill_kernel", "gdn_get_prefill_kernel",
               "gdn_prefill_kernel_for", "gdn_decode_tokens", "gdn_decode_step_slots",
-              "gdn_chunk_fwd_varlen"):
+              "gdn_chunk_fwd_varlen", "gdn_chunk_fwd_split", "gdn_chunk_fwd_split_workspace"):
         assert n in names, names
 
 
@@ -195,3 +195,30 @@ def test_chunk_varlen_argument_checks(lib):
     assert call(ptr=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
     assert call(N=0) == binding.GDN_OK
     assert call(T=0) == binding.GDN_OK          # every sequence empty, no S_final: nothing to do
+
+
+def test_split_workspace_sizes(lib):
+    hs = 128 * 128
+    # B=1, T=4096, 48 heads, 2 segments of 2048 tokens: D (2 segments), M (1), R (2048
+    # rows), S_start (1), each rounded up to 1 KiB
+    need = binding.split_workspace_bytes(1, 4096, 48, segments=2)
+    assert need == 2 * 48 * hs * 4 + 48 * hs * 4 + 2048 * 48 * 128 * 2 + 48 * hs * 2
+    # whole chunks per segment: 385 tokens (7 chunks) in 3 segments of 3 chunks
+    need3 = binding.split_workspace_bytes(2, 385, 6, segments=3)
+    D = 2 * 3 * 6 * hs * 4
+    M = 2 * 2 * 6 * hs * 4
+    R = 2 * (385 - 192) * 6 * 128 * 2
+    align = lambda x: (x + 1023) // 1024 * 1024   # noqa: E731
+    assert need3 == align(align(align(align(D) + M) + R) + M // 2)
+    assert binding.split_workspace_bytes(1, 64, 48, segments=4) == 0     # one chunk: no split
+    assert binding.split_workspace_bytes(1, 4096, 48, segments=1) == 0
+    assert binding.split_workspace_bytes(1, 4096, 48, segments=17) == 0
+    assert lib.gdn_chunk_fwd_split_workspace(1, 4096, 48, 64, 128, 2) == 0
+
+
+def test_split_argument_checks(lib):
+    def call(segments=2, ws=FAKE, nbytes=1 << 40, dtype=1, ptr=FAKE):
+        return lib.gdn_chunk_fwd_split(ptr, FAKE, FAKE, FAKE, FAKE, None, FAKE, None,
+                                       1, 4096, 16, 48, 128, 128, 64, segments, dtype, ws, nbytes, None)
+    assert call(segments=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(segments=17) == binding.GDN_ERR_INVALID_ARG

@@ -185,6 +185,7 @@ def test_prefill_long_context_workload_sampled():
     w = inputs.PREFILL_256K
     d = inputs.workload_inputs(w, device=DEV)
     outs = {kernel: run_chunk(d, kernel=kernel) for kernel in TC_KERNELS}
+    outs["split"] = run_split(d)
     for h in (0, 47):
         o_ref, S_ref = oracle_ref(_sub_problem(d, 0, h, h + 1, w.Hv, w.Hqk))
         for kernel, (o, S) in outs.items():
@@ -511,3 +512,56 @@ def test_prefill_varlen_workload_sampled():
         o_ref, S_ref = oracle_ref({k: v.cpu() for k, v in _sub_problem(sub, 0, h0, h1, w.Hv, w.Hqk).items()})
         check(o[a:b, h0:h1][None], o_ref, TAU_BF16, f"o seq {n} h={h0}:{h1}")
         check(S[n:n + 1, h0:h1], S_ref, TAU_BF16, f"S_final seq {n} h={h0}:{h1}")
+
+
+# ----------------------------------------------------------------------------- segment-parallel prefill
+def run_split(d, segments=0):
+    B, T, Hqk, dk = d["q"].shape
+    Hv, dv = d["v"].shape[2], d["v"].shape[3]
+    o = torch.empty_like(d["v"])
+    S = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=DEV)
+    binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S,
+                                segments=segments)
+    torch.cuda.synchronize()
+    return o, S
+
+
+@pytest.mark.parametrize("segments", [2, 3, 4])
+@pytest.mark.parametrize("T", [130, 385])
+def test_prefill_split_segments_against_oracle(T, segments):
+    """Every sequence cut into segments of whole chunks (the last one ragged),
+    nonzero S0: outputs and the final state against the oracle."""
+    d = inputs.prefill_inputs(2, T, 2, 6, dtype=torch.bfloat16, s0_std=0.3, seed=500 + T + segments)
+    o_ref, S_ref = oracle_ref(d)
+    need = binding.split_workspace_bytes(2, T, 6, segments)
+    assert need > 0
+    o, S = run_split(to_dev(d), segments)
+    check(o, o_ref, TAU_BF16, f"o T={T} segments={segments}")
+    check(S, S_ref, TAU_BF16, f"S_final T={T} segments={segments}")
+
+
+def test_prefill_split_model_dims_workload():
+    """B=1, T=4096, 16/48 heads with the automatic segment count: every output
+    against the oracle."""
+    w = inputs.PREFILL_4K
+    d = inputs.workload_inputs(w, device=DEV)
+    assert binding.split_workspace_bytes(w.B, w.T, w.Hv, 0) > 0
+    o, S = run_split(d)
+    o_ref, S_ref = oracle_ref(d)
+    check(o, o_ref, TAU_BF16, "o")
+    check(S, S_ref, TAU_BF16, "S_final")
+
+
+def test_prefill_split_in_place_and_workspace_checks():
+    d = to_dev(inputs.prefill_inputs(1, 300, 2, 6, dtype=torch.bfloat16, s0_std=0.2, seed=61))
+    o_ref, S_ref = run_split(d, 2)
+    S = d["S0"].clone()
+    o = torch.empty_like(o_ref)
+    binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S, o, S, segments=2)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(S, S_ref)
+    need = binding.split_workspace_bytes(1, 300, 6, 2)
+    short = torch.empty(need - 1024, dtype=torch.uint8, device=DEV)
+    with pytest.raises(binding.GdnError, match="INVALID_ARG"):
+        binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S, o, S,
+                                    segments=2, workspace=short)
