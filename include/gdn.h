@@ -149,6 +149,32 @@ gdn_status gdn_chunk_fwd_split(const void *q, const void *k, const void *v,
                                size_t workspace_bytes, void *stream);
 
 /*
+ * gdn_chunk_fwd_split_noalloc -- gdn_chunk_fwd_split for callers that cannot
+ * allocate device memory: its scratch is a static device array inside the
+ * library (48 MiB, 256-byte aligned) instead of a caller workspace.
+ *
+ * The pages have no counterpart of this entry point; it is a deployment
+ * variant of gdn_chunk_fwd_split, which defines what it computes.
+ *
+ * Arguments and results as gdn_chunk_fwd_split without workspace and
+ * workspace_bytes.
+ * - A GDN_BF16 problem whose scratch (gdn_chunk_fwd_split_workspace) is over
+ *   48 MiB returns GDN_ERR_UNSUPPORTED.
+ * - The first call on a device looks up the array's address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   A failed lookup returns GDN_ERR_CUDA.
+ * - Every call shares the one array, so calls that overlap on the GPU (on
+ *   different streams, or from different threads) race.
+ * - Nothing in the array has to start at zero.
+ * - The call allocates nothing.
+ */
+gdn_status gdn_chunk_fwd_split_noalloc(const void *q, const void *k, const void *v,
+                                       const float *alpha, const float *beta, const float *S0,
+                                       void *o, float *S_final,
+                                       int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                                       int segments, gdn_dtype dtype, void *stream);
+
+/*
  * gdn_decode_step -- one token for each of B sequences (autoregressive decode).
  *
  * Defines: the first form of the update in section 2.1 "Gated DeltaNet",

@@ -56,6 +56,9 @@ def library():
         lib.gdn_chunk_fwd_split.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
                                             I, I, I, I, I, I, I, I, I, vp, ctypes.c_size_t, vp]
         lib.gdn_chunk_fwd_split.restype = I
+        lib.gdn_chunk_fwd_split_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
+                                                    I, I, I, I, I, I, I, I, I, vp]
+        lib.gdn_chunk_fwd_split_noalloc.restype = I
         lib.gdn_decode_tokens.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp,
                                           I, I, I, I, I, I, I, vp]
         lib.gdn_decode_tokens.restype = I
@@ -232,6 +235,29 @@ def gdn_chunk_fwd_split(q, k, v, alpha, beta, S0, o, S_final, segments=0, worksp
                                          chunk, segments, _DTYPES[q.dtype], _ptr(workspace),
                                          workspace.numel(), _stream_handle(stream, dev)),
            "gdn_chunk_fwd_split")
+
+
+def gdn_chunk_fwd_split_noalloc(q, k, v, alpha, beta, S0, o, S_final, segments=0, chunk=64,
+                                stream=None):
+    """gdn_chunk_fwd_split with the library's static scratch (C entry point
+    ``gdn_chunk_fwd_split_noalloc``); the same arguments without a workspace."""
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, T, Hv, dv), q.dtype),
+                               ("o", o, (B, T, Hv, dv), q.dtype),
+                               ("alpha", alpha, (B, T, Hv), torch.float32),
+                               ("beta", beta, (B, T, Hv), torch.float32)):
+        _expect(t, name, shape, dt, dev)
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None:
+            _expect(t, name, (B, Hv, dk, dv), torch.float32, dev)
+    _check(library().gdn_chunk_fwd_split_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+                                                 _ptr(S0), _ptr(o), _ptr(S_final), B, T, Hqk, Hv,
+                                                 dk, dv, chunk, segments, _DTYPES[q.dtype],
+                                                 _stream_handle(stream, dev)),
+           "gdn_chunk_fwd_split_noalloc")
 
 
 def gdn_chunk_fwd_varlen(q, k, v, alpha, beta, S0, o, S_final, cu_seqlens, chunk=64,
