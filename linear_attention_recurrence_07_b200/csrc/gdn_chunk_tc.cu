@@ -29,11 +29,11 @@
 //               group has its inputs ready, state-dependent groups first
 //   warps 2-5   "prep" warpgroup, runs ahead of the state: gates, A and P from
 //               the grams, the triangular solve (fp32 CUDA cores + TF32 warp
-//               MMAs for the block merges), W^T to shared memory and K~
+//               MMAs for the block merges), Bw and Bu, and K~
 //   warps 6-9   "chain" warpgroup, the state-dependent path: S^T -> bf16
-//               operand (+ decay of the fp32 state), U^T -> bf16 operand, the
-//               gamma scaling of the S-part of O^T in TMEM, and the O epilogue
-//               (staged in shared memory, one TMA store)
+//               operand (+ decay of the fp32 state), W^T -> bf16 W operand,
+//               U^T -> bf16 operand, the gamma scaling of the S-part of O^T in
+//               TMEM, and the O epilogue (staged in shared memory, one TMA store)
 // The U^T and O^T accumulators are double-buffered, so the prep work of the
 // next chunk never waits for the state-dependent chain of the current one.
 //
@@ -84,9 +84,9 @@ enum : int {
     B_G_FULL = 6,    // grams done
     B_W_FULL = 7,    // W^T, U~^T done
     B_SOLVE = 8,     // prep: Bw, Bu, P written (128)
-    B_PREP = 9,      // prep: W, K~ written (128)
+    B_PREP = 9,      // prep: K~ written, the K of its stage read (128)
     B_GATES = 10,    // 2: gates of a chunk written
-    B_S_READY = 12,  // chain: S^T bf16 written (128)
+    B_S_READY = 12,  // chain: S^T and W bf16 written, W^T read from TMEM (128)
     B_U_FULL = 13,   // U^T done
     B_U_READY = 14,  // chain: U^T bf16 of a chunk with even index written (128); odd: B_U_READY1
     B_S_FULL = 15,   // state update done
@@ -275,7 +275,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     issued = true;
                 } else if (nwu < ng && mbar_test(&bar[B_SOLVE], nwu & 1) &&
                            mbar_test(&bar[B_V_FULL], nwu & 1) &&
-                           (nwu < 1 || mbar_test(&bar[B_PREP], (nwu - 1) & 1)) &&
+                           (nwu < 1 || mbar_test(&bar[B_S_READY], (nwu - 1) & 1)) &&
                            (nwu < 2 || mbar_test(&bar[u_ready(nwu)], ((nwu >> 1) - 1) & 1))) {
                     const int c = nwu, s = c & 1;
                     const uint32_t st = sbase + OFF_KQ + s * KQ_STAGE;
@@ -355,6 +355,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             named_sync(1, 128);
             if (pt == 0) mbar_arrive(&bar[B_GATES + s]);
+            GDN_TRACE_AT(c, 9, pt == 0);
             // ---- grams -> A (rows 0-63, fp32) and P (rows 64-127, bf16 operand).
             //      Decay factors Gam[r][x] = prod_{x<j<=r} alpha_j are running products
             //      along the row (no special-function work): descending from x = r,
@@ -381,26 +382,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // ---- T = (I + A)^-1, then Bw = T diag(beta gamma) (threads 0-63, row pt)
             //      and Bu = T diag(beta) (threads 64-127, row pt - 64) as bf16 operands
             unit_lower_inverse(sA, sY, pt, 1);
+            GDN_TRACE_AT(c, 22, pt == 0);
+            // the single-buffered Bw, Bu were last read by the W^T / U~^T MMAs of c-1
+            ok = named_and(1, 128, c < 1 || ctl.wait(B_W_FULL, (c - 1) & 1));
+            if (!ok) break;
+            GDN_TRACE_AT(c, 23, pt == 0);
             write_bw_bu(gv, sA, pt, sm + OFF_BW, sm + OFF_BU);
             fence_proxy_async_smem();
             mbar_arrive(&bar[B_SOLVE]);
             GDN_TRACE_AT(c, 12, pt == 0);
-            // ---- W^T -> W [d][r] (MN-major B) ; K~ = diag(g) K.  The single-buffered
-            //      W and K~ must no longer be read by the previous chunk's MMAs.
-            ok = ctl.wait(B_W_FULL, c & 1) && (c < 1 || ctl.wait(B_U_FULL, (c - 1) & 1)) &&
-                 (c < 1 || ctl.wait(B_O_FULL, (c - 1) & 1));   // also frees P of chunk c-1
-            ok = named_and(1, 128, ok);
+            // ---- K~ = diag(g) K.  The single-buffered K~ (and P of chunk c-1) must no
+            //      longer be read by the previous chunk's MMAs.  (W^T -> W is the
+            //      chain's: it waits for the W^T MMA of c anyway.)
+            ok = named_and(1, 128, c < 1 || ctl.wait(B_O_FULL, (c - 1) & 1));
             if (!ok) break;
             tc_fence_after();
             GDN_TRACE_AT(c, 13, pt == 0);
-            {
-                float w0[32], w1[32];
-                tmem_ld32(t_row + COL_W, w0);
-                tmem_ld32(t_row + COL_W + 32, w1);
-                tmem_wait_ld();
-                store_half_row_bf16(sm + OFF_W, row, 0, w0);
-                store_half_row_bf16(sm + OFF_W, row, 1, w1);
-            }
             {
                 const int i = pt >> 1, half = pt & 1;
                 scale_row_bf16(sm + OFF_KQ + s * KQ_STAGE + 2 * half * TILE,
@@ -477,9 +474,24 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tmem_st32(t_row + COL_S + c0 + 32, v + 32);
             }
             tmem_wait_st();
+            GDN_TRACE_AT(c, 24, leader);
+            // W^T (TMEM, lane d) -> W [d][r] bf16 (MN-major B of the U MMAs); the U MMAs
+            // of c-1 that read W last have completed (U_FULL(c-1) waited in c-1)
+            ok = named_and(2, 128, ctl.wait(B_W_FULL, c & 1));
+            if (!ok) break;
+            GDN_TRACE_AT(c, 25, leader);
+            tc_fence_after();
+            {
+                float w0[32], w1[32];
+                tmem_ld32(t_row + COL_W, w0);
+                tmem_ld32(t_row + COL_W + 32, w1);
+                tmem_wait_ld();
+                store_half_row_bf16(sm + OFF_W, j, 0, w0);
+                store_half_row_bf16(sm + OFF_W, j, 1, w1);
+            }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bar[B_S_READY]);
+            mbar_arrive(&bar[B_S_READY]);            // bf16 S^T and W written
             GDN_TRACE_AT(c, 18, leader);
             // O epilogue of the previous chunk: O^T (lane j) -> bf16 tile [r][j] in the
             // U^T buffer (idle from the state update of c-1 to the U^T of c) -> TMA store
