@@ -480,6 +480,11 @@ def main():
     kernel = binding.prefill_kernel_for(w.B, w.Hv, w.dtype)
 
     segs = binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv) > 0
+    # kernels per split step: chunk kernel + one finishing launch for two segments,
+    # chunk kernel + segment chain + output fix-up for more (same plan <=> same size)
+    two = (binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv)
+           == binding.split_workspace_bytes(w.B, w.T, w.Hv, 2, w.dk, w.dv))
+    split_launches = (2 if two else 3) if segs else 1
     with ClockSampler(local) as clocks:
         pre = time_prefill(w, args.steps, args.warmup, world, rank, split=segs)
         plain = time_prefill(w, max(args.steps // 5, 3), args.warmup, world, rank, split=False)
@@ -569,7 +574,7 @@ def main():
         "e2e": {"value": job_throughput(tokens_per_step, args.e2e_steps, world, e2e["total_ms"]),
                 "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"]},
-        "gpu_launches": pre["launches"] * (3 if segs else 1),
+        "gpu_launches": pre["launches"] * split_launches,
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:

@@ -123,7 +123,9 @@ gdn_status gdn_chunk_fwd_varlen(const void *q, const void *k, const void *v,
  *   - M and the rows r_t come from a run from S = I with v = 0;
  *   - one launch runs these for every segment at once;
  *   - a short fp32 walk over the segments then gives each S_start, and a
- *     tensor-core pass adds R S_start to the outputs.
+ *     tensor-core pass adds R S_start to the outputs (with two segments,
+ *     S_start = D of the first, and one launch does both the pass and the
+ *     final state).
  * The serial chain is one segment long.  Use: long contexts at small batch
  * ("Qwen3.8-Flash-Next 技术总结 -- Qwen4 架构的探路者", section 2.1 and the model
  * card's 262,144-token native context).

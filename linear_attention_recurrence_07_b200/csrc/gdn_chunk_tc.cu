@@ -18,24 +18,32 @@
 //   G    = [K;Q] K^T      (lanes 0-63: K K^T, lanes 64-127: Q K^T)    M=128 N=64  K=128
 //   W^T  = K^T (T diag(beta gamma))^T                                  M=128 N=64  K=64
 //   U^T  = V^T (T diag(beta))^T  -  S^T W^T                            M=128 N=64  K=64+128
-//   O^T  = diag(gamma) (S^T Q^T) + U^T P^T,  P = masked Gam o Q K^T
-//   S^T <- gamma_{C-1} S^T + U^T K~,  K~ = diag(g) K                   M=128 N=128 K=64
+//   O^T  = S^T Q~^T + U^T P^T,  Q~ = diag(gamma) Q,  P = masked Gam o Q K^T
+//   S^T <- gamma_{C-1} S^T + (U^T diag(g)) K                            M=128 N=128 K=64
 // The state S^T (128 lanes x 128 fp32 columns) stays in TMEM for the whole
-// sequence; its bf16 copy in shared memory is only an MMA operand.
+// sequence.  The two state-side A operands, S^T and U^T, go to the tensor core
+// from TMEM as packed bf16 (written by the chain with tcgen05.st): they never
+// touch shared memory, whose bandwidth the operand reads of the other MMAs and
+// the CUDA-core prep work already share.
 //
 // One CTA per (sequence, V head), warp-specialised:
-//   warp 0      TMA producer: K, Q (double-buffered) and V tiles, 128B swizzle
+//   warp 0      TMA producer: K, Q (three stages) and V tiles, 128B swizzle
 //   warp 1      MMA issuer (one thread), event-driven: it issues whichever MMA
 //               group has its inputs ready, state-dependent groups first
-//   warps 2-5   "prep" warpgroup, runs ahead of the state: gates, A and P from
-//               the grams, the triangular solve (fp32 CUDA cores + TF32 warp
-//               MMAs for the block merges), Bw and Bu, and K~
-//   warps 6-9   "chain" warpgroup, the state-dependent path: S^T -> bf16
-//               operand (+ decay of the fp32 state), W^T -> bf16 W operand,
-//               U^T -> bf16 operand, the gamma scaling of the S-part of O^T in
-//               TMEM, and the O epilogue (staged in shared memory, one TMA store)
-// The U^T and O^T accumulators are double-buffered, so the prep work of the
-// next chunk never waits for the state-dependent chain of the current one.
+//   warps 2-9   two "prep" warpgroups (even / odd chunks), running ahead of the
+//               state: gates, A and P from the grams, the triangular solve (fp32
+//               CUDA cores + TF32 warp MMAs for the block merges), Bw, Bu, and
+//               Q~ = diag(gamma) Q in place
+//   warps 10-13 "chain" warpgroup, the state-dependent path: W^T -> bf16 W
+//               operand (shared memory), S^T -> bf16 A operand in TMEM (+ decay
+//               of the fp32 state), U^T -> two bf16 A operands in TMEM (in place:
+//               U^T for the O update, U^T diag(g) for the state update), and
+//               the O epilogue (O^T blocks transposed into a bf16 tile staged in
+//               the idle W tile by stmatrix, one TMA store per chunk)
+// TMEM columns are reused: the bf16 S^T takes the W^T columns once W^T has been
+// read, the two bf16 copies of U^T the two halves of its own fp32 buffer.  The U^T and O^T
+// accumulators are double-buffered, so the prep work of the next chunk never
+// waits for the state-dependent chain of the current one.
 //
 // Every wait is bounded.  On a timeout the CTA raises a device error flag, the
 // other roles see a shared abort flag and stop, in-flight copies and MMAs are
@@ -46,62 +54,73 @@ namespace gdn {
 
 namespace {
 
-constexpr int NT = 320;            // 10 warps
+constexpr int NT = 448;            // 14 warps
 
 // TMEM columns (fp32 accumulators over 128 lanes)
 constexpr uint32_t COL_S = 0;      // S^T: 128 columns
 constexpr uint32_t COL_G = 128;    // [K;Q] K^T
-constexpr uint32_t COL_W = 192;    // W^T
-constexpr uint32_t COL_U = 256;    // U^T, two buffers (256, 320)
+constexpr uint32_t COL_W = 192;    // W^T; after the chain read it: S^T bf16 (64 packed columns)
+constexpr uint32_t COL_U = 256;    // U^T, two buffers (256, 320); then U^T, U^T diag(g) bf16 (32 + 32)
 constexpr uint32_t COL_O = 384;    // O^T, two buffers (384, 448)
 constexpr uint32_t TMEM_COLS = 512;
 
 // Shared-memory plan (byte offsets from a 1024-aligned base).
-constexpr uint32_t OFF_KQ = 0;                    // 2 stages x [K d0-63][Q d0-63][K d64-127][Q d64-127]
+constexpr int NKQ = 3;                            // K/Q stages, chunk c uses c % NKQ
+constexpr uint32_t OFF_KQ = 0;                    // NKQ stages x [K d0-63][Q d0-63][K d64-127][Q d64-127]
 constexpr uint32_t KQ_STAGE = 4 * TILE;
-constexpr uint32_t OFF_V = OFF_KQ + 2 * KQ_STAGE; // [V j0-63][V j64-127]
-constexpr uint32_t OFF_KT = OFF_V + 2 * TILE;     // K~ = diag(g) K, same layout as [K0][K1]
-constexpr uint32_t OFF_P = OFF_KT + 2 * TILE;     // 2 x P [r][i] K-major
+constexpr uint32_t OFF_V = OFF_KQ + NKQ * KQ_STAGE;  // [V j0-63][V j64-127]
+constexpr uint32_t OFF_P = OFF_V + 2 * TILE;      // 2 x P [r][i] K-major
 constexpr uint32_t OFF_BW = OFF_P + 2 * TILE;     // T diag(beta gamma) [r][i]
 constexpr uint32_t OFF_BU = OFF_BW + TILE;        // T diag(beta)       [r][i]
 constexpr uint32_t OFF_W = OFF_BU + TILE;         // W stored [d][r] (MN-major B), 128 rows
-constexpr uint32_t OFF_S = OFF_W + 2 * TILE;      // S^T bf16 [j][d], two 64-column halves
-constexpr uint32_t OFF_U = OFF_S + 4 * TILE;      // U^T bf16 [j][i]; between chunks: O staging [r][j]
-constexpr uint32_t OFF_A = OFF_U + 2 * TILE;      // A, then T = (I + A)^-1, fp32 [64][LDA]
-constexpr uint32_t OFF_Y = OFF_A + 64 * LDA * 4;  // solve scratch, fp32 [32][LDY]
-constexpr uint32_t OFF_GATE = OFF_Y + 32 * LDY * 4;  // 2 buffers of gate vectors
-constexpr uint32_t OFF_BAR = OFF_GATE + 2 * GATE_BUF;
-constexpr uint32_t NBAR = 23;
+constexpr uint32_t SA_BYTES = 64 * LDA * 4, SY_BYTES = 32 * LDY * 4;
+constexpr uint32_t OFF_A = OFF_W + 2 * TILE;      // 2 x A, then T = (I + A)^-1, fp32 [64][LDA]
+constexpr uint32_t OFF_Y = OFF_A + 2 * SA_BYTES;  // 2 x solve scratch, fp32 [32][LDY]
+constexpr int NGATE = 3;                          // gate buffers, chunk c uses c % NGATE
+constexpr uint32_t OFF_GATE = OFF_Y + 2 * SY_BYTES;
+constexpr uint32_t OFF_BAR = OFF_GATE + NGATE * GATE_BUF;
+constexpr uint32_t NBAR = 34;
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;    // tmem slot, abort flag
 constexpr uint32_t SMEM_USED = OFF_MISC + 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // slack for aligning the base
+static_assert(OFF_V % 1024 == 0 && OFF_W % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(OFF_GATE % 16 == 0 && GATE_BUF % 16 == 0, "gate vectors are read as float4");
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 
-// barrier indices (arrival count 1 unless noted)
+// Barrier indices (arrival count 1 unless noted).  "x2" barriers are per chunk
+// parity (chunk c uses index c & 1), "x3" per gate buffer (c % 3): a role that
+// waits for chunk c - 2 (or c - 3) while another chunk's phase may already have
+// completed on a shared barrier would read the wrong phase, so every barrier that
+// such a role waits on completes once per chunk of its own class, in order.
 enum : int {
-    B_KQ_FULL = 0,   // 2: TMA K/Q stage landed
-    B_KQ_EMPTY = 2,  // 2: stage no longer read
-    B_V_FULL = 4, B_V_EMPTY = 5,
-    B_G_FULL = 6,    // grams done
-    B_W_FULL = 7,    // W^T, U~^T done
-    B_SOLVE = 8,     // prep: Bw, Bu, P written (128)
-    B_PREP = 9,      // prep: K~ written, the K of its stage read (128)
-    B_GATES = 10,    // 2: gates of a chunk written
-    B_S_READY = 12,  // chain: S^T and W bf16 written, W^T read from TMEM (128)
-    B_U_FULL = 13,   // U^T done
-    B_U_READY = 14,  // chain: U^T bf16 of a chunk with even index written (128); odd: B_U_READY1
-    B_S_FULL = 15,   // state update done
-    B_O_FREE = 16,   // 2: O accumulator read out (128)
-    B_DRAIN = 18,    // final MMA drain
-    B_G_FREE = 19,   // prep: grams read out of TMEM (128)
-    B_U_READY1 = 20,
-    B_X_FULL = 21,   // S-part of O^T (S^T Q^T) done
-    B_O_FULL = 22,   // O^T complete (after U^T P^T)
+    B_KQ_FULL = 0,   // x3 (per K/Q stage): TMA K/Q stage landed
+    B_KQ_EMPTY = 3,  // x3: stage no longer read (after the state update)
+    B_V_FULL = 6, B_V_EMPTY = 7,
+    B_G_FULL = 8,    // x2: grams done
+    B_W_FULL = 10,   // x2: W^T, U~^T done
+    B_SOLVE = 12,    // x2: prep: Bw, Bu written, the K of its stage read (128)
+    B_PREP = 14,     // x2: prep: P written (128)
+    B_GATES = 16,    // x3: gates of a chunk written
+    B_GFREE = 19,    // x3: chain: gates of a chunk no longer read (128)
+    B_S_READY = 22,  // chain: S^T bf16 (TMEM) and W bf16 written (128)
+    B_U_FULL = 23,   // U^T done
+    B_U_READY = 24,  // x2: chain: U^T bf16 (TMEM) written, O^T scaled (128)
+    B_S_FULL = 26,   // state update done
+    B_O_FREE = 27,   // x2: O accumulator read out (128)
+    B_DRAIN = 29,    // final MMA drain
+    B_G_FREE = 30,   // prep: grams read out of TMEM (128)
+    B_X_FULL = 31,   // S-part of O^T (S^T Q^T) done
+    B_O_FULL = 32,   // x2: O^T complete (after U^T P^T)
 };
-// One U_READY barrier per U^T buffer, so that a parity probe of chunk c - 2's
-// phase can never alias with a later completion on the same barrier.
-__host__ __device__ constexpr int u_ready(int c) { return (c & 1) ? B_U_READY1 : B_U_READY; }
+__host__ __device__ constexpr int u_ready(int c) { return B_U_READY + (c & 1); }
+__host__ __device__ constexpr bool many_arrivals(int i) {
+    return i == B_SOLVE || i == B_SOLVE + 1 || i == B_PREP || i == B_PREP + 1 ||
+           (i >= B_GFREE && i < B_GFREE + NGATE) || i == B_S_READY || i == B_U_READY ||
+           i == B_U_READY + 1 || i == B_O_FREE || i == B_O_FREE + 1 || i == B_G_FREE;
+}
+static_assert(B_O_FULL + 2 <= (int)NBAR, "barrier count");
 
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __maxnreg__(128)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                 const __grid_constant__ CUtensorMap tm_r, const TcParams p)
@@ -124,8 +143,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     bool trans = false;                          // transition run: v = 0, S0 = I
     const float *s0_src;                         // null: zero start
     float *sf_dst;                               // null: no final state
-    const CUtensorMap *out_map = &tm_o;
-    int out_t0 = 0;                              // output row = token row - out_t0
+    __nv_bfloat16 *sst_dst = nullptr;            // bf16 S^T of the final state, or null
+    const CUtensorMap *out_map = &tm_o;          // output rows [., out_T, Hv, 128]
+    __nv_bfloat16 *out = p.o;
+    int out_T = p.T, out_t0 = 0;                 // output row = token row - out_t0
     const size_t hstate = (size_t)kHeadDim * kHeadDim;
     if (p.seg_len > 0) {
         int y = blockIdx.y, k;
@@ -134,6 +155,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             k = y % p.nseg;
             s0_src = (k == 0 && p.S0) ? p.S0 + ((size_t)b * p.Hv + h) * hstate : nullptr;
             sf_dst = p.seg_D + (((size_t)b * p.nseg + k) * p.Hv + h) * hstate;
+            if (k == 0 && p.sst) sst_dst = p.sst + ((size_t)b * p.Hv + h) * hstate;
         } else {
             y -= p.B * p.nseg;
             b = y / (p.nseg - 1);
@@ -142,6 +164,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             s0_src = nullptr;
             sf_dst = p.seg_M + (((size_t)b * (p.nseg - 1) + k - 1) * p.Hv + h) * hstate;
             out_map = &tm_r;
+            out = p.r;
+            out_T = p.T - p.seg_len;
             out_t0 = p.seg_len;
         }
         sq = SeqSpan{k * p.seg_len, min(p.seg_len, p.T - k * p.seg_len), b};
@@ -158,12 +182,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(out_map);
-        for (int i = 0; i < (int)NBAR; ++i) {
-            const bool many = (i == B_SOLVE || i == B_PREP || i == B_S_READY || i == B_U_READY ||
-                               i == B_U_READY1 || i == B_O_FREE || i == B_O_FREE + 1 ||
-                               i == B_G_FREE);
-            mbar_init(&bar[i], many ? 128 : 1);
-        }
+        for (int i = 0; i < (int)NBAR; ++i) mbar_init(&bar[i], many_arrivals(i) ? 128 : 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -183,44 +202,81 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
     if (warp == 0) {
         // ======================================================== TMA producer
+        // K/Q (NKQ stages) and V (one buffer) are independent queues: whichever has
+        // a free buffer is loaded next.
         if (lane == 0) {
-            bool ok = true;
-            int issued_kq0 = -1, issued_kq1 = -1, issued_v = -1;
-            for (int c = 0; c < nchunks && ok; ++c) {
-                const int s = c & 1, t0 = sq.tb + c * C;
-                if (c >= 2) ok = ctl.wait(B_KQ_EMPTY + s, ((c >> 1) - 1) & 1);
-                if (!ok) break;
-                unsigned char *st = sm + OFF_KQ + s * KQ_STAGE;
-                mbar_arrive_expect_tx(&bar[B_KQ_FULL + s], KQ_STAGE);
-                tma_load_4d(st + 0 * TILE, &tm_k, &bar[B_KQ_FULL + s], 0, hq, t0, sq.bt);
-                tma_load_4d(st + 1 * TILE, &tm_q, &bar[B_KQ_FULL + s], 0, hq, t0, sq.bt);
-                tma_load_4d(st + 2 * TILE, &tm_k, &bar[B_KQ_FULL + s], 64, hq, t0, sq.bt);
-                tma_load_4d(st + 3 * TILE, &tm_q, &bar[B_KQ_FULL + s], 64, hq, t0, sq.bt);
-                if (s) issued_kq1 = c; else issued_kq0 = c;
-                if (c >= 1) ok = ctl.wait(B_V_EMPTY, (c - 1) & 1);
-                if (!ok) break;
-                if (trans) {                 // v = 0: the zero tile stays; only signal it
-                    mbar_arrive(&bar[B_V_FULL]);
-                    continue;
+            int nkq = 0, nv = 0;
+            int issued_kq[NKQ] = {-1, -1, -1}, issued_v = -1;
+            long long idle_since = clock64();
+            while (nkq < nchunks || nv < nchunks) {
+                if (*abort_flag) break;
+                bool issued = false;
+                if (nkq < nchunks &&
+                    (nkq < NKQ || mbar_test(&bar[B_KQ_EMPTY + nkq % NKQ], ((nkq / NKQ) - 1) & 1))) {
+                    const int s = nkq % NKQ, t0 = sq.tb + nkq * C;
+                    unsigned char *st = sm + OFF_KQ + s * KQ_STAGE;
+                    mbar_arrive_expect_tx(&bar[B_KQ_FULL + s], KQ_STAGE);
+                    tma_load_4d(st + 0 * TILE, &tm_k, &bar[B_KQ_FULL + s], 0, hq, t0, sq.bt);
+                    tma_load_4d(st + 1 * TILE, &tm_q, &bar[B_KQ_FULL + s], 0, hq, t0, sq.bt);
+                    tma_load_4d(st + 2 * TILE, &tm_k, &bar[B_KQ_FULL + s], 64, hq, t0, sq.bt);
+                    tma_load_4d(st + 3 * TILE, &tm_q, &bar[B_KQ_FULL + s], 64, hq, t0, sq.bt);
+                    issued_kq[s] = nkq++;
+                    issued = true;
+                    // the stage's next chunk into L2, so that its load is an L2 hit
+                    // (on a lightly loaded GPU: with every SM busy the extra requests
+                    // cost more than the latency they hide)
+                    const int cf = nkq - 1 + NKQ;
+                    if (p.l2_prefetch && cf < nchunks) {
+                        const int tf = sq.tb + cf * C;
+                        tma_prefetch_4d(&tm_k, 0, hq, tf, sq.bt);
+                        tma_prefetch_4d(&tm_q, 0, hq, tf, sq.bt);
+                        tma_prefetch_4d(&tm_k, 64, hq, tf, sq.bt);
+                        tma_prefetch_4d(&tm_q, 64, hq, tf, sq.bt);
+                        if (!trans) {
+                            tma_prefetch_4d(&tm_v, 0, h, tf, sq.bt);
+                            tma_prefetch_4d(&tm_v, 64, h, tf, sq.bt);
+                        }
+                    }
                 }
-                mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * TILE);
-                tma_load_4d(sm + OFF_V, &tm_v, &bar[B_V_FULL], 0, h, t0, sq.bt);
-                tma_load_4d(sm + OFF_V + TILE, &tm_v, &bar[B_V_FULL], 64, h, t0, sq.bt);
-                issued_v = c;
+                if (nv < nchunks && (nv < 1 || mbar_test(&bar[B_V_EMPTY], (nv - 1) & 1))) {
+                    if (trans) {                 // v = 0: the zero tile stays; only signal it
+                        mbar_arrive(&bar[B_V_FULL]);
+                    } else {
+                        const int t0 = sq.tb + nv * C;
+                        mbar_arrive_expect_tx(&bar[B_V_FULL], 2 * TILE);
+                        tma_load_4d(sm + OFF_V, &tm_v, &bar[B_V_FULL], 0, h, t0, sq.bt);
+                        tma_load_4d(sm + OFF_V + TILE, &tm_v, &bar[B_V_FULL], 64, h, t0, sq.bt);
+                        issued_v = nv;
+                    }
+                    ++nv;
+                    issued = true;
+                }
+                if (issued) {
+                    idle_since = clock64();
+                } else {
+                    __nanosleep(64);
+                    if (clock64() - idle_since > (1ll << 32)) {
+                        *abort_flag = 1;
+                        atomicOr(&g_tc_error, 1u);
+                        break;
+                    }
+                }
             }
             if (*abort_flag) {
                 // Let copies still in flight land before the CTA's memory goes away.
-                if (issued_kq0 >= 0) mbar_wait(&bar[B_KQ_FULL], (issued_kq0 >> 1) & 1, 1ll << 28);
-                if (issued_kq1 >= 0) mbar_wait(&bar[B_KQ_FULL + 1], (issued_kq1 >> 1) & 1, 1ll << 28);
+                for (int s = 0; s < NKQ; ++s)
+                    if (issued_kq[s] >= 0)
+                        mbar_wait(&bar[B_KQ_FULL + s], (issued_kq[s] / NKQ) & 1, 1ll << 28);
                 if (issued_v >= 0) mbar_wait(&bar[B_V_FULL], issued_v & 1, 1ll << 28);
             }
         }
     } else if (warp == 1) {
         // ======================================================== MMA issuer
         // Issues, as soon as their inputs are ready, in this priority order:
-        //   YS(c): O^T += U^T P^T, S^T += U^T K~     needs U^T bf16 of chunk c
-        //   UO(c): U^T += S^T (-W)^T, O^T = S^T Q^T   needs S^T bf16 and prep of c
-        //   WU(c): W^T, U~^T                          needs the solve of c
+        //   YS(c): S^T += (U^T diag(g)) K, O^T += U^T P^T   needs U^T bf16 and P of c
+        //   UO(c): U^T += S^T (-W)^T, O^T = S^T Q^T   needs S^T bf16 and W of c
+        //   WU(c): W^T, U~^T                          needs the solve of c and the
+        //                                             UO MMAs of c-1 completed
         //   G(c):  [K;Q] K^T                          needs the K/Q tiles of c
         if (lane == 0) {
             int ng = 0, nwu = 0, nuo = 0, nys = 0;
@@ -228,57 +284,58 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             while (nys < nchunks) {
                 if (*abort_flag) break;
                 bool issued = false;
-                if (nys < nuo && mbar_test(&bar[u_ready(nys)], (nys >> 1) & 1)) {
+                if (nys < nuo && mbar_test(&bar[u_ready(nys)], (nys >> 1) & 1) &&
+                    mbar_test(&bar[B_PREP + (nys & 1)], (nys >> 1) & 1)) {
                     const int c = nys, s = c & 1;
                     tc_fence_after();
                     const uint32_t col_o = COL_O + s * 64;
                     // the state update first: the next chunk waits for it
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_bf16(tmem + COL_S, smem_desc_sw128(sbase + OFF_U + k * 32, 16, 1024),
-                                 smem_desc_sw128(sbase + OFF_KT + k * 2048, TILE, 1024), ID_S, true);
+                        mma_bf16_ts(tmem + COL_S, tmem + COL_U + s * 64 + 32 + k * 8,
+                                    smem_desc_sw128(sbase + OFF_KQ + (c % NKQ) * KQ_STAGE + k * 2048, 2 * TILE, 1024),
+                                    ID_S, true);
                     mma_commit(&bar[B_S_FULL]);
+                    mma_commit(&bar[B_KQ_EMPTY + c % NKQ]);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_bf16(tmem + col_o, smem_desc_sw128(sbase + OFF_U + k * 32, 16, 1024),
-                                 smem_desc_sw128(sbase + OFF_P + s * TILE + k * 32, 16, 1024), ID_O, true);
-                    mma_commit(&bar[B_O_FULL]);
+                        mma_bf16_ts(tmem + col_o, tmem + COL_U + s * 64 + k * 8,
+                                    smem_desc_sw128(sbase + OFF_P + s * TILE + k * 32, 16, 1024), ID_O, true);
+                    mma_commit(&bar[B_O_FULL + s]);
                     GDN_TRACE_AT(c, 5, true);
                     ++nys;
                     issued = true;
-                } else if (nuo < nwu && mbar_test(&bar[B_PREP], nuo & 1) &&
-                           mbar_test(&bar[B_S_READY], nuo & 1) &&
+                } else if (nuo < nwu && mbar_test(&bar[B_S_READY], nuo & 1) &&
                            (nuo < 2 || mbar_test(&bar[B_O_FREE + (nuo & 1)], ((nuo >> 1) - 1) & 1))) {
                     const int c = nuo, s = c & 1;
-                    const uint32_t st = sbase + OFF_KQ + s * KQ_STAGE;
+                    const uint32_t st = sbase + OFF_KQ + (c % NKQ) * KQ_STAGE;
                     const uint32_t col_o = COL_O + s * 64, col_u = COL_U + s * 64;
                     tc_fence_after();
                     GDN_TRACE_AT(c, 1, true);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t koff = (k >> 2) * 2 * TILE + (k & 3) * 32;
-                        mma_bf16(tmem + col_u, smem_desc_sw128(sbase + OFF_S + koff, 16, 1024),
-                                 smem_desc_sw128(sbase + OFF_W + k * 2048, 2 * TILE, 1024), ID_U, true);
-                    }
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16_ts(tmem + col_u, tmem + COL_W + k * 8,
+                                    smem_desc_sw128(sbase + OFF_W + k * 2048, 2 * TILE, 1024), ID_U, true);
                     mma_commit(&bar[B_U_FULL]);
-                    // S-part of O with the unscaled Q; the chain applies gamma_r afterwards
+                    // S-part of O with Q~ = diag(gamma) Q (scaled in place by the prep)
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t koff = (k >> 2) * 2 * TILE + (k & 3) * 32;
-                        mma_bf16(tmem + col_o, smem_desc_sw128(sbase + OFF_S + koff, 16, 1024),
-                                 smem_desc_sw128(st + TILE + koff, 16, 1024), ID_O, k > 0);
+                        mma_bf16_ts(tmem + col_o, tmem + COL_W + k * 8,
+                                    smem_desc_sw128(st + TILE + koff, 16, 1024), ID_O, k > 0);
                     }
                     mma_commit(&bar[B_X_FULL]);
-                    mma_commit(&bar[B_KQ_EMPTY + s]);
                     GDN_TRACE_AT(c, 2, true);
                     ++nuo;
                     issued = true;
-                } else if (nwu < ng && mbar_test(&bar[B_SOLVE], nwu & 1) &&
+                } else if (nwu < ng && mbar_test(&bar[B_SOLVE + (nwu & 1)], (nwu >> 1) & 1) &&
                            mbar_test(&bar[B_V_FULL], nwu & 1) &&
-                           (nwu < 1 || mbar_test(&bar[B_S_READY], (nwu - 1) & 1)) &&
-                           (nwu < 2 || mbar_test(&bar[u_ready(nwu)], ((nwu >> 1) - 1) & 1))) {
+                           // the UO MMAs of c-1 (last readers of the S^T bf16 in the W^T
+                           // columns) have completed; so have the YS MMAs of c-2 (readers
+                           // of the U^T bf16 in this U^T buffer), issued before them
+                           (nwu < 1 || mbar_test(&bar[B_X_FULL], (nwu - 1) & 1))) {
                     const int c = nwu, s = c & 1;
-                    const uint32_t st = sbase + OFF_KQ + s * KQ_STAGE;
+                    const uint32_t st = sbase + OFF_KQ + (c % NKQ) * KQ_STAGE;
                     const uint32_t col_u = COL_U + s * 64;
                     tc_fence_after();
 #pragma unroll
@@ -289,15 +346,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     for (int k = 0; k < 4; ++k)
                         mma_bf16(tmem + col_u, smem_desc_sw128(sbase + OFF_V + k * 2048, TILE, 1024),
                                  smem_desc_sw128(sbase + OFF_BU + k * 32, 16, 1024), ID_UT, k > 0);
-                    mma_commit(&bar[B_W_FULL]);
+                    mma_commit(&bar[B_W_FULL + s]);
                     mma_commit(&bar[B_V_EMPTY]);
                     GDN_TRACE_AT(c, 6, true);
                     ++nwu;
                     issued = true;
-                } else if (ng < nchunks && mbar_test(&bar[B_KQ_FULL + (ng & 1)], (ng >> 1) & 1) &&
+                } else if (ng < nchunks && mbar_test(&bar[B_KQ_FULL + ng % NKQ], (ng / NKQ) & 1) &&
                            (ng < 1 || mbar_test(&bar[B_G_FREE], (ng - 1) & 1))) {
                     const int c = ng;
-                    const uint32_t st = sbase + OFF_KQ + (c & 1) * KQ_STAGE;
+                    const uint32_t st = sbase + OFF_KQ + (c % NKQ) * KQ_STAGE;
                     tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -305,7 +362,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         mma_bf16(tmem + COL_G, smem_desc_sw128(st + koff, 16, 1024),
                                  smem_desc_sw128(st + koff, 16, 1024), ID_G, k > 0);
                     }
-                    mma_commit(&bar[B_G_FULL]);
+                    mma_commit(&bar[B_G_FULL + (c & 1)]);
                     GDN_TRACE_AT(c, 3, true);
                     ++ng;
                     issued = true;
@@ -325,49 +382,53 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             mma_commit(&bar[B_DRAIN]);
             mbar_wait(&bar[B_DRAIN], 0, 1ll << 30);
         }
-    } else if (warp < 6) {
-        // ======================================================== prep warpgroup
-        const int pt = tid - 64;                      // 0..127
+    } else if (warp < 10) {
+        // ======================================================== prep warpgroups
+        // Two warpgroups prepare alternate chunks (warps 2-5 the even ones, warps
+        // 6-9 the odd ones), each with its own A / solve scratch and P buffer; Bw
+        // and Bu are shared and written in chunk order (each writer waits for the
+        // MMAs of the chunk before that read them).
+        const int wg = (warp - 2) >> 2;               // 0: even chunks, 1: odd chunks
+        const int pt = tid - 64 - 128 * wg;           // 0..127
+        const int nb = wg ? 3 : 1;                    // named barrier of this warpgroup
         const int q4 = warp & 3;                      // TMEM lane quarter
         const int row = q4 * 32 + lane;               // TMEM lane = matrix row
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
-        float *sA = reinterpret_cast<float *>(sm + OFF_A);
-        float *sY = reinterpret_cast<float *>(sm + OFF_Y);
+        float *sA = reinterpret_cast<float *>(sm + OFF_A + wg * SA_BYTES);
+        float *sY = reinterpret_cast<float *>(sm + OFF_Y + wg * SY_BYTES);
+        const bool gate_warp = pt < 32;               // first warp of the warpgroup
         bool ok = true;
-        // gate prefetch (warp 2): alpha, beta of the next chunk are in flight while
-        // the current chunk is prepared
+        // gate prefetch: alpha, beta of this warpgroup's next chunk are in flight
+        // while the current one is prepared
         float nx_a0 = 1.f, nx_a1 = 1.f, nx_b0 = 0.f, nx_b1 = 0.f;
-        if (warp == 2 && nchunks > 0) load_gates(p, sq, h, 0, lane, nx_a0, nx_a1, nx_b0, nx_b1);
-        for (int c = 0; c < nchunks && ok; ++c) {
-            const int s = c & 1;
-            float *gv = reinterpret_cast<float *>(sm + OFF_GATE + s * GATE_BUF);
+        if (gate_warp && wg < nchunks) load_gates(p, sq, h, wg, lane, nx_a0, nx_a1, nx_b0, nx_b1);
+        for (int c = wg; c < nchunks && ok; c += 2) {
+            const int s = c & 1, gb = c % NGATE;
+            float *gv = reinterpret_cast<float *>(sm + OFF_GATE + gb * GATE_BUF);
             GDN_TRACE_AT(c, 8, pt == 0);
-#ifdef GDN_TRACE
-            if (pt == 0 && blockIdx.x == 0 && blockIdx.y == 0 && c < kTraceChunks)
-                g_trace[c][7] = (unsigned long long)clock64();
-#endif
-            // ---- gates (warp 2): b in log2 units, gamma, beta, g, beta gamma, e32;
-            //      padded rows carry alpha = 1, beta = 0 (neutral)
-            if (warp == 2) {
+            // ---- gates (first warp): b in log2 units, gamma, beta, g, beta gamma, e32;
+            //      padded rows carry alpha = 1, beta = 0 (neutral).  The chain is done
+            //      with the gates of chunk c - NGATE, the last user of this buffer.
+            if (c >= NGATE) ok = ctl.wait(B_GFREE + gb, ((c / NGATE) - 1) & 1);
+            if (ok && gate_warp) {
                 const float a0 = nx_a0, a1 = nx_a1, be0 = nx_b0, be1 = nx_b1;
-                if (c + 1 < nchunks) load_gates(p, sq, h, c + 1, lane, nx_a0, nx_a1, nx_b0, nx_b1);
+                if (c + 2 < nchunks) load_gates(p, sq, h, c + 2, lane, nx_a0, nx_a1, nx_b0, nx_b1);
                 compute_gates(gv, a0, a1, be0, be1, lane);
             }
-            named_sync(1, 128);
-            if (pt == 0) mbar_arrive(&bar[B_GATES + s]);
+            ok = named_and(nb, 128, ok);
+            if (!ok) break;
+            if (pt == 0) mbar_arrive(&bar[B_GATES + gb]);
             GDN_TRACE_AT(c, 9, pt == 0);
-            // ---- grams -> A (rows 0-63, fp32) and P (rows 64-127, bf16 operand).
-            //      Decay factors Gam[r][x] = prod_{x<j<=r} alpha_j are running products
-            //      along the row (no special-function work): descending from x = r,
-            //      Gam[r][x-1] = Gam[r][x] alpha_x.  Rows r >= 32 continue into columns
-            //      x < 32 through the table d31[x] = Gam[31][x]: Gam[r][x] = Gam[r][31] d31[x].
-            //      (P buffer s is free again: the previous prep iteration waited for
-            //      the last reader of that buffer, the O update of chunk c - 2.)
-            ok = ctl.wait(B_KQ_FULL + s, (c >> 1) & 1) && ctl.wait(B_G_FULL, c & 1);
-            ok = named_and(1, 128, ok);   // same decision in the whole warpgroup
+            // ---- grams -> A rows (lanes 0-63, fp32 into sA) and P rows (lanes 64-127,
+            //      bf16 pairs kept in registers until the P buffer is free).  Decay
+            //      factors Gam[r][x] = prod_{x<j<=r} alpha_j are running products along
+            //      the row (no special-function work).
+            ok = ctl.wait(B_KQ_FULL + c % NKQ, (c / NKQ) & 1) && ctl.wait(B_G_FULL + s, (c >> 1) & 1);
+            ok = named_and(nb, 128, ok);
             if (!ok) break;
             tc_fence_after();
             GDN_TRACE_AT(c, 10, pt == 0);
+            uint32_t pk[32];
             {
                 float g0[32], g1[32];
                 tmem_ld32(t_row + COL_G, g0);
@@ -375,43 +436,64 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tmem_wait_ld();
                 tc_fence_before();
                 mbar_arrive(&bar[B_G_FREE]);
-                ap_row(gv, row, g0, g1, sA, sm + OFF_P + s * TILE);
+                ap_row_values(gv, row, g0, g1);
+                if (row < 64) {
+                    float4 *dst = reinterpret_cast<float4 *>(sA + row * LDA);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+                        dst[x] = make_float4(g0[4 * x], g0[4 * x + 1], g0[4 * x + 2], g0[4 * x + 3]);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x)
+                        dst[8 + x] = make_float4(g1[4 * x], g1[4 * x + 1], g1[4 * x + 2], g1[4 * x + 3]);
+                }
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    pk[x] = pack_bf16x2(g0[2 * x], g0[2 * x + 1]);
+                    pk[16 + x] = pack_bf16x2(g1[2 * x], g1[2 * x + 1]);
+                }
             }
-            named_sync(1, 128);
+            named_sync(nb, 128);
             GDN_TRACE_AT(c, 11, pt == 0);
             // ---- T = (I + A)^-1, then Bw = T diag(beta gamma) (threads 0-63, row pt)
             //      and Bu = T diag(beta) (threads 64-127, row pt - 64) as bf16 operands
-            unit_lower_inverse(sA, sY, pt, 1);
+            unit_lower_inverse(sA, sY, pt, nb);
             GDN_TRACE_AT(c, 22, pt == 0);
-            // the single-buffered Bw, Bu were last read by the W^T / U~^T MMAs of c-1
-            ok = named_and(1, 128, c < 1 || ctl.wait(B_W_FULL, (c - 1) & 1));
+            // the shared Bw, Bu were last read by the W^T / U~^T MMAs of c-1
+            ok = named_and(nb, 128, c < 1 || ctl.wait(B_W_FULL + ((c - 1) & 1), ((c - 1) >> 1) & 1));
             if (!ok) break;
             GDN_TRACE_AT(c, 23, pt == 0);
             write_bw_bu(gv, sA, pt, sm + OFF_BW, sm + OFF_BU);
+            // ---- Q~ = diag(gamma) Q in place (row pt >> 1, key half pt & 1): the grams
+            //      have read Q; the UO MMAs, issued after SOLVE, read Q~
+            {
+                const int i = pt >> 1, half = pt & 1;
+                unsigned char *qt = sm + OFF_KQ + (c % NKQ) * KQ_STAGE + (2 * half + 1) * TILE;
+                scale_row_bf16(qt, qt, i, gv[GV_GAM + i]);
+            }
             fence_proxy_async_smem();
-            mbar_arrive(&bar[B_SOLVE]);
+            mbar_arrive(&bar[B_SOLVE + s]);
             GDN_TRACE_AT(c, 12, pt == 0);
-            // ---- K~ = diag(g) K.  The single-buffered K~ (and P of chunk c-1) must no
-            //      longer be read by the previous chunk's MMAs.  (W^T -> W is the
-            //      chain's: it waits for the W^T MMA of c anyway.)
-            ok = named_and(1, 128, c < 1 || ctl.wait(B_O_FULL, (c - 1) & 1));
+            // ---- P into this parity's buffer, last read by the YS MMAs of c-2
+            ok = named_and(nb, 128, c < 2 || ctl.wait(B_O_FULL + s, ((c - 2) >> 1) & 1));
             if (!ok) break;
             tc_fence_after();
             GDN_TRACE_AT(c, 13, pt == 0);
-            {
-                const int i = pt >> 1, half = pt & 1;
-                scale_row_bf16(sm + OFF_KQ + s * KQ_STAGE + 2 * half * TILE,
-                               sm + OFF_KT + half * TILE, i, gv[GV_G + i]);
+            if (row >= 64) {
+                unsigned char *ptile = sm + OFF_P + s * TILE;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    *reinterpret_cast<uint4 *>(ptile + sw128_chunk(row - 64, ch)) =
+                        make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bar[B_PREP]);
+            mbar_arrive(&bar[B_PREP + s]);
             GDN_TRACE_AT(c, 14, pt == 0);
         }
     } else {
         // ======================================================== chain warpgroup
         const int q4 = warp & 3;
-        const int j = q4 * 32 + lane;                 // TMEM lane = value column j
+        const int j = q4 * 32 + lane;                 // TMEM lane = value column j (W^T: key dim d)
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
         const bool leader = (j == 0);
         bool ok = true;
@@ -428,58 +510,88 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             tmem_wait_st();
         }
-        // Staged O^T of chunk cp (bf16 tile [r][j] at OFF_U) -> o: one TMA store,
-        // except for the last chunk of a packed sequence that ends inside it,
-        // whose rows past the end belong to the next sequence: its rows are
-        // stored one by one (rows past the array's end are clipped by the TMA).
-        auto store_staged_o = [&](int cp, bool wait_read) {
+        // O epilogue of chunk cp: O^T (lane j) -> bf16 o[t][h][j].  A full chunk is
+        // staged as a bf16 tile [r][j] in the W tile (idle from the end of the UO
+        // MMAs of the chunk after cp to the next W conversion, which first waits
+        // for the store to have read it) and written by one TMA store; a chunk cut
+        // by the end of its sequence is stored row by row from registers (a warp
+        // writes 64 contiguous bytes per row), rows past the end skipped.
+        const size_t row_stride = (size_t)p.Hv * kHeadDim;
+        __nv_bfloat16 *out_h = out + ((size_t)sq.bt * out_T + (sq.tb - out_t0)) * row_stride +
+                               (size_t)h * kHeadDim + j;
+        auto epilogue = [&](int cp) -> bool {
+            if (leader) bulk_wait_group_read0();     // the previous store has read the W tile
+            if (!named_and(2, 128, ctl.wait(B_O_FULL + (cp & 1), (cp >> 1) & 1))) return false;
+            tc_fence_after();
+            const uint32_t col_o = COL_O + (cp & 1) * 64;
             const int rows = min(C, sq.L - cp * C);
-            if (p.cu_seqlens && rows < C) {
-                const size_t row_stride = (size_t)p.Hv * kHeadDim;
-                const unsigned char *ot = sm + OFF_U + (j >> 6) * TILE;
-                __nv_bfloat16 *dst = p.o + ((size_t)sq.bt * p.T + sq.tb + (size_t)cp * C) * row_stride +
-                                     (size_t)h * kHeadDim + j;
+            if (rows == C) {
+                // 8 x 8 blocks (8 lanes j x 8 columns r) come out of TMEM in the m16n8
+                // fragment layout and go to the [r][j] tile transposed by stmatrix
+                const uint32_t stage = smem_u32(sm + OFF_W);
+                const int mt = lane >> 3, mi = lane & 7;   // stored row mi of matrix mt
+                auto emit = [&](const uint32_t *rr, int sl, int cb) {
+#pragma unroll
+                    for (int kk = 0; kk < 2; ++kk) {
+                        uint32_t m[4];
+#pragma unroll
+                        for (int mm = 0; mm < 4; ++mm) {
+                            const int k = 2 * kk + (mm >> 1), g = mm & 1;
+                            m[mm] = pack_bf16x2(__uint_as_float(rr[4 * k + 2 * g]),
+                                                __uint_as_float(rr[4 * k + 2 * g + 1]));
+                        }
+                        const int k = 2 * kk + (mt >> 1), g = mt & 1;
+                        const int orow = 32 * cb + 8 * k + mi;          // output row r
+                        const int jst = q4 * 32 + 16 * sl + 8 * g;      // first j of the block
+                        stmatrix_x4_trans(stage + (jst >> 6) * TILE + sw128_chunk(orow, (jst & 63) >> 3),
+                                          m[0], m[1], m[2], m[3]);
+                    }
+                };
 #pragma unroll 1
-                for (int r = 0; r < rows; ++r)
-                    dst[(size_t)r * row_stride] =
-                        *reinterpret_cast<const __nv_bfloat16 *>(ot + sw128_offset(r, j & 63));
-            } else if (leader) {
-                tma_store_4d(out_map, sm + OFF_U, 0, h, sq.tb + cp * C - out_t0, sq.bt);
-                tma_store_4d(out_map, sm + OFF_U + TILE, 64, h, sq.tb + cp * C - out_t0, sq.bt);
-                bulk_commit_group();
-                if (wait_read) bulk_wait_group_read0();
+                for (int sl = 0; sl < 2; ++sl) {             // 16-lane slab
+                    uint32_t ra[16], rb[16];                 // 32-column blocks 0, 1
+                    const uint32_t ta = tmem + ((uint32_t)(q4 * 32 + 16 * sl) << 16) + col_o;
+                    tmem_ld16x256b_x4(ta, ra);
+                    tmem_ld16x256b_x4(ta + 32, rb);
+                    tmem_wait_ld();
+                    emit(ra, sl, 0);
+                    emit(rb, sl, 1);
+                }
+                tc_fence_before();
+                mbar_arrive(&bar[B_O_FREE + (cp & 1)]);
+                fence_proxy_async_smem();
+                named_sync(2, 128);
+                if (leader) {
+                    tma_store_4d(out_map, sm + OFF_W, 0, h, sq.tb + cp * C - out_t0, sq.bt);
+                    tma_store_4d(out_map, sm + OFF_W + TILE, 64, h, sq.tb + cp * C - out_t0, sq.bt);
+                    bulk_commit_group();
+                }
+                return true;
             }
+            __nv_bfloat16 *dst = out_h + (size_t)cp * C * row_stride;
+#pragma unroll 1
+            for (int r0 = 0; r0 < C; r0 += 32) {
+                float ov[32];
+                tmem_ld32(t_row + col_o + r0, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                    if (r0 + x < rows) dst[(size_t)(r0 + x) * row_stride] = __float2bfloat16_rn(ov[x]);
+            }
+            tc_fence_before();
+            mbar_arrive(&bar[B_O_FREE + (cp & 1)]);
+            return true;
         };
         for (int c = 0; c < nchunks && ok; ++c) {
-            const int s = c & 1;
+            const int s = c & 1, gb = c % NGATE;
+            const float *gv = reinterpret_cast<const float *>(sm + OFF_GATE + gb * GATE_BUF);
             GDN_TRACE_AT(c, 16, leader);
-            if (c > 0) ok = ctl.wait(B_S_FULL, (c - 1) & 1);
-            ok = ok && ctl.wait(B_GATES + s, (c >> 1) & 1);
-            ok = named_and(2, 128, ok);
+            // W^T (TMEM, lane d) -> W [d][r] bf16 (MN-major B of the U MMAs).  The UO
+            // MMAs of c-1 have completed (X_FULL(c-1), waited in c-1) and the O
+            // store staged in the W tile has read it (waited for by the leader).
+            if (leader) bulk_wait_group_read0();
+            ok = named_and(2, 128, ctl.wait(B_W_FULL + s, (c >> 1) & 1));
             if (!ok) break;
-            tc_fence_after();
-            GDN_TRACE_AT(c, 17, leader);
-            const float glast = reinterpret_cast<const float *>(sm + OFF_GATE + s * GATE_BUF)[GV_GAM + C - 1];
-            // S^T -> bf16 operand, and S^T <- gamma_{C-1} S^T
-#pragma unroll 1
-            for (int c0 = 0; c0 < kHeadDim; c0 += 64) {
-                float v[64];
-                tmem_ld32(t_row + COL_S + c0, v);
-                tmem_ld32(t_row + COL_S + c0 + 32, v + 32);
-                tmem_wait_ld();
-                store_row_bf16(sm + OFF_S + (c0 >> 6) * 2 * TILE, j, v);
-#pragma unroll
-                for (int x = 0; x < 64; ++x) v[x] *= glast;
-                tmem_st32(t_row + COL_S + c0, v);
-                tmem_st32(t_row + COL_S + c0 + 32, v + 32);
-            }
-            tmem_wait_st();
-            GDN_TRACE_AT(c, 24, leader);
-            // W^T (TMEM, lane d) -> W [d][r] bf16 (MN-major B of the U MMAs); the U MMAs
-            // of c-1 that read W last have completed (U_FULL(c-1) waited in c-1)
-            ok = named_and(2, 128, ctl.wait(B_W_FULL, c & 1));
-            if (!ok) break;
-            GDN_TRACE_AT(c, 25, leader);
             tc_fence_after();
             {
                 float w0[32], w1[32];
@@ -489,96 +601,70 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 store_half_row_bf16(sm + OFF_W, j, 0, w0);
                 store_half_row_bf16(sm + OFF_W, j, 1, w1);
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar[B_S_READY]);            // bf16 S^T and W written
-            GDN_TRACE_AT(c, 18, leader);
-            // O epilogue of the previous chunk: O^T (lane j) -> bf16 tile [r][j] in the
-            // U^T buffer (idle from the state update of c-1 to the U^T of c) -> TMA store
-            if (c > 0) ok = named_and(2, 128, ctl.wait(B_O_FULL, (c - 1) & 1));
-            if (!ok) break;
-            if (c > 0) {
-                tc_fence_after();
-                const int cp = c - 1;
-                const uint32_t col_o = COL_O + (cp & 1) * 64;
-                unsigned char *ot = sm + OFF_U + (j >> 6) * TILE;
-                const uint32_t jc = j & 63;
-#pragma unroll 1
-                for (int r0 = 0; r0 < C; r0 += 32) {
-                    float ov[32];
-                    tmem_ld32(t_row + col_o + r0, ov);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_offset(r0 + x, jc)) =
-                            __float2bfloat16_rn(ov[x]);
-                }
-                tc_fence_before();
-                mbar_arrive(&bar[B_O_FREE + (cp & 1)]);
-                fence_proxy_async_smem();
-                named_sync(2, 128);
-                store_staged_o(cp, true);      // staging must be read before U^T reuses it
-            }
-            GDN_TRACE_AT(c, 19, leader);
-            // U^T -> bf16 operand
-            ok = ctl.wait(B_U_FULL, c & 1);
+            GDN_TRACE_AT(c, 25, leader);
+            // S^T -> packed bf16 A operand in the (now read) W^T columns, and
+            // S^T <- gamma_{C-1} S^T
+            if (c > 0) ok = ctl.wait(B_S_FULL, (c - 1) & 1);
+            ok = ok && ctl.wait(B_GATES + gb, (c / NGATE) & 1);
             ok = named_and(2, 128, ok);
+            if (!ok) break;
+            tc_fence_after();
+            GDN_TRACE_AT(c, 17, leader);
+            const float glast = gv[GV_GAM + C - 1];
+#pragma unroll 1
+            for (int c0 = 0; c0 < kHeadDim; c0 += 64) {
+                float v[64];
+                uint32_t pk[32];
+                tmem_ld32(t_row + COL_S + c0, v);
+                tmem_ld32(t_row + COL_S + c0 + 32, v + 32);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) pk[x] = pack_bf16x2(v[2 * x], v[2 * x + 1]);
+                tmem_st32u(t_row + COL_W + (c0 >> 1), pk);
+#pragma unroll
+                for (int x = 0; x < 64; ++x) v[x] *= glast;
+                tmem_st32(t_row + COL_S + c0, v);
+                tmem_st32(t_row + COL_S + c0 + 32, v + 32);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();                // the W tile, for the tensor core
+            tc_fence_before();
+            mbar_arrive(&bar[B_S_READY]);
+            GDN_TRACE_AT(c, 18, leader);
+            // U^T -> packed bf16 A operands, in place: U^T (columns 0-31 of its buffer)
+            // for the O update, U^T diag(g) (columns 32-63) for the state update
+            ok = named_and(2, 128, ctl.wait(B_U_FULL, c & 1));
             if (!ok) break;
             tc_fence_after();
             GDN_TRACE_AT(c, 20, leader);
             {
                 float u[64];
+                uint32_t pk[32];
                 tmem_ld32(t_row + COL_U + s * 64, u);
                 tmem_ld32(t_row + COL_U + s * 64 + 32, u + 32);
                 tmem_wait_ld();
-                store_row_bf16(sm + OFF_U, j, u);
-            }
-            // O^T S-part: column r times gamma_r (Q~ = diag(gamma) Q applied here)
-            ok = named_and(2, 128, ctl.wait(B_X_FULL, c & 1));
-            if (!ok) break;
-            tc_fence_after();
-            {
-                const float *gam = reinterpret_cast<const float *>(sm + OFF_GATE + s * GATE_BUF) + GV_GAM;
-                const uint32_t col_o = COL_O + s * 64;
-#pragma unroll 1
-                for (int r0 = 0; r0 < C; r0 += 32) {
-                    float xv[32];
-                    tmem_ld32(t_row + col_o + r0, xv);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) xv[x] *= gam[r0 + x];
-                    tmem_st32(t_row + col_o + r0, xv);
+                for (int x = 0; x < 32; ++x) pk[x] = pack_bf16x2(u[2 * x], u[2 * x + 1]);
+                tmem_st32u(t_row + COL_U + s * 64, pk);
+                const float4 *g4 = reinterpret_cast<const float4 *>(gv + GV_G);
+#pragma unroll
+                for (int x = 0; x < 16; ++x) {
+                    const float4 g = g4[x];
+                    pk[2 * x] = pack_bf16x2(u[4 * x] * g.x, u[4 * x + 1] * g.y);
+                    pk[2 * x + 1] = pack_bf16x2(u[4 * x + 2] * g.z, u[4 * x + 3] * g.w);
                 }
-                tmem_wait_st();
+                tmem_st32u(t_row + COL_U + s * 64 + 32, pk);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bar[u_ready(c)]);
+            mbar_arrive(&bar[B_GFREE + gb]);         // gates of c no longer read
             GDN_TRACE_AT(c, 21, leader);
+            // O epilogue of the previous chunk, while the YS MMAs of c run
+            if (c > 0 && !(ok = epilogue(c - 1))) break;
+            GDN_TRACE_AT(c, 19, leader);
         }
-        if (ok && nchunks > 0) {
-            ok = named_and(2, 128, ctl.wait(B_O_FULL, (nchunks - 1) & 1));
-            if (ok) {
-                tc_fence_after();
-                const int cp = nchunks - 1;
-                const uint32_t col_o = COL_O + (cp & 1) * 64;
-                unsigned char *ot = sm + OFF_U + (j >> 6) * TILE;
-                const uint32_t jc = j & 63;
-#pragma unroll 1
-                for (int r0 = 0; r0 < C; r0 += 32) {
-                    float ov[32];
-                    tmem_ld32(t_row + col_o + r0, ov);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        *reinterpret_cast<__nv_bfloat16 *>(ot + sw128_offset(r0 + x, jc)) =
-                            __float2bfloat16_rn(ov[x]);
-                }
-                fence_proxy_async_smem();
-                named_sync(2, 128);
-                store_staged_o(cp, false);
-            }
-        }
+        if (ok && nchunks > 0) ok = epilogue(nchunks - 1);
         if (ok && sf_dst) {
             float *dst = sf_dst;
 #pragma unroll 1
@@ -588,6 +674,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tmem_wait_ld();
 #pragma unroll
                 for (int x = 0; x < 32; ++x) dst[(size_t)(c0 + x) * kHeadDim + j] = v[x];
+                if (sst_dst) {   // row j of S^T, bf16: 64 contiguous bytes
+                    uint4 *row = reinterpret_cast<uint4 *>(sst_dst + (size_t)j * kHeadDim + c0);
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        row[x] = make_uint4(pack_bf16x2(v[8 * x], v[8 * x + 1]), pack_bf16x2(v[8 * x + 2], v[8 * x + 3]),
+                                            pack_bf16x2(v[8 * x + 4], v[8 * x + 5]), pack_bf16x2(v[8 * x + 6], v[8 * x + 7]));
+                }
             }
         }
         if (leader) bulk_wait_group0();
@@ -614,6 +707,18 @@ extern "C" int gdn_trace_read(unsigned long long *host, int n)
 }
 #endif
 
+// A grid that leaves at least half of the SMs idle.
+static int light_grid(long long ctas)
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return 2 * ctas <= sms ? 1 : 0;
+}
+
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
 {
     CUtensorMap tk, tq, tv, to;
@@ -627,12 +732,14 @@ cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream)
     if (err != cudaSuccess) return err;
     TcParams p{a.alpha, a.beta, a.S0, a.S_final, a.T, a.Hqk, a.Hv,
                static_cast<__nv_bfloat16 *>(a.o), a.cu_seqlens};
+    p.l2_prefetch = light_grid((long long)a.Hv * a.B);
     chunk_tc_kernel<<<dim3((unsigned)a.Hv, (unsigned)a.B), NT, SMEM_BYTES, stream>>>(tk, tq, tv, to, to, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, float *segD,
-                                     float *segM, __nv_bfloat16 *R, cudaStream_t stream)
+                                     float *segM, __nv_bfloat16 *R, __nv_bfloat16 *sst,
+                                     cudaStream_t stream)
 {
     CUtensorMap tk, tq, tv, to, tr;
     if (!make_map(&tk, a.k, a.B, a.T, a.Hqk) || !make_map(&tq, a.q, a.B, a.T, a.Hqk) ||
@@ -644,8 +751,9 @@ cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, 
                                            (int)SMEM_BYTES);
     if (err != cudaSuccess) return err;
     TcParams p{a.alpha, a.beta, a.S0, nullptr, a.T, a.Hqk, a.Hv,
-               static_cast<__nv_bfloat16 *>(a.o), nullptr, a.B, seg_len, nseg, segD, segM};
+               static_cast<__nv_bfloat16 *>(a.o), nullptr, a.B, seg_len, nseg, segD, segM, R, sst};
     const unsigned rows = (unsigned)(a.B * nseg + a.B * (nseg - 1));
+    p.l2_prefetch = light_grid((long long)a.Hv * rows);
     chunk_tc_kernel<<<dim3((unsigned)a.Hv, rows), NT, SMEM_BYTES, stream>>>(tk, tq, tv, to, tr, p);
     return cudaGetLastError();
 }

@@ -48,8 +48,10 @@ bool chunk_tc_cluster_fits(int B, int Hv);   // all B * Hv clusters resident at 
 size_t chunk_tc_split_workspace(int B, int T, int Hv, int segments);
 cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *workspace,
                                   cudaStream_t stream);
+// sst: null, or where the first segments write S_start(1)^T in bf16 (see TcParams).
 cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, float *segD,
-                                     float *segM, __nv_bfloat16 *R, cudaStream_t stream);
+                                     float *segM, __nv_bfloat16 *R, __nv_bfloat16 *sst,
+                                     cudaStream_t stream);
 
 // Element conversions used by the kernels.
 __device__ __forceinline__ float to_f32(float x) { return x; }

@@ -15,6 +15,9 @@
 //      in bf16;
 //   3. out_fix_kernel adds R S_start(k) to the outputs of segment k >= 1
 //      (bf16 warp MMAs, fp32 accumulation, one rounding to bf16).
+// With two segments, S_start(1) = D_0: the chunk kernel writes its bf16 transpose
+// itself, and the fix-up and the final state M_1 D_0 + D_1 no longer depend on
+// each other, so one launch (split2_finish_kernel) runs both side by side.
 // The serial chain of chunk steps is one segment long instead of the sequence.
 #include "tc_common.cuh"
 
@@ -29,42 +32,44 @@ constexpr int kLdR = kHeadDim + 8;        // padded bf16 row strides in shared m
 constexpr int kLdS = kHeadDim + 8;
 
 // S_start of every later segment, in order: S_start(1) = D_0, S_start(k+1) =
-// M_k S_start(k) + D_k (fp32); writes S_start(k)^T in bf16 ([j][d]) for k >= 1 and
-// the final state.  Columns of the state evolve independently, so one CTA takes
-// kChainCols columns of one (head, sequence): M_k whole and its columns of S in
-// shared memory.
-__global__ void __launch_bounds__(kChainThreads, 1)
-seg_chain_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
-                 __nv_bfloat16 *__restrict__ sstT, float *S_final, int nseg, int Hv)
+// M_k S_start(k) + D_k (fp32); writes S_start(k)^T in bf16 ([j][d]) for k >= 1 if
+// write_sst, and the final state.  Columns of the state evolve independently, so
+// one CTA of kThreads threads takes kCols columns of one (head, sequence): M_k
+// whole and its columns of S in shared memory (chain_smem, kHeadDim * (kHeadDim +
+// kCols) floats); each thread owns a 4 x 4 tile of the product.
+template <int kThreads, int kCols>
+__device__ __forceinline__ void chain_columns(const float *__restrict__ segD, const float *__restrict__ segM,
+                                              __nv_bfloat16 *__restrict__ sstT, float *S_final, int nseg,
+                                              int Hv, int h, int b, int j_base, bool write_sst,
+                                              float *chain_smem)
 {
-    extern __shared__ __align__(16) float chain_smem[];
+    static_assert((kHeadDim / 4) * (kCols / 4) == kThreads, "one 4 x 4 tile per thread");
     float *Ms = chain_smem;                        // M_k: [i][d]
-    float *Sc = chain_smem + kHeadDim * kHeadDim;  // S_start columns: [d][c], c < kChainCols
-    const int h = blockIdx.x, b = blockIdx.y, j_base = blockIdx.z * kChainCols;
+    float *Sc = chain_smem + kHeadDim * kHeadDim;  // S_start columns: [d][c], c < kCols
     const int tid = threadIdx.x;
     const size_t hs = (size_t)kHeadDim * kHeadDim;
     const float *D0 = segD + (((size_t)b * nseg + 0) * Hv + h) * hs;
 #pragma unroll 16
-    for (int e = tid; e < kHeadDim * kChainCols; e += kChainThreads) {
-        const int d = e / kChainCols, c = e % kChainCols;
+    for (int e = tid; e < kHeadDim * kCols; e += kThreads) {
+        const int d = e / kCols, c = e % kCols;
         Sc[e] = D0[(size_t)d * kHeadDim + j_base + c];
     }
-    // thread tile: rows i0 .. i0+3 (of 128), columns c0 .. c0+3 (of kChainCols)
-    const int i0 = 4 * (tid / 8), c0 = 4 * (tid % 8);
+    // thread tile: rows i0 .. i0+3 (of 128), columns c0 .. c0+3 (of kCols)
+    const int i0 = 4 * (tid / (kCols / 4)), c0 = 4 * (tid % (kCols / 4));
     for (int k = 1; k < nseg; ++k) {
         const float *Mk = segM + (((size_t)b * (nseg - 1) + (k - 1)) * Hv + h) * hs;
         const float *Dk = segD + (((size_t)b * nseg + k) * Hv + h) * hs;
         __nv_bfloat16 *dst = sstT + (((size_t)b * (nseg - 1) + (k - 1)) * Hv + h) * hs;
         __syncthreads();                           // Sc complete; Ms free
 #pragma unroll 16
-        for (int e = tid; e < kHeadDim * kHeadDim / 4; e += kChainThreads)
+        for (int e = tid; e < kHeadDim * kHeadDim / 4; e += kThreads)
             reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(Mk)[e];
         // S_start(k)^T for the output fix-up: row j = j_base + c, 128 bf16 (d)
-        for (int e = tid; e < kChainCols * (kHeadDim / 8); e += kChainThreads) {
+        for (int e = tid; write_sst && e < kCols * (kHeadDim / 8); e += kThreads) {
             const int c = e / (kHeadDim / 8), d8 = 8 * (e % (kHeadDim / 8));
             __align__(16) __nv_bfloat16 v8[8];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) v8[x] = __float2bfloat16_rn(Sc[(d8 + x) * kChainCols + c]);
+            for (int x = 0; x < 8; ++x) v8[x] = __float2bfloat16_rn(Sc[(d8 + x) * kCols + c]);
             *reinterpret_cast<uint4 *>(dst + (size_t)(j_base + c) * kHeadDim + d8) =
                 *reinterpret_cast<const uint4 *>(v8);
         }
@@ -79,7 +84,7 @@ seg_chain_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
             float mi[4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) mi[x] = Ms[(i0 + x) * kHeadDim + d];
-            const float4 sv = *reinterpret_cast<const float4 *>(&Sc[d * kChainCols + c0]);
+            const float4 sv = *reinterpret_cast<const float4 *>(&Sc[d * kCols + c0]);
             const float sj[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
             for (int x = 0; x < 4; ++x)
@@ -90,7 +95,7 @@ seg_chain_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
             const float4 dv = *reinterpret_cast<const float4 *>(&Dk[(size_t)(i0 + x) * kHeadDim + j_base + c0]);
-            *reinterpret_cast<float4 *>(&Sc[(i0 + x) * kChainCols + c0]) =
+            *reinterpret_cast<float4 *>(&Sc[(i0 + x) * kCols + c0]) =
                 make_float4(acc[x][0] + dv.x, acc[x][1] + dv.y, acc[x][2] + dv.z, acc[x][3] + dv.w);
         }
     }
@@ -98,34 +103,44 @@ seg_chain_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
     if (S_final) {
         float *out = S_final + ((size_t)b * Hv + h) * hs;
 #pragma unroll 16
-        for (int e = tid; e < kHeadDim * kChainCols; e += kChainThreads) {
-            const int d = e / kChainCols, c = e % kChainCols;
+        for (int e = tid; e < kHeadDim * kCols; e += kThreads) {
+            const int d = e / kCols, c = e % kCols;
             out[(size_t)d * kHeadDim + j_base + c] = Sc[e];
         }
     }
+}
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+seg_chain_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
+                 __nv_bfloat16 *__restrict__ sstT, float *S_final, int nseg, int Hv)
+{
+    extern __shared__ __align__(16) float chain_smem[];
+    chain_columns<kChainThreads, kChainCols>(segD, segM, sstT, S_final, nseg, Hv, blockIdx.x, blockIdx.y,
+                                             blockIdx.z * kChainCols, true, chain_smem);
 }
 
 __device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16 *p) {
     return *reinterpret_cast<const uint32_t *>(p);
 }
 
-// o[t] += R[t - seg_len] S_start(k) for the rows t of segment k >= 1.  One CTA per
-// kFixTiles x kFixRows rows of one segment of one (head, sequence); 4 warps of 16
-// rows x 128 columns per tile.
-__global__ void __launch_bounds__(128)
-out_fix_kernel(const __nv_bfloat16 *__restrict__ Rr, const __nv_bfloat16 *__restrict__ sstT,
-               __nv_bfloat16 *__restrict__ o, int T, int seg_len, int nseg, int Hv)
+// o[t] += R[t - seg_len] S_start(k) for the rows t of segment k >= 1.  One CTA of
+// 128 threads per kFixTiles x kFixRows rows (row group `grp`, counting the groups
+// of every later segment in order) of one (head, sequence); 4 warps of 16 rows x
+// 128 columns per tile.
+__device__ __forceinline__ void fix_rows(const __nv_bfloat16 *__restrict__ Rr,
+                                         const __nv_bfloat16 *__restrict__ sstT,
+                                         __nv_bfloat16 *__restrict__ o, int T, int seg_len, int nseg,
+                                         int Hv, int grp, int h, int b, __nv_bfloat16 *fix_smem)
 {
-    extern __shared__ __align__(16) __nv_bfloat16 fix_smem[];
     __nv_bfloat16 *sS = fix_smem;                        // S_start^T: [j][kLdS]
     __nv_bfloat16 *sR = fix_smem + kHeadDim * kLdS;      // R tile: [kFixRows][kLdR]
     __nv_bfloat16 *sO = sR + kFixRows * kLdR;            // o tile: [kFixRows][kLdR]
-    const int h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    const int tid = threadIdx.x;
     const int TR = T - seg_len;                          // rows of R
     const int groups = (seg_len + kFixTiles * kFixRows - 1) / (kFixTiles * kFixRows);
-    const int k = 1 + blockIdx.x / groups;               // segment
+    const int k = 1 + grp / groups;                      // segment
     const int seg_r0 = (k - 1) * seg_len;                // its first R row
-    const int r_begin = seg_r0 + (blockIdx.x % groups) * kFixTiles * kFixRows;
+    const int r_begin = seg_r0 + (grp % groups) * kFixTiles * kFixRows;
     const int r_end = min(min(r_begin + kFixTiles * kFixRows, seg_r0 + seg_len), TR);
     const size_t row_stride = (size_t)Hv * kHeadDim;
     const __nv_bfloat16 *St = sstT + (((size_t)b * (nseg - 1) + (k - 1)) * Hv + h) * kHeadDim * kHeadDim;
@@ -206,6 +221,39 @@ out_fix_kernel(const __nv_bfloat16 *__restrict__ Rr, const __nv_bfloat16 *__rest
     }
 }
 
+__global__ void __launch_bounds__(128)
+out_fix_kernel(const __nv_bfloat16 *__restrict__ Rr, const __nv_bfloat16 *__restrict__ sstT,
+               __nv_bfloat16 *__restrict__ o, int T, int seg_len, int nseg, int Hv)
+{
+    extern __shared__ __align__(16) __nv_bfloat16 fix_smem[];
+    fix_rows(Rr, sstT, o, T, seg_len, nseg, Hv, blockIdx.x, blockIdx.y, blockIdx.z, fix_smem);
+}
+
+// Two segments: CTAs [0, n_state) compute the final state M_1 D_0 + D_1 (kStateCols
+// columns of one (head, sequence) each), the rest the output fix-up of segment 1,
+// whose S_start(1)^T the chunk kernel has written.
+constexpr int kStateCols = 16;            // 128 threads: one 4 x 4 tile each
+__global__ void __launch_bounds__(128)
+split2_finish_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
+                     const __nv_bfloat16 *__restrict__ Rr, const __nv_bfloat16 *__restrict__ sstT,
+                     __nv_bfloat16 *__restrict__ o, float *S_final, int T, int seg_len, int Hv, int B)
+{
+    extern __shared__ __align__(16) unsigned char finish_smem[];
+    constexpr int per_head = kHeadDim / kStateCols;
+    const int n_state = S_final ? B * Hv * per_head : 0;
+    const int x = blockIdx.x;
+    if (x < n_state) {
+        const int jb = x % per_head, bh = x / per_head;
+        chain_columns<128, kStateCols>(segD, segM, nullptr, S_final, 2, Hv, bh % Hv, bh / Hv,
+                                       jb * kStateCols, false, reinterpret_cast<float *>(finish_smem));
+        return;
+    }
+    const int groups = (seg_len + kFixTiles * kFixRows - 1) / (kFixTiles * kFixRows);
+    const int y = x - n_state;                           // (b, h, group)
+    fix_rows(Rr, sstT, o, T, seg_len, 2, Hv, y % groups, (y / groups) % Hv, y / (groups * Hv),
+             reinterpret_cast<__nv_bfloat16 *>(finish_smem));
+}
+
 constexpr size_t align_up(size_t x) { return (x + 1023) & ~(size_t)1023; }
 
 struct SplitPlan {
@@ -250,7 +298,21 @@ cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *worksp
     __nv_bfloat16 *R = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_R);
     __nv_bfloat16 *sstT = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_S);
 
-    cudaError_t err = launch_chunk_tc_segments(a, pl.seg_len, pl.nseg, segD, segM, R, stream);
+    const size_t fix_smem = (size_t)(2 * kFixRows * kLdR + kHeadDim * kLdS) * sizeof(__nv_bfloat16);
+    const int groups = (pl.seg_len + kFixTiles * kFixRows - 1) / (kFixTiles * kFixRows);
+    if (pl.nseg == 2) {
+        cudaError_t err = launch_chunk_tc_segments(a, pl.seg_len, pl.nseg, segD, segM, R, sstT, stream);
+        if (err != cudaSuccess) return err;
+        const size_t state_smem = ((size_t)kHeadDim * kHeadDim + (size_t)kHeadDim * kStateCols) * sizeof(float);
+        const size_t smem = state_smem > fix_smem ? state_smem : fix_smem;
+        err = cudaFuncSetAttribute(split2_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+        const int n_state = a.S_final ? a.B * a.Hv * (kHeadDim / kStateCols) : 0;
+        split2_finish_kernel<<<(unsigned)(n_state + a.B * a.Hv * groups), 128, smem, stream>>>(
+            segD, segM, R, sstT, static_cast<__nv_bfloat16 *>(a.o), a.S_final, a.T, pl.seg_len, a.Hv, a.B);
+        return cudaGetLastError();
+    }
+    cudaError_t err = launch_chunk_tc_segments(a, pl.seg_len, pl.nseg, segD, segM, R, nullptr, stream);
     if (err != cudaSuccess) return err;
     const size_t chain_smem = ((size_t)kHeadDim * kHeadDim + (size_t)kHeadDim * kChainCols) * sizeof(float);
     err = cudaFuncSetAttribute(seg_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -261,10 +323,8 @@ cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *worksp
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     // each CTA covers up to kFixTiles x kFixRows rows of one segment
-    const size_t fix_smem = (size_t)(2 * kFixRows * kLdR + kHeadDim * kLdS) * sizeof(__nv_bfloat16);
     err = cudaFuncSetAttribute(out_fix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fix_smem);
     if (err != cudaSuccess) return err;
-    const int groups = (pl.seg_len + kFixTiles * kFixRows - 1) / (kFixTiles * kFixRows);
     out_fix_kernel<<<dim3((unsigned)((pl.nseg - 1) * groups), (unsigned)a.Hv, (unsigned)a.B),
                      128, fix_smem, stream>>>(R, sstT, static_cast<__nv_bfloat16 *>(a.o), a.T, pl.seg_len,
                                        pl.nseg, a.Hv);

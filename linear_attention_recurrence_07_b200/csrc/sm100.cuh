@@ -82,6 +82,11 @@ __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, u
         ::"r"(smem_u32(dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
         : "memory");
 }
+// Brings a box of the tensor into L2 ahead of its load (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];"
+                 ::"l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, const void *src,
                                              int c0, int c1, int c2, int c3) {
     asm volatile(
@@ -133,6 +138,18 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16.  A (M x 16) sits in TMEM K-major:
+// lane = row, two bf16 per 32-bit column (even K index in the low half), so one
+// 16-wide K slice spans 8 columns.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"((uint32_t)accumulate)
+        : "memory");
+}
 // Arrives once on `bar` when all previously issued tcgen05.mma of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile(
@@ -173,6 +190,33 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
           "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
           "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
+}
+
+// 16 lanes x 256 bits, four times along the columns (32 columns): thread t of the
+// warp gets, for k = 0..3, r[4k], r[4k+1] = lane (base + t/4), columns
+// col + 8k + 2(t%4) and +1, and r[4k+2], r[4k+3] = the same columns of lane
+// (base + 8 + t/4): the layout of an m16n8 accumulator fragment.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+// Four 8x8 bf16 matrices, stored transposed: register i of thread t holds row t/4,
+// columns 2(t%4), +1 of matrix i; thread t gives the address of stored row t%8 of
+// matrix t/8, which receives column t%8 of the matrix (16 bytes).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c,
+                                                  uint32_t d) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};"
+                 ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// 32 consecutive 32-bit columns of packed data (e.g. bf16 pairs), same lane mapping.
+__device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t *r) {
+    tmem_st32(taddr, reinterpret_cast<const float *>(r));
 }
 
 // ---------------------------------------------------------------- descriptors

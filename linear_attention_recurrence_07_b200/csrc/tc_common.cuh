@@ -76,10 +76,14 @@ struct TcParams {
     // y / nseg from its start state (S0 for the first segment, zero otherwise),
     // writing o and its final state to seg_D; the B*(nseg-1) rows after them run
     // segments 1.. from S = I with v = 0, writing their outputs (M_t^T q_t) through
-    // the second output map and their final state (the segment's transition) to
-    // seg_M.
+    // the second output map (or r) and their final state (the segment's
+    // transition) to seg_M.
     int B, seg_len, nseg;
     float *seg_D, *seg_M;
+    __nv_bfloat16 *r;   // transition-row outputs [B, T - seg_len, Hv, 128], segment mode
+    __nv_bfloat16 *sst; // segment mode, or null: S_start(1)^T = bf16 of the first
+                        // segment's final state, transposed, [B, Hv, 128 (j), 128 (d)]
+    int l2_prefetch;    // 1: pull each K/Q/V tile into L2 a few chunks before its load
 };
 
 // Token rows of sequence b: rows tb .. tb + L of batch row bt of the token arrays.
@@ -368,8 +372,8 @@ __device__ __forceinline__ void compute_gates(float *gv, float a0, float a1, flo
 // g0 (columns 0-31) / g1 (32-63) held by this thread.  Decay factors are running
 // products of alpha along the row, Gam[r][x-1] = Gam[r][x] alpha_x from x = r down;
 // rows r >= 32 continue into columns x < 32 with d31[x] = Gam[31][x].
-__device__ __forceinline__ void ap_row(const float *gv, int row, float *g0, float *g1, float *sA,
-                                       unsigned char *ptile) {
+// (ap_row_values computes the row in place in g0 / g1; ap_row also stores it.)
+__device__ __forceinline__ void ap_row_values(const float *gv, int row, float *g0, float *g1) {
     const int r = row & 63;
     const bool is_a = row < 64;                // A rows: strict lower; P rows: i <= r
     const bool low = r < 32;                   // warp-uniform
@@ -399,7 +403,12 @@ __device__ __forceinline__ void ap_row(const float *gv, int row, float *g0, floa
 #pragma unroll
         for (int x = 0; x < 32; ++x) g0[x] = run * gv[GV_D31 + x] * g0[x];
     }
-    if (is_a) {
+}
+__device__ __forceinline__ void ap_row(const float *gv, int row, float *g0, float *g1, float *sA,
+                                       unsigned char *ptile) {
+    ap_row_values(gv, row, g0, g1);
+    const int r = row & 63;
+    if (row < 64) {
         float4 *dst = reinterpret_cast<float4 *>(sA + r * LDA);
 #pragma unroll
         for (int x = 0; x < 8; ++x) dst[x] = make_float4(g0[4 * x], g0[4 * x + 1], g0[4 * x + 2], g0[4 * x + 3]);

@@ -115,14 +115,19 @@ def test_prefill_tc_kernels_beyond_one_wave(kernel):
 
 
 @pytest.mark.parametrize("B,T,Hqk,Hv,seed", [(1, 385, 2, 6, 21), (2, 4096, 16, 48, 22)])
-def test_prefill_tc_kernels_agree_bitwise(B, T, Hqk, Hv, seed):
-    """The cluster kernel spreads the one-CTA kernel's arithmetic over two CTAs with
-    the same operand values and rounding points: both return the same bits."""
+def test_prefill_tc_kernels_agree(B, T, Hqk, Hv, seed):
+    """The two tensor-core kernels round the decay factors into their bf16 operands
+    at different points: the one-CTA kernel rounds Q~ = diag(gamma) Q and
+    U^T diag(g), the cluster kernel scales the fp32 product gamma_r (S^T q_r) and
+    rounds K~ = diag(g) K.  Each of those roundings is one bf16 ulp (2^-8
+    relative), so the two agree to a few ulp of the largest value."""
     d = to_dev(inputs.prefill_inputs(B, T, Hqk, Hv, dtype=torch.bfloat16, s0_std=0.3, seed=seed))
     o1, S1 = run_chunk(d, kernel="tc")
     o2, S2 = run_chunk(d, kernel="tc_cluster")
-    assert torch.equal(o1, o2), (o1.float() - o2.float()).abs().max().item()
-    assert torch.equal(S1, S2), (S1 - S2).abs().max().item()
+    err_s = (S1 - S2).abs().max().item()
+    assert err_s <= 2 ** -6 * S2.abs().max().item(), err_s
+    err = (o1.float() - o2.float()).abs().max().item()
+    assert err <= 2 ** -6 * o2.float().abs().max().item(), err
 
 
 def test_prefill_strong_and_no_decay():
