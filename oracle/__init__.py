@@ -9,6 +9,9 @@ no code with the CUDA path.
   checked against.
 * ``chunk_forward``: an fp64 numpy restatement of the chunkwise WY form, used
   by the tests as an independent reformulation that must agree with it.
+* ``backward``: fp64 gradients of every input (the adjoint of the token
+  recurrence), for the backward pass.
 """
 from .oracle import decode_step, default_threads, forward  # noqa: F401
 from .chunk_form import chunk_forward  # noqa: F401
+from .backward import backward  # noqa: F401
