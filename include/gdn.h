@@ -284,6 +284,44 @@ gdn_prefill_kernel gdn_get_prefill_kernel(void);
  */
 int gdn_prefill_kernel_for(int B, int Hv, gdn_dtype dtype);
 
+/*
+ * gdn_bwd -- gradients of the chunked / token forward with respect to every input
+ * (training).
+ *
+ * Defines: the derivative of L = sum_t <dO_t, o_t> + <dS_final, S_T> through the
+ * recurrence of "Qwen3.8-Flash-Next 技术总结 -- Qwen4 架构的探路者", section 2.1
+ * "Gated DeltaNet" (the pages give the forward only and say that the chunkwise
+ * form is what makes training efficient; the gradients are the chain rule
+ * applied to it).  Walking t down with G = dL/dS_t:
+ *   G += q_t dO_t^T;  x = G^T k_t;  w = S_{t-1}^T k_t;  r = v_t - alpha_t w
+ *   dq_t += S_t dO_t;  dk_t += beta_t G r - alpha_t beta_t S_{t-1} x;  dv_t = beta_t x
+ *   dbeta_t = x . r;  dalpha_t = <G, S_{t-1}> - beta_t x . w
+ *   G <- alpha_t (G - beta_t k_t x^T);   dS0 = G at the end.
+ * dq and dk of a QK head sum over the V heads that read it.  The forward states
+ * are recomputed inside the call (from checkpoints every 16 tokens kept in the
+ * workspace); the gradients do not depend on how the forward was evaluated.
+ *
+ * In:  q, k [B, T, Hqk, dk]; v [B, T, Hv, dv]; dO [B, T, Hv, dv], all of dtype;
+ *      alpha, beta [B, T, Hv] fp32; S0, dS_final [B, Hv, dk, dv] fp32 or NULL
+ *      (zeros).
+ * Out (fp32, overwritten): dq, dk [B, T, Hqk, dk]; dv [B, T, Hv, dv];
+ *      dalpha, dbeta [B, T, Hv]; dS0 [B, Hv, dk, dv].  Outputs must not overlap
+ *      inputs or each other.
+ * workspace: device scratch of at least gdn_bwd_workspace(B, T, Hv, dk, dv)
+ *      bytes (B * Hv * (ceil(T/16) + 16) * 64 KiB), 256-byte aligned, owned by
+ *      the caller; contents on entry do not matter; calls sharing it must not
+ *      overlap.  May be NULL when that size is 0 (T == 0).
+ * Sizes and errors as gdn_chunk_fwd (heads, dtype; B <= 65535); pointers other
+ * than the workspace 16-byte aligned.  dq, dk, dalpha, dbeta are accumulated
+ * with fp32 atomic adds, so their last bits may differ between calls.
+ */
+size_t gdn_bwd_workspace(int B, int T, int Hv, int dk, int dv);
+gdn_status gdn_bwd(const void *q, const void *k, const void *v, const float *alpha,
+                   const float *beta, const float *S0, const void *dO, const float *dS_final,
+                   float *dq, float *dk, float *dv, float *dalpha, float *dbeta, float *dS0,
+                   int B, int T, int Hqk, int Hv, int dk_, int dv_, gdn_dtype dtype,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static, NUL-terminated name of a status code. */
 const char *gdn_status_string(gdn_status status);
 

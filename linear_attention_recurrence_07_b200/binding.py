@@ -65,6 +65,11 @@ def library():
         lib.gdn_decode_step_slots.argtypes = [vp, vp, vp, fp, fp, fp, vp, vp,
                                               I, I, I, I, I, I, I, vp]
         lib.gdn_decode_step_slots.restype = I
+        lib.gdn_bwd_workspace.argtypes = [I, I, I, I, I]
+        lib.gdn_bwd_workspace.restype = ctypes.c_size_t
+        lib.gdn_bwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp,
+                                I, I, I, I, I, I, I, vp, ctypes.c_size_t, vp]
+        lib.gdn_bwd.restype = I
         lib.gdn_status_string.argtypes = [I]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_last_cuda_error.argtypes = []
@@ -235,6 +240,46 @@ def gdn_chunk_fwd_split(q, k, v, alpha, beta, S0, o, S_final, segments=0, worksp
                                          chunk, segments, _DTYPES[q.dtype], _ptr(workspace),
                                          workspace.numel(), _stream_handle(stream, dev)),
            "gdn_chunk_fwd_split")
+
+
+def bwd_workspace_bytes(B, T, Hv, dk=128, dv=128):
+    """Device scratch bytes gdn_bwd needs (C entry point ``gdn_bwd_workspace``)."""
+    return library().gdn_bwd_workspace(B, T, Hv, dk, dv)
+
+
+def gdn_bwd(q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, dS0,
+            workspace=None, stream=None):
+    """Gradients of sum <dO, o> + <dS_final, S_final> (C entry point ``gdn_bwd``).
+
+    q, k, v, dO: the forward's dtype; alpha, beta, S0, dS_final fp32 (S0 and
+    dS_final may be None).  Outputs (fp32, overwritten): dq, dk like q; dv like v;
+    dalpha, dbeta like alpha; dS0 [B, Hv, dk, dv].  ``workspace``: uint8 CUDA
+    tensor of at least bwd_workspace_bytes(...) bytes; None allocates one."""
+    B, T, Hqk, dkk = q.shape
+    Hv, dvv = v.shape[2], v.shape[3]
+    dev = q.device
+    _expect_cuda(q)
+    f32 = torch.float32
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, T, Hv, dvv), q.dtype),
+                               ("dO", dO, (B, T, Hv, dvv), q.dtype),
+                               ("alpha", alpha, (B, T, Hv), f32), ("beta", beta, (B, T, Hv), f32),
+                               ("dq", dq, q.shape, f32), ("dk", dk, q.shape, f32),
+                               ("dv", dv, (B, T, Hv, dvv), f32), ("dalpha", dalpha, (B, T, Hv), f32),
+                               ("dbeta", dbeta, (B, T, Hv), f32), ("dS0", dS0, (B, Hv, dkk, dvv), f32)):
+        _expect(t, name, shape, dt, dev)
+    for name, t in (("S0", S0), ("dS_final", dS_final)):
+        if t is not None:
+            _expect(t, name, (B, Hv, dkk, dvv), f32, dev)
+    if workspace is None:
+        workspace = torch.empty(max(bwd_workspace_bytes(B, T, Hv, dkk, dvv), 1), dtype=torch.uint8,
+                                device=dev)
+    elif workspace.device != dev or workspace.dtype != torch.uint8:
+        raise GdnError("workspace must be a uint8 tensor on the inputs' device")
+    _check(library().gdn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(dO),
+                             _ptr(dS_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(dbeta),
+                             _ptr(dS0), B, T, Hqk, Hv, dkk, dvv, _DTYPES[q.dtype], _ptr(workspace),
+                             workspace.numel(), _stream_handle(stream, dev)),
+           "gdn_bwd")
 
 
 def gdn_chunk_fwd_split_noalloc(q, k, v, alpha, beta, S0, o, S_final, segments=0, chunk=64,

@@ -48,6 +48,17 @@ bool chunk_tc_cluster_fits(int B, int Hv);   // all B * Hv clusters resident at 
 size_t chunk_tc_split_workspace(int B, int T, int Hv, int segments);
 cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *workspace,
                                   cudaStream_t stream);
+// Backward pass (gdn_bwd.cu): gradients of q, k, v, alpha, beta, S0.
+struct BwdLaunch {
+    const void *q, *k, *v, *dO;
+    const float *alpha, *beta, *S0, *dS_final;
+    float *dq, *dk, *dv, *dalpha, *dbeta, *dS0;
+    float *work;
+    int B, T, Hqk, Hv;
+};
+size_t bwd_workspace(int B, int T, int Hv);
+cudaError_t launch_bwd(const BwdLaunch &L, gdn_dtype dtype, cudaStream_t stream);
+
 // sst: null, or where the first segments write S_start(1)^T in bf16 (see TcParams).
 cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, float *segD,
                                      float *segM, __nv_bfloat16 *R, __nv_bfloat16 *sst,

@@ -35,7 +35,8 @@ def test_header_declares_the_entry_points():
     for n in ("gdn_chunk_fwd", "gdn_decode_step", "gdn_status_string", "gdn_last_cuda_error",
               "gdn_version", "gdn_set_prefill_kernel", "gdn_get_prefill_kernel",
               "gdn_prefill_kernel_for", "gdn_decode_tokens", "gdn_decode_step_slots",
-              "gdn_chunk_fwd_varlen", "gdn_chunk_fwd_split", "gdn_chunk_fwd_split_workspace"):
+              "gdn_chunk_fwd_varlen", "gdn_chunk_fwd_split", "gdn_chunk_fwd_split_workspace",
+              "gdn_bwd", "gdn_bwd_workspace"):
         assert n in names, names
 
 
@@ -222,3 +223,33 @@ def test_split_argument_checks(lib):
                                        1, 4096, 16, 48, 128, 128, 64, segments, dtype, ws, nbytes, None)
     assert call(segments=-1) == binding.GDN_ERR_INVALID_ARG
     assert call(segments=17) == binding.GDN_ERR_INVALID_ARG
+
+
+def test_bwd_workspace_sizes(lib):
+    # checkpoints every 16 tokens plus a 16-state scratch, per (sequence, head),
+    # each state 128 x 128 fp32
+    assert binding.bwd_workspace_bytes(1, 4096, 48) == 48 * (256 + 16) * 128 * 128 * 4
+    assert binding.bwd_workspace_bytes(2, 17, 6) == 2 * 6 * (2 + 16) * 128 * 128 * 4
+    assert binding.bwd_workspace_bytes(1, 0, 48) == 0
+    assert lib.gdn_bwd_workspace(1, 64, 48, 64, 128) == 0
+
+
+def test_bwd_argument_checks(lib):
+    def call(B=1, T=64, Hqk=1, Hv=1, dk=128, dv=128, dtype=1, ptr=FAKE, dS0=FAKE, ws=FAKE,
+             nbytes=1 << 40, out=FAKE):
+        return lib.gdn_bwd(ptr, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, out, FAKE, FAKE, FAKE,
+                           FAKE, dS0, B, T, Hqk, Hv, dk, dv, dtype, ws, nbytes, None)
+    assert call(B=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(T=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(dtype=3) == binding.GDN_ERR_INVALID_ARG
+    assert call(Hqk=2, Hv=3) == binding.GDN_ERR_UNSUPPORTED
+    assert call(dk=64) == binding.GDN_ERR_UNSUPPORTED
+    assert call(B=70000) == binding.GDN_ERR_UNSUPPORTED
+    assert call(ptr=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(out=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(dS0=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(ptr=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert call(ws=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(nbytes=1024) == binding.GDN_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(0x1010)) == binding.GDN_ERR_INVALID_ARG   # not 256-byte aligned
+    assert call(B=0) == binding.GDN_OK
