@@ -41,7 +41,19 @@ L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# The backward pass is plain fp32 CUDA-core arithmetic: its ceiling is the FP32 rate,
+# 148 SMs x 128 FP32 lanes x 2 FLOP (FMA) x 1965 MHz (the B200's max SM clock).
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
 # ----------------------------------------------------------------------------- counts
+def bwd_flops_per_token(w):
+    """fp32 FLOPs per token and V head the gradients need at the least: one forward
+    step to rebuild S_{t-1} (S^T k, rank-1 update: 5 dk dv) and the backward step
+    (G += q dO^T, G^T k, S^T k, <G, S>, S_t dO, G r, S x, the G update: 16 dk dv)."""
+    return 21 * w.dk * w.dv * w.Hv
+
+
 def prefill_flops_per_token(w, C=64):
     """Algorithmic FLOPs of the chunkwise form per token: per V head the products
     U~, W (2C(dk+dv)), U = U~ - W S, Q S, S update (2 dk dv each) and the masked
@@ -341,6 +353,29 @@ def time_calls(call, steps, warmup, world):
             "launches": steps, "window": (wall0, wall1)}
 
 
+def time_backward(w, steps, warmup, world):
+    """gdn_bwd on the prefill workload: dO random, no S0 / dS_final (the
+    workload's own S0 is none either)."""
+    d = inputs.workload_inputs(w, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(w.seed + 7)
+    dO = torch.randn((w.B, w.T, w.Hv, w.dv), generator=g, device="cuda").to(w.dtype)
+    f32 = dict(dtype=torch.float32, device="cuda")
+    dq = torch.empty((w.B, w.T, w.Hqk, w.dk), **f32)
+    dk = torch.empty_like(dq)
+    dv = torch.empty((w.B, w.T, w.Hv, w.dv), **f32)
+    da = torch.empty((w.B, w.T, w.Hv), **f32)
+    db = torch.empty_like(da)
+    dS0 = torch.empty((w.B, w.Hv, w.dk, w.dv), **f32)
+    ws = torch.empty(binding.bwd_workspace_bytes(w.B, w.T, w.Hv, w.dk, w.dv), dtype=torch.uint8,
+                     device="cuda")
+
+    def call(i):
+        binding.gdn_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], dO, None,
+                        dq, dk, dv, da, db, dS0, workspace=ws)
+
+    return time_calls(call, steps, warmup, world)
+
+
 def time_verify(w, steps, warmup, world):
     """gdn_decode_tokens: n draft tokens for each of B sequences, state in place,
     the state after every token written to S_steps."""
@@ -460,6 +495,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--verify-steps", type=int, default=50)
     ap.add_argument("--varlen-steps", type=int, default=20)
+    ap.add_argument("--bwd-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--prefill-kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto",
                     help="prefill kernel to time (default: the library's own choice)")
@@ -493,6 +529,7 @@ def main():
     with ClockSampler(local) as clocks2:
         ver = time_verify(wv, args.verify_steps, args.warmup, world)
         vl = time_varlen(wl, args.varlen_steps, args.warmup, world)
+        bw = time_backward(w, args.bwd_steps, 3, world)
     e2e = time_prefill_e2e(w, args.e2e_steps, 3, world, split=segs)
 
     tokens_per_step = w.B * w.T
@@ -555,6 +592,17 @@ def main():
                              peak_source=f"{peak_src} copy bandwidth",
                              algorithmic_bytes_per_launch=verify_bytes_per_call(wv)),
             "gpu_launches": ver["launches"],
+        },
+        "backward": {
+            "metric": "backward tokens/s (gdn_bwd: dq, dk, dv, dalpha, dbeta, dS0)",
+            "workload": w.name, "B": w.B, "T": w.T,
+            "value": job_throughput(tokens_per_step, args.bwd_steps, world, bw["total_ms"]),
+            "unit": "tokens/s", "ms_per_call": bw["total_ms"] / args.bwd_steps,
+            "roofline": dict(roofline("alu", bwd_flops_per_token(w) * tokens_per_step
+                                      / (bw["per_launch_ms"] * 1e-3) / 1e12,
+                                      FP32_ALU_TFLOPS, "TFLOP/s", None),
+                             peak_source="fp32 lanes x max SM clock (148 x 128 x 2 x 1965 MHz)"),
+            "gpu_launches": bw["launches"],
         },
         "varlen_prefill": {
             "metric": "packed-prefill tokens/s (gdn_chunk_fwd_varlen)",

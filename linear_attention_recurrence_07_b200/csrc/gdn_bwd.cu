@@ -276,16 +276,26 @@ bwd_kernel(const BwdArgs<T> A)
             // row sums of this thread: S_t dO, G r, S_{t-1} x; and x . r, x . w
             float sdo = 0.f, gr = 0.f, px = 0.f, xr = 0.f, xw = 0.f;
 #pragma unroll
-            for (int c = 0; c < kCols; ++c) {
-                const float w = s_tot[0][c], x = s_tot[1][c], v = blk.v[i][c], o = blk.dO[i][c];
-                const float st = a * (P[c] - bk * w) + bk * v;       // S_t
-                const float r = v - a * w;
-                sdo = fmaf(st, o, sdo);
-                gr = fmaf(G[c], r, gr);
-                px = fmaf(P[c], x, px);
-                xr = fmaf(x, r, xr);
-                xw = fmaf(x, w, xw);
-                G[c] = a * (G[c] - bk * x);                          // gradient w.r.t. S_{t-1}
+            for (int c4 = 0; c4 < kCols; c4 += 4) {
+                const float4 w4 = *reinterpret_cast<const float4 *>(&s_tot[0][c4]);
+                const float4 x4 = *reinterpret_cast<const float4 *>(&s_tot[1][c4]);
+                const float4 v4 = *reinterpret_cast<const float4 *>(&blk.v[i][c4]);
+                const float4 o4 = *reinterpret_cast<const float4 *>(&blk.dO[i][c4]);
+                const float wv[4] = {w4.x, w4.y, w4.z, w4.w}, xv[4] = {x4.x, x4.y, x4.z, x4.w};
+                const float vv[4] = {v4.x, v4.y, v4.z, v4.w}, ov[4] = {o4.x, o4.y, o4.z, o4.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int c = c4 + e;
+                    const float w = wv[e], x = xv[e], v = vv[e];
+                    const float st = a * (P[c] - bk * w) + bk * v;   // S_t
+                    const float r = v - a * w;
+                    sdo = fmaf(st, ov[e], sdo);
+                    gr = fmaf(G[c], r, gr);
+                    px = fmaf(P[c], x, px);
+                    xr = fmaf(x, r, xr);
+                    xw = fmaf(x, w, xw);
+                    G[c] = a * (G[c] - bk * x);                      // gradient w.r.t. S_{t-1}
+                }
             }
             const size_t row = (size_t)b * nT + t;
             const size_t qk = (row * A.Hqk + hq) * kHeadDim + d;
