@@ -27,15 +27,18 @@ namespace {
 constexpr int kChainThreads = 256;
 constexpr int kChainCols = 32;            // state columns per CTA of seg_chain_kernel
 constexpr int kFixRows = 64;              // output rows per tile of out_fix_kernel
-constexpr int kFixTiles = 4;              // tiles per CTA (the S_start tile is staged once)
+constexpr int kFixTiles = 2;              // tiles per CTA (the S_start tile is staged once)
 constexpr int kLdR = kHeadDim + 8;        // padded bf16 row strides in shared memory
 constexpr int kLdS = kHeadDim + 8;
+constexpr int kLdM = kHeadDim + 1;        // padded row stride of the staged M (floats): the
+                                          // threads of a warp read rows i0 + x at one d, in
+                                          // distinct banks
 
 // S_start of every later segment, in order: S_start(1) = D_0, S_start(k+1) =
 // M_k S_start(k) + D_k (fp32); writes S_start(k)^T in bf16 ([j][d]) for k >= 1 if
 // write_sst, and the final state.  Columns of the state evolve independently, so
 // one CTA of kThreads threads takes kCols columns of one (head, sequence): M_k
-// whole and its columns of S in shared memory (chain_smem, kHeadDim * (kHeadDim +
+// whole and its columns of S in shared memory (chain_smem, kHeadDim * (kLdM +
 // kCols) floats); each thread owns a 4 x 4 tile of the product.
 template <int kThreads, int kCols>
 __device__ __forceinline__ void chain_columns(const float *__restrict__ segD, const float *__restrict__ segM,
@@ -44,8 +47,8 @@ __device__ __forceinline__ void chain_columns(const float *__restrict__ segD, co
                                               float *chain_smem)
 {
     static_assert((kHeadDim / 4) * (kCols / 4) == kThreads, "one 4 x 4 tile per thread");
-    float *Ms = chain_smem;                        // M_k: [i][d]
-    float *Sc = chain_smem + kHeadDim * kHeadDim;  // S_start columns: [d][c], c < kCols
+    float *Ms = chain_smem;                        // M_k: [i][d], row stride kLdM
+    float *Sc = chain_smem + kHeadDim * kLdM;      // S_start columns: [d][c], c < kCols
     const int tid = threadIdx.x;
     const size_t hs = (size_t)kHeadDim * kHeadDim;
     const float *D0 = segD + (((size_t)b * nseg + 0) * Hv + h) * hs;
@@ -62,8 +65,11 @@ __device__ __forceinline__ void chain_columns(const float *__restrict__ segD, co
         __nv_bfloat16 *dst = sstT + (((size_t)b * (nseg - 1) + (k - 1)) * Hv + h) * hs;
         __syncthreads();                           // Sc complete; Ms free
 #pragma unroll 16
-        for (int e = tid; e < kHeadDim * kHeadDim / 4; e += kThreads)
-            reinterpret_cast<float4 *>(Ms)[e] = reinterpret_cast<const float4 *>(Mk)[e];
+        for (int e = tid; e < kHeadDim * kHeadDim / 4; e += kThreads) {
+            const float4 v = reinterpret_cast<const float4 *>(Mk)[e];
+            float *row = Ms + (e / (kHeadDim / 4)) * kLdM + 4 * (e % (kHeadDim / 4));
+            row[0] = v.x; row[1] = v.y; row[2] = v.z; row[3] = v.w;
+        }
         // S_start(k)^T for the output fix-up: row j = j_base + c, 128 bf16 (d)
         for (int e = tid; write_sst && e < kCols * (kHeadDim / 8); e += kThreads) {
             const int c = e / (kHeadDim / 8), d8 = 8 * (e % (kHeadDim / 8));
@@ -83,7 +89,7 @@ __device__ __forceinline__ void chain_columns(const float *__restrict__ segD, co
         for (int d = 0; d < kHeadDim; ++d) {
             float mi[4];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) mi[x] = Ms[(i0 + x) * kHeadDim + d];
+            for (int x = 0; x < 4; ++x) mi[x] = Ms[(i0 + x) * kLdM + d];
             const float4 sv = *reinterpret_cast<const float4 *>(&Sc[d * kCols + c0]);
             const float sj[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
@@ -303,7 +309,7 @@ cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *worksp
     if (pl.nseg == 2) {
         cudaError_t err = launch_chunk_tc_segments(a, pl.seg_len, pl.nseg, segD, segM, R, sstT, stream);
         if (err != cudaSuccess) return err;
-        const size_t state_smem = ((size_t)kHeadDim * kHeadDim + (size_t)kHeadDim * kStateCols) * sizeof(float);
+        const size_t state_smem = ((size_t)kHeadDim * kLdM + (size_t)kHeadDim * kStateCols) * sizeof(float);
         const size_t smem = state_smem > fix_smem ? state_smem : fix_smem;
         err = cudaFuncSetAttribute(split2_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
@@ -314,7 +320,7 @@ cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *worksp
     }
     cudaError_t err = launch_chunk_tc_segments(a, pl.seg_len, pl.nseg, segD, segM, R, nullptr, stream);
     if (err != cudaSuccess) return err;
-    const size_t chain_smem = ((size_t)kHeadDim * kHeadDim + (size_t)kHeadDim * kChainCols) * sizeof(float);
+    const size_t chain_smem = ((size_t)kHeadDim * kLdM + (size_t)kHeadDim * kChainCols) * sizeof(float);
     err = cudaFuncSetAttribute(seg_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)chain_smem);
     if (err != cudaSuccess) return err;
