@@ -5,6 +5,7 @@
     python -m linear_attention_recurrence_07_b200.profile_cases decode [--B 64] [--launches 5]
     python -m linear_attention_recurrence_07_b200.profile_cases prefill-fp32 [--T 1024]
     python -m linear_attention_recurrence_07_b200.profile_cases prefill-split [--segments 0]
+    python -m linear_attention_recurrence_07_b200.profile_cases bwd [--T 4096] [--launches 3]
 
 Each case builds its seeded inputs on the GPU, runs the entry point `--launches`
 times and synchronizes; it prints nothing but "ok".  Point a profiler at it with
@@ -20,7 +21,7 @@ from . import binding, inputs
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["prefill", "decode", "prefill-fp32", "prefill-split"])
+    ap.add_argument("case", choices=["prefill", "decode", "prefill-fp32", "prefill-split", "bwd"])
     ap.add_argument("--segments", type=int, default=0)
     ap.add_argument("--T", type=int, default=None)
     ap.add_argument("--B", type=int, default=None)
@@ -46,6 +47,22 @@ def main():
                                             o, S, segments=args.segments, workspace=ws)
             else:
                 binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S)
+    elif args.case == "bwd":
+        w = inputs.PREFILL_4K
+        T = args.T or w.T
+        B = args.B or w.B
+        d = inputs.prefill_inputs(B, T, w.Hqk, w.Hv, w.dk, w.dv, w.dtype, w.log_alpha,
+                                  w.s0_std, w.seed, "cuda")
+        g = torch.Generator(device="cuda").manual_seed(w.seed + 7)
+        dO = torch.randn((B, T, w.Hv, w.dv), generator=g, device="cuda").to(w.dtype)
+        f32 = dict(dtype=torch.float32, device="cuda")
+        grads = [torch.empty((B, T, w.Hqk, w.dk), **f32), torch.empty((B, T, w.Hqk, w.dk), **f32),
+                 torch.empty((B, T, w.Hv, w.dv), **f32), torch.empty((B, T, w.Hv), **f32),
+                 torch.empty((B, T, w.Hv), **f32), torch.empty((B, w.Hv, w.dk, w.dv), **f32)]
+        ws = torch.empty(max(binding.bwd_workspace_bytes(B, T, w.Hv), 1), dtype=torch.uint8, device="cuda")
+        for _ in range(args.launches):
+            binding.gdn_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], dO, None, *grads,
+                            workspace=ws)
     else:
         w = inputs.DECODE_B256
         B = args.B or 64
