@@ -11,7 +11,10 @@ no code with the CUDA path.
   by the tests as an independent reformulation that must agree with it.
 * ``backward``: fp64 gradients of every input (the adjoint of the token
   recurrence), for the backward pass.
+* ``chunk_backward``: the same gradients through the chunkwise WY form (the
+  blocked algebra of a chunked backward kernel), required to agree with it.
 """
 from .oracle import decode_step, default_threads, forward  # noqa: F401
 from .chunk_form import chunk_forward  # noqa: F401
 from .backward import backward  # noqa: F401
+from .chunk_backward import chunk_backward  # noqa: F401

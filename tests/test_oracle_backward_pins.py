@@ -123,3 +123,27 @@ def test_backward_head_range_selects_heads():
                     h_range=(1, 2))
     np.testing.assert_allclose(part[2][:, :, 1], full[2][:, :, 1], rtol=1e-12)
     np.testing.assert_array_equal(part[2][:, :, 0], 0.0)
+
+
+@pytest.mark.parametrize("chunk", [4, 7, 64])
+def test_chunk_backward_agrees_with_token_adjoint(chunk):
+    """The chunkwise-WY backward (the blocked algebra a chunked kernel follows,
+    gate gradients through the cumulative log-decays included) gives the token
+    adjoint's gradients; several chunks, a ragged tail, shared QK heads."""
+    from oracle.chunk_backward import chunk_backward
+    d = _problem(2, 29, 1, 2, 6, 5, seed=20 + chunk)
+    ref = backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["dO"], d["S0"], d["dS_final"])
+    got = chunk_backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["dO"], d["S0"], d["dS_final"],
+                         chunk=chunk)
+    for name, g, r in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dS0"), got, ref):
+        np.testing.assert_allclose(g, r, rtol=1e-9, atol=1e-11, err_msg=name)
+
+
+def test_chunk_backward_head_dim_128_and_no_states():
+    from oracle.chunk_backward import chunk_backward
+    d = _problem(1, 70, 1, 1, 128, 128, seed=33, s0=False, dsf=False)
+    ref = backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["dO"])
+    got = chunk_backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["dO"], chunk=64)
+    for name, g, r in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dS0"), got, ref):
+        scale = max(np.abs(r).max(), 1e-300)
+        assert np.abs(g - r).max() <= 1e-9 * scale, name
