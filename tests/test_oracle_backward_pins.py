@@ -147,3 +147,104 @@ def test_chunk_backward_head_dim_128_and_no_states():
     for name, g, r in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dS0"), got, ref):
         scale = max(np.abs(r).max(), 1e-300)
         assert np.abs(g - r).max() <= 1e-9 * scale, name
+
+
+# --------------------------------------------------------------------------- mutants
+def _adjoint(mistake=None):
+    """The adjoint walk with one planted mistake, to check that the pins catch it."""
+    def impl(q, k, v, alpha, beta, dO, S0=None, dS_final=None):
+        B, T, Hqk, dk = q.shape
+        Hv, dv = v.shape[2], v.shape[3]
+        g = Hv // Hqk
+        dq, dkk, dvv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
+        dal, dbe = np.zeros_like(alpha), np.zeros_like(beta)
+        dS0 = np.zeros((B, Hv, dk, dv))
+        for b in range(B):
+            for h in range(Hv):
+                hq = h // g
+                kk, qq = k[b, :, hq], q[b, :, hq]
+                s0 = np.zeros((dk, dv)) if S0 is None else S0[b, h]
+                S = forward_states(kk, v[b, :, h], alpha[b, :, h], beta[b, :, h], s0)
+                G = np.zeros((dk, dv)) if dS_final is None else dS_final[b, h].copy()
+                for t in range(T - 1, -1, -1):
+                    a, be = alpha[b, t, h], beta[b, t, h]
+                    kt, do = kk[t], dO[b, t, h]
+                    P = S[t - 1]
+                    if mistake != "readout_grad_after_update":
+                        G = G + np.outer(qq[t], do)
+                    dq[b, t, hq] += (P if mistake == "dq_from_previous_state" else S[t]) @ do
+                    x, w = G.T @ kt, P.T @ kt
+                    r = v[b, t, h] - a * w
+                    dvv[b, t, h] = x if mistake == "dv_without_beta" else be * x
+                    dbe[b, t, h] = x @ (v[b, t, h] if mistake == "dbeta_without_correction" else r)
+                    dal[b, t, h] = np.sum(G * P) - (0.0 if mistake == "dalpha_without_write_term" else be * (x @ w))
+                    sgn = -1.0 if mistake == "dk_sign" else 1.0
+                    dkk[b, t, hq] += be * (G @ r) - sgn * a * be * (P @ x)
+                    if mistake == "G_without_decay":
+                        G = G - be * np.outer(kt, x)
+                    else:
+                        G = a * (G - be * np.outer(kt, x))
+                    if mistake == "readout_grad_after_update":
+                        G = G + np.outer(qq[t], do)
+                dS0[b, h] = G
+        return dq, dkk, dvv, dal, dbe, dS0
+    return impl
+
+
+def _pin_finite_differences(impl):
+    d = _problem(1, 4, 1, 2, 3, 2, seed=5)
+    grads = impl(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["dO"], d["S0"], d["dS_final"])
+    eps = 1e-6
+    for name, grad in zip(["q", "k", "v", "alpha", "beta", "S0"], grads):
+        x = d[name]
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            keep = x[idx]
+            x[idx] = keep + eps
+            lp = _loss(d)
+            x[idx] = keep - eps
+            lm = _loss(d)
+            x[idx] = keep
+            fd[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, fd, rtol=1e-6, atol=1e-7, err_msg=name)
+
+
+def _pin_closed_form(impl):
+    d = _problem(1, 5, 1, 1, 3, 2, seed=6)
+    d["alpha"][:] = 1.0
+    d["beta"][:] = 0.0
+    dq, dk, dv, dal, dbe, dS0 = impl(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["dO"], d["S0"],
+                                     d["dS_final"])
+    S0, q, k, v, dO = d["S0"][0, 0], d["q"][0, :, 0], d["k"][0, :, 0], d["v"][0, :, 0], d["dO"][0, :, 0]
+    np.testing.assert_allclose(dk, 0.0, atol=1e-12)
+    np.testing.assert_allclose(dv, 0.0, atol=1e-12)
+    G = d["dS_final"][0, 0].copy()
+    for t in range(4, -1, -1):
+        G = G + np.outer(q[t], dO[t])
+        np.testing.assert_allclose(dq[0, t, 0], S0 @ dO[t], rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dbe[0, t, 0], k[t] @ G @ (v[t] - S0.T @ k[t]), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(dal[0, t, 0], np.sum(G * S0), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dS0[0, 0], G, rtol=1e-10, atol=1e-12)
+
+
+BACKWARD_PINS = [_pin_finite_differences, _pin_closed_form]
+BACKWARD_MUTANTS = ["readout_grad_after_update", "dq_from_previous_state", "dv_without_beta",
+                    "dbeta_without_correction", "dalpha_without_write_term", "dk_sign",
+                    "G_without_decay"]
+
+
+def test_backward_oracle_and_unmutated_adjoint_pass_pins():
+    for pin in BACKWARD_PINS:
+        pin(backward)
+        pin(_adjoint(None))
+
+
+@pytest.mark.parametrize("mistake", BACKWARD_MUTANTS)
+def test_backward_pins_catch_mutants(mistake):
+    caught = []
+    for pin in BACKWARD_PINS:
+        try:
+            pin(_adjoint(mistake))
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin rejects the planted mistake {mistake!r}"
