@@ -54,7 +54,8 @@ typedef enum {
     GDN_OK = 0,
     GDN_ERR_INVALID_ARG = 1,
     GDN_ERR_UNSUPPORTED = 2,
-    GDN_ERR_CUDA = 3
+    GDN_ERR_CUDA = 3,
+    GDN_ERR_TIMEOUT = 4   /* a bounded wait inside a kernel gave up (see gdn_device_status) */
 } gdn_status;
 
 typedef enum {
@@ -149,6 +150,68 @@ gdn_status gdn_chunk_fwd_split(const void *q, const void *k, const void *v,
                                int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
                                int segments, gdn_dtype dtype, void *workspace,
                                size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_chunk_fwd_pipelined -- gdn_chunk_fwd with the state-independent part of
+ * every chunk prepared on SMs of its own and streamed to the SMs that carry the
+ * states (one cooperative launch).
+ *
+ * Defines: the same function as gdn_chunk_fwd (section 2.1 "Gated DeltaNet" of
+ * the page above, chunkwise WY evaluation).  Of each chunk's WY work, the gates,
+ * the grams, the masked decay products, the triangular inverse (I + A)^-1 and
+ * the scaled inverses do not depend on the state; "prep" CTAs compute them (the
+ * grams once per QK head group) and pass them through a ring in the workspace
+ * to "chain" CTAs, which keep each (sequence, V head)'s fp32 state in tensor
+ * memory and run the state-dependent products chunk after chunk.  With few
+ * sequences x heads (long prompts at small batch) most SMs prepare and the
+ * chains run at the speed of their own products; with many, chains and prep
+ * share the SMs.
+ *
+ * Arguments as gdn_chunk_fwd, plus:
+ *   opts       NULL for the defaults, or:
+ *                chain_ctas         CTAs that carry states (0 = automatic: all
+ *                                   B*Hv heads at once when that is at most half
+ *                                   of the SMs, else about 60% of them); rounded
+ *                                   down to a multiple of Hv/Hqk
+ *                wait_limit_cycles  SM clocks any wait inside the kernel may take
+ *                                   before it gives up (0 = 2^32, about 2 s); a
+ *                                   wait that gives up makes every CTA stop and
+ *                                   is reported by gdn_device_status (the
+ *                                   outputs are then undefined)
+ *   workspace  device scratch of at least gdn_chunk_fwd_pipelined_workspace(...)
+ *              bytes (for this device), 256-byte aligned, owned by the caller;
+ *              its contents on entry do not matter; calls sharing it must not
+ *              overlap.
+ * Only GDN_BF16 takes this path; GDN_F32 (and B == 0 or T == 0) is
+ * gdn_chunk_fwd, workspace unused.  Needs all its CTAs resident at once (one per
+ * SM); if other work on the device prevents that, the launch waits for it, and a
+ * device too small returns GDN_ERR_CUDA.  Rounding matches gdn_chunk_fwd's
+ * tensor-core kernel (same products in the same precisions).
+ */
+typedef struct {
+    int chain_ctas;
+    long long wait_limit_cycles;
+} gdn_pipeline_options;
+
+size_t gdn_chunk_fwd_pipelined_workspace(int B, int Hqk, int Hv, int dk, int dv);
+gdn_status gdn_chunk_fwd_pipelined(const void *q, const void *k, const void *v,
+                                   const float *alpha, const float *beta, const float *S0,
+                                   void *o, float *S_final,
+                                   int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                                   gdn_dtype dtype, const gdn_pipeline_options *opts,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * gdn_device_status -- waits for `stream`, then reports and clears the device
+ * error words of the tensor-core prefill kernels.  Returns GDN_ERR_TIMEOUT if a
+ * bounded wait inside any of them gave up since the last call (on any stream:
+ * the words are per library, not per call), GDN_ERR_CUDA if the stream reports
+ * an error, else GDN_OK.  The kernels never trap or hang: a wait that gives up
+ * ends its launch early, leaves its outputs undefined and the device usable.
+ * This call synchronises, so call it where a check is wanted (tests, after a
+ * batch), not on every step.
+ */
+gdn_status gdn_device_status(void *stream);
 
 /*
  * gdn_chunk_fwd_split_noalloc -- gdn_chunk_fwd_split for callers that cannot

@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIBRARY_PATH = os.path.join(_PKG, "libgdn.so")
 
-GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA = 0, 1, 2, 3
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT = 0, 1, 2, 3, 4
 GDN_F32, GDN_BF16 = 0, 1
 _DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
 # gdn_prefill_kernel values
@@ -31,6 +31,11 @@ class GdnError(RuntimeError):
 
 
 _lib = None
+
+
+class PipelineOptions(ctypes.Structure):
+    """gdn_pipeline_options: chain_ctas (0 = automatic), wait_limit_cycles (0 = 2^32)."""
+    _fields_ = [("chain_ctas", ctypes.c_int), ("wait_limit_cycles", ctypes.c_longlong)]
 
 
 def library():
@@ -70,6 +75,14 @@ def library():
         lib.gdn_bwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp,
                                 I, I, I, I, I, I, I, vp, ctypes.c_size_t, vp]
         lib.gdn_bwd.restype = I
+        lib.gdn_chunk_fwd_pipelined_workspace.argtypes = [I, I, I, I, I]
+        lib.gdn_chunk_fwd_pipelined_workspace.restype = ctypes.c_size_t
+        lib.gdn_chunk_fwd_pipelined.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
+                                                I, I, I, I, I, I, I, I,
+                                                ctypes.POINTER(PipelineOptions), vp, ctypes.c_size_t, vp]
+        lib.gdn_chunk_fwd_pipelined.restype = I
+        lib.gdn_device_status.argtypes = [vp]
+        lib.gdn_device_status.restype = I
         lib.gdn_status_string.argtypes = [I]
         lib.gdn_status_string.restype = ctypes.c_char_p
         lib.gdn_last_cuda_error.argtypes = []
@@ -84,6 +97,13 @@ def library():
         lib.gdn_prefill_kernel_for.restype = I
         _lib = lib
     return _lib
+
+
+def _call(dev, fn, *args):
+    """Runs the C entry point with ``dev`` as the current CUDA device (the library
+    looks up per-device state, such as static scratch, on the current device)."""
+    with torch.cuda.device(dev):
+        return fn(*args)
 
 
 def _check(status, what):
@@ -144,7 +164,7 @@ def gdn_chunk_fwd(q, k, v, alpha, beta, S0, o, S_final, chunk=64, stream=None):
     for name, t in (("S0", S0), ("S_final", S_final)):
         if t is not None:
             _expect(t, name, (B, Hv, dk, dv), torch.float32, dev)
-    _check(library().gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+    _check(_call(dev, library().gdn_chunk_fwd, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
                                    _ptr(o), _ptr(S_final), B, T, Hqk, Hv, dk, dv, chunk,
                                    _DTYPES[q.dtype], _stream_handle(stream, dev)),
            "gdn_chunk_fwd")
@@ -165,7 +185,7 @@ def gdn_decode_step(q, k, v, alpha, beta, S, o, S_new, stream=None):
                                ("S", S, (B, Hv, dk, dv), torch.float32),
                                ("S_new", S_new, (B, Hv, dk, dv), torch.float32)):
         _expect(t, name, shape, dt, dev)
-    _check(library().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+    _check(_call(dev, library().gdn_decode_step, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
                                      _ptr(o), _ptr(S_new), B, Hqk, Hv, dk, dv,
                                      _DTYPES[q.dtype], _stream_handle(stream, dev)),
            "gdn_decode_step")
@@ -235,7 +255,7 @@ def gdn_chunk_fwd_split(q, k, v, alpha, beta, S0, o, S_final, segments=0, worksp
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     elif workspace.device != dev or workspace.dtype != torch.uint8:
         raise GdnError("workspace must be a uint8 tensor on the inputs' device")
-    _check(library().gdn_chunk_fwd_split(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+    _check(_call(dev, library().gdn_chunk_fwd_split, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                          _ptr(S0), _ptr(o), _ptr(S_final), B, T, Hqk, Hv, dk, dv,
                                          chunk, segments, _DTYPES[q.dtype], _ptr(workspace),
                                          workspace.numel(), _stream_handle(stream, dev)),
@@ -275,7 +295,7 @@ def gdn_bwd(q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, d
                                 device=dev)
     elif workspace.device != dev or workspace.dtype != torch.uint8:
         raise GdnError("workspace must be a uint8 tensor on the inputs' device")
-    _check(library().gdn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(dO),
+    _check(_call(dev, library().gdn_bwd, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(dO),
                              _ptr(dS_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(dbeta),
                              _ptr(dS0), B, T, Hqk, Hv, dkk, dvv, _DTYPES[q.dtype], _ptr(workspace),
                              workspace.numel(), _stream_handle(stream, dev)),
@@ -298,7 +318,7 @@ def gdn_chunk_fwd_split_noalloc(q, k, v, alpha, beta, S0, o, S_final, segments=0
     for name, t in (("S0", S0), ("S_final", S_final)):
         if t is not None:
             _expect(t, name, (B, Hv, dk, dv), torch.float32, dev)
-    _check(library().gdn_chunk_fwd_split_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+    _check(_call(dev, library().gdn_chunk_fwd_split_noalloc, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                                  _ptr(S0), _ptr(o), _ptr(S_final), B, T, Hqk, Hv,
                                                  dk, dv, chunk, segments, _DTYPES[q.dtype],
                                                  _stream_handle(stream, dev)),
@@ -325,7 +345,7 @@ def gdn_chunk_fwd_varlen(q, k, v, alpha, beta, S0, o, S_final, cu_seqlens, chunk
     for name, t in (("S0", S0), ("S_final", S_final)):
         if t is not None:
             _expect(t, name, (N, Hv, dk, dv), torch.float32, dev)
-    _check(library().gdn_chunk_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+    _check(_call(dev, library().gdn_chunk_fwd_varlen, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                           _ptr(S0), _ptr(o), _ptr(S_final), _ptr(cu_seqlens),
                                           N, T, Hqk, Hv, dk, dv, chunk, _DTYPES[q.dtype],
                                           _stream_handle(stream, dev)),
@@ -350,7 +370,7 @@ def gdn_decode_tokens(q, k, v, alpha, beta, S, o, S_new, S_steps=None, stream=No
         _expect(t, name, shape, dt, dev)
     if S_steps is not None:
         _expect(S_steps, "S_steps", (B, n, Hv, dk, dv), torch.float32, dev)
-    _check(library().gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
+    _check(_call(dev, library().gdn_decode_tokens, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S),
                                        _ptr(o), _ptr(S_new), _ptr(S_steps), B, n, Hqk, Hv, dk, dv,
                                        _DTYPES[q.dtype], _stream_handle(stream, dev)),
            "gdn_decode_tokens")
@@ -373,11 +393,58 @@ def gdn_decode_step_slots(q, k, v, alpha, beta, state_pool, slots, o, stream=Non
                                ("state_pool", state_pool, (n_slots, Hv, dk, dv), torch.float32),
                                ("slots", slots, (B,), torch.int32)):
         _expect(t, name, shape, dt, dev)
-    _check(library().gdn_decode_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
+    _check(_call(dev, library().gdn_decode_step_slots, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta),
                                            _ptr(state_pool), _ptr(slots), _ptr(o), B, n_slots,
                                            Hqk, Hv, dk, dv, _DTYPES[q.dtype],
                                            _stream_handle(stream, dev)),
            "gdn_decode_step_slots")
+
+
+def pipelined_workspace_bytes(B, Hqk, Hv, dk=128, dv=128):
+    """Device scratch bytes gdn_chunk_fwd_pipelined needs on the current device (C
+    entry point ``gdn_chunk_fwd_pipelined_workspace``)."""
+    return library().gdn_chunk_fwd_pipelined_workspace(B, Hqk, Hv, dk, dv)
+
+
+def gdn_chunk_fwd_pipelined(q, k, v, alpha, beta, S0, o, S_final, chain_ctas=0,
+                            wait_limit_cycles=0, workspace=None, chunk=64, stream=None):
+    """Prefill with the chunks' WY preparation streamed from SMs of its own (C entry
+    point ``gdn_chunk_fwd_pipelined``): the same arguments and results as
+    gdn_chunk_fwd.  ``workspace`` is a uint8 CUDA tensor of at least
+    pipelined_workspace_bytes(...) bytes; None allocates one for this call."""
+    B, T, Hqk, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dev = q.device
+    _expect_cuda(q)
+    for name, t, shape, dt in (("k", k, q.shape, q.dtype), ("v", v, (B, T, Hv, dv), q.dtype),
+                               ("o", o, (B, T, Hv, dv), q.dtype),
+                               ("alpha", alpha, (B, T, Hv), torch.float32),
+                               ("beta", beta, (B, T, Hv), torch.float32)):
+        _expect(t, name, shape, dt, dev)
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None:
+            _expect(t, name, (B, Hv, dk, dv), torch.float32, dev)
+    if workspace is None:
+        with torch.cuda.device(dev):
+            need = pipelined_workspace_bytes(B, Hqk, Hv, dk, dv)
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    elif workspace.device != dev or workspace.dtype != torch.uint8:
+        raise GdnError("workspace must be a uint8 tensor on the inputs' device")
+    opts = PipelineOptions(int(chain_ctas), int(wait_limit_cycles))
+    _check(_call(dev, library().gdn_chunk_fwd_pipelined, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                 _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_final), B, T, Hqk, Hv, dk, dv, chunk,
+                 _DTYPES[q.dtype], ctypes.byref(opts), _ptr(workspace), workspace.numel(),
+                 _stream_handle(stream, dev)),
+           "gdn_chunk_fwd_pipelined")
+
+
+def device_status(stream=None, device=None):
+    """Waits for ``stream`` and returns (and clears) the library's device error
+    state as a status name: "GDN_OK", or "GDN_ERR_TIMEOUT" if a bounded wait inside
+    a kernel gave up (C entry point ``gdn_device_status``)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    code = _call(dev, library().gdn_device_status, _stream_handle(stream, dev))
+    return library().gdn_status_string(code).decode()
 
 
 def chunk_fwd(q, k, v, alpha, beta, S0=None, chunk=64, stream=None):

@@ -263,6 +263,54 @@ gdn_status gdn_chunk_fwd_split(const void *q, const void *k, const void *v,
                                                   static_cast<cudaStream_t>(stream)));
 }
 
+size_t gdn_chunk_fwd_pipelined_workspace(int B, int Hqk, int Hv, int dk, int dv)
+{
+    if (dk != gdn::kHeadDim || dv != gdn::kHeadDim) return 0;
+    return gdn::chunk_pipe_workspace(B, Hqk, Hv);
+}
+
+gdn_status gdn_chunk_fwd_pipelined(const void *q, const void *k, const void *v,
+                                   const float *alpha, const float *beta, const float *S0,
+                                   void *o, float *S_final,
+                                   int B, int T, int Hqk, int Hv, int dk, int dv, int chunk,
+                                   gdn_dtype dtype, const gdn_pipeline_options *opts,
+                                   void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (opts && (opts->chain_ctas < 0 || opts->wait_limit_cycles < 0)) return GDN_ERR_INVALID_ARG;
+    // fp32 inputs, empty problems and builds without the tensor-map encoder take the
+    // plain prefill (same function; the workspace is not used)
+    if (dtype != GDN_BF16 || B <= 0 || T <= 0 || !gdn::chunk_tc_available())
+        return gdn_chunk_fwd(q, k, v, alpha, beta, S0, o, S_final, B, T, Hqk, Hv, dk, dv, chunk,
+                             dtype, stream);
+    gdn_status st = check_heads(Hqk, Hv, dk, dv);
+    if (st != GDN_OK) return st;
+    if (chunk != gdn::kChunk) return GDN_ERR_UNSUPPORTED;
+    if (B > 65535) return GDN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !alpha || !beta || !o) return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, beta, S0, o, S_final};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn::chunk_pipe_workspace(B, Hqk, Hv);
+    if (need == 0) return GDN_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return GDN_ERR_INVALID_ARG;
+    gdn::ChunkArgs a{q, k, v, alpha, beta, S0, o, S_final, B, T, Hqk, Hv};
+    return cuda_status(gdn::launch_chunk_pipe(a, opts ? opts->chain_ctas : 0,
+                                              opts ? opts->wait_limit_cycles : 0, workspace,
+                                              workspace_bytes, static_cast<cudaStream_t>(stream)));
+}
+
+gdn_status gdn_device_status(void *stream)
+{
+    cudaError_t err = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (err != cudaSuccess) return cuda_status(err);
+    unsigned a = 0, b = 0;
+    err = gdn::chunk_pipe_take_error(&a);
+    if (err == cudaSuccess) err = gdn::chunk_tc_take_error(&b);
+    if (err != cudaSuccess) return cuda_status(err);
+    return (a | b) ? GDN_ERR_TIMEOUT : GDN_OK;
+}
+
 const char *gdn_status_string(gdn_status status)
 {
     switch (status) {
@@ -270,6 +318,7 @@ const char *gdn_status_string(gdn_status status)
     case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG";
     case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED";
     case GDN_ERR_CUDA: return "GDN_ERR_CUDA";
+    case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT";
     }
     return "GDN_UNKNOWN_STATUS";
 }

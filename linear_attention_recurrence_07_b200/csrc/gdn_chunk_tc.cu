@@ -698,6 +698,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 
 bool chunk_tc_available() { return encode_fn() != nullptr; }
 
+cudaError_t chunk_tc_take_error(unsigned *out)
+{
+    unsigned v = 0, zero = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_tc_error, sizeof(v));
+    if (err == cudaSuccess && v) err = cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(zero));
+    *out = v;
+    return err;
+}
+
 #ifdef GDN_TRACE
 // Copies the trace of the last traced launch (kTraceChunks x kTraceSlots ns stamps).
 extern "C" int gdn_trace_read(unsigned long long *host, int n)

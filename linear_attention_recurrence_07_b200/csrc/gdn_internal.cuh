@@ -59,6 +59,16 @@ struct BwdLaunch {
 size_t bwd_workspace(int B, int T, int Hv);
 cudaError_t launch_bwd(const BwdLaunch &L, gdn_dtype dtype, cudaStream_t stream);
 
+// Pipelined prefill (gdn_chunk_pipe.cu): prep CTAs stream each chunk's WY operands
+// to state-carrying chain CTAs through a ring in the workspace (cooperative launch).
+int chunk_pipe_chain_ctas(int B, int Hqk, int Hv, int sms, int req);
+size_t chunk_pipe_workspace(int B, int Hqk, int Hv);
+cudaError_t launch_chunk_pipe(const ChunkArgs &a, int chain_ctas, long long wait_limit,
+                              void *workspace, size_t workspace_bytes, cudaStream_t stream);
+// Read and clear a kernel file's device error word (bit 0: a bounded wait gave up).
+cudaError_t chunk_pipe_take_error(unsigned *out);
+cudaError_t chunk_tc_take_error(unsigned *out);
+
 // sst: null, or where the first segments write S_start(1)^T in bf16 (see TcParams).
 cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, float *segD,
                                      float *segM, __nv_bfloat16 *R, __nv_bfloat16 *sst,

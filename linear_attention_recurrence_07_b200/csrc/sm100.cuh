@@ -214,6 +214,17 @@ __device__ __forceinline__ void stmatrix_x4_trans(uint32_t saddr, uint32_t a, ui
                  ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+// 16 consecutive 32-bit columns, same lane mapping as tmem_st32.
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+          "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+          "r"(r[15])
+        : "memory");
+}
+
 // 32 consecutive 32-bit columns of packed data (e.g. bf16 pairs), same lane mapping.
 __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t *r) {
     tmem_st32(taddr, reinterpret_cast<const float *>(r));
