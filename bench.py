@@ -1,23 +1,31 @@
 """Benchmark of the Gated DeltaNet token mixer on B200 (prints ONE JSON line).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--prefill-entry pipelined|split|plain]
+    python bench.py --profile-case CASE [--launches L] ...   (no timing; for profilers)
 
-A step is one pass of the hot path over one batch of synthetic input:
-gdn_chunk_fwd over the model-dims prefill workload (B=1, T=4096, 16 QK heads,
-48 V heads, head dim 128, bf16 q/k/v, fp32 gates and state, chunk 64).  The
-headline ``value`` is prefill tokens/s over all ranks with inputs resident in
-HBM; L2 is flushed (256 MiB write) before every timed step and each step is
-timed with CUDA events on the launching stream.  The decode step (B=256
-sequences, one token, state updated in place) is measured in the same run and
-reported under ``decode`` (steps/s).  ``e2e`` repeats the prefill through the
-same C entry point with pinned HOST buffers, the host<->device copies inside
-the timed region.  ``cpu_baseline`` times the fp64 oracle on rank 0 on a
-bounded sample.  ``--impl reference`` times that oracle alone (the CPU
+A step is one pass of the hot path over one batch of synthetic input: the
+prefill of the model-dims workload (B=1, T=4096, 16 QK heads, 48 V heads, head
+dim 128, bf16 q/k/v, fp32 gates and state, chunk 64) through the library's
+prefill entry point (default gdn_chunk_fwd_split, its workspace allocated
+once).  The headline ``value`` is prefill tokens/s over all ranks with inputs
+resident in HBM; L2 is flushed (256 MiB write) before every timed step and each
+step is timed with CUDA events on the launching stream.  Measured in the same
+run and reported beside it: the batched prefill (B=8, T=8192, S0 != 0) and the
+long-context prefill (B=1, T=262,144) through the same entry point, the decode
+step (B=256 sequences, one token, state updated in place), draft verification,
+packed prefill and the backward pass.  ``e2e`` repeats the headline prefill
+through the same C entry point with pinned HOST buffers, the host<->device
+copies inside the timed region.  ``cpu_baseline`` times the fp64 oracle on rank
+0 on a bounded sample.  ``--impl reference`` times that oracle alone (the CPU
 reference arm).
 
 Multi-GPU (torchrun): every rank runs the same per-GPU workload on its own
 sequences (weak scaling); the only collectives are the timing barrier and the
 max-reduction of the elapsed time.
+
+``--profile-case`` runs one entry point a few times on one workload and prints
+"ok": the command the committed ncu summaries under profiles/ were taken with.
 """
 import argparse
 import hashlib
@@ -99,20 +107,23 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_traffic(kernel):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
-    current sources of that kernel (all files it is built from; else None)."""
+def kernel_traffic(key, workload):
+    """DRAM bytes of one timed step from the committed ncu summary: only if the entry
+    was captured on this workload (its ``workload_name``) from the current sources of
+    every kernel of the step (their hash); else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            entry = json.load(f)[kernel]
+            entry = json.load(f)[key]
+        if entry.get("workload_name") != workload:
+            return None
         h = hashlib.sha256()
         for src in entry["sources"]:
             with open(os.path.join(ROOT, src), "rb") as f:
                 h.update(f.read())
         if h.hexdigest()[:16] != entry["sources_sha256_16"]:
             return None
-        return float(entry["bytes_per_launch"])
+        return float(entry["bytes_per_step"])
     except (OSError, KeyError, ValueError):
         return None
 
@@ -217,31 +228,54 @@ def job_throughput(units_per_rank_per_step, steps, world, max_total_ms):
 
 
 # ----------------------------------------------------------------------------- timing
-def prefill_call(w, split, stream):
-    """The prefill entry point the bench times: gdn_chunk_fwd_split with the
-    automatic segment count (workspace allocated once), or plain gdn_chunk_fwd."""
+PREFILL_ENTRIES = ("pipelined", "split", "plain")
+
+
+def prefill_call(w, entry, stream, B=None, T=None):
+    """The prefill entry point a step calls: gdn_chunk_fwd_pipelined or
+    gdn_chunk_fwd_split (workspace allocated once, here) or plain gdn_chunk_fwd."""
+    B = w.B if B is None else B
+    T = w.T if T is None else T
     ws = None
-    if split:
-        need = binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv)
+    if entry == "split":
+        need = binding.split_workspace_bytes(B, T, w.Hv, 0, w.dk, w.dv)
         ws = torch.empty(max(need, 1), dtype=torch.uint8, device="cuda")
+    elif entry == "pipelined":
+        ws = torch.empty(max(binding.pipelined_workspace_bytes(B, w.Hqk, w.Hv, w.dk, w.dv), 1),
+                         dtype=torch.uint8, device="cuda")
 
     def call(d, o, S_final):
-        if split:
+        if entry == "split":
             binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o,
                                         S_final, segments=0, workspace=ws, stream=stream)
+        elif entry == "pipelined":
+            binding.gdn_chunk_fwd_pipelined(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o,
+                                            S_final, workspace=ws, stream=stream)
         else:
             binding.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o,
                                   S_final, stream=stream)
     return call
 
 
-def time_prefill(w, steps, warmup, world, rank, split=True):
+def launches_per_call(w, entry):
+    """Kernels of this library one prefill call launches (the pipelined entry also
+    clears its flags with one cudaMemsetAsync, not a kernel of ours)."""
+    if entry != "split":
+        return 1
+    if binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv) == 0:
+        return 1
+    two = (binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv)
+           == binding.split_workspace_bytes(w.B, w.T, w.Hv, 2, w.dk, w.dv))
+    return 2 if two else 3
+
+
+def time_prefill(w, steps, warmup, world, rank, entry="pipelined", flush_l2=True):
     d = inputs.workload_inputs(w, device="cuda")
     o = torch.empty((w.B, w.T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
     S_final = torch.empty((w.B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(L2_FLUSH_BYTES if flush_l2 else 16, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
-    call = prefill_call(w, split, stream)
+    call = prefill_call(w, entry, stream)
 
     def step():
         call(d, o, S_final)
@@ -268,7 +302,7 @@ def time_prefill(w, steps, warmup, world, rank, split=True):
             "window": (wall0, wall1)}
 
 
-def time_prefill_e2e(w, steps, warmup, world, split=True):
+def time_prefill_e2e(w, steps, warmup, world, entry="pipelined"):
     """Same call with inputs from pinned host memory and results read back."""
     host = {k: (None if v is None else v.cpu().pin_memory())
             for k, v in inputs.workload_inputs(w, device="cpu").items()}
@@ -280,7 +314,7 @@ def time_prefill_e2e(w, steps, warmup, world, split=True):
     stream = torch.cuda.current_stream()
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = o_h.numel() * o_h.element_size() + S_h.numel() * 4
-    call = prefill_call(w, split, stream)
+    call = prefill_call(w, entry, stream)
 
     def step():
         for k_, v in host.items():
@@ -475,14 +509,89 @@ def run_reference(args, rank, world):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hqk": w.Hqk, "Hv": w.Hv,
-                       "dk": w.dk, "dv": w.dv, "chunk": w.chunk},
+            "config": {"workload": w.name, "B": w.B, "T": per_step_T, "Hqk": w.Hqk, "Hv": w.Hv,
+                       "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+                       "sample_of": f"{w.name}: the first {per_step_T} of its {w.T} tokens per step"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"each step: oracle pass over B=1, T={per_step_T} "
                                        f"(all {w.Hv} V heads) of the workload"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+ENTRY_NAMES = {"pipelined": "gdn_chunk_fwd_pipelined (prep and chain CTAs, one cooperative launch)",
+               "split": "gdn_chunk_fwd_split (segments chosen by the library)",
+               "plain": "gdn_chunk_fwd"}
+# What each entry's timed step is (for the roofline record).
+ENTRY_TIMED = {"pipelined": "the whole pipelined launch (prep and chain CTAs) and its flag reset",
+               "split": "the whole split step: segment launch of the chunk kernel, segment chain, output fix-up",
+               "plain": "the one-CTA chunk kernel"}
+# Targets of the prefill workloads (time per call at 50% of the measured bf16 peak).
+PREFILL_TARGET_FRAC = 0.5
+
+
+def prefill_leg(w, entry, steps, warmup, world, rank, peaks, peak_src):
+    """One prefill workload through `entry` (inputs larger than L2: no flush)."""
+    r = time_prefill(w, steps, warmup, world, rank, entry=entry, flush_l2=False)
+    tok = w.B * w.T
+    t = r["per_launch_ms"] * 1e-3
+    flops = prefill_flops_per_token(w) * tok
+    target_ms = flops / (PREFILL_TARGET_FRAC * peaks["bf16_tflops"] * 1e12) * 1e3
+    return {"metric": f"prefill tokens/s ({ENTRY_NAMES[entry]})", "workload": w.name, "B": w.B,
+            "T": w.T, "S0": w.s0_std > 0, "value": job_throughput(tok, steps, world, r["total_ms"]),
+            "unit": "tokens/s", "ms_per_call": r["total_ms"] / steps,
+            "target_ms": target_ms, "meets_target": r["total_ms"] / steps <= target_ms,
+            "roofline": dict(roofline("tensor", flops / t / 1e12, peaks["bf16_tflops"], "TFLOP/s",
+                                      kernel_traffic(f"prefill_{entry}", w.name)),
+                             peak_source=f"{peak_src} bf16 burst", algorithmic_flops_per_launch=flops,
+                             hbm_frac=(prefill_bytes_per_token(w) * tok + w.B * prefill_state_bytes(w))
+                             / t / 1e9 / peaks["hbm_gbs"]),
+            "gpu_launches": r["launches"] * launches_per_call(w, entry),
+            "window": r["window"]}
+
+
+def profile_case(args):
+    """Runs one entry point `--launches` times on one workload and synchronizes
+    (no timing, prints "ok"): the command the ncu summaries in profiles/ name."""
+    torch.cuda.set_device(0)
+    stream = torch.cuda.current_stream()
+    case = args.profile_case
+    if case in ("prefill", "prefill-batched", "prefill-long"):
+        w = {"prefill": inputs.PREFILL_4K, "prefill-batched": inputs.PREFILL_BATCH8_8K,
+             "prefill-long": inputs.PREFILL_256K}[case]
+        T = args.T or w.T
+        d = inputs.workload_inputs(w, device="cuda", T=T)
+        o = torch.empty((w.B, T, w.Hv, w.dv), dtype=w.dtype, device="cuda")
+        S = torch.empty((w.B, w.Hv, w.dk, w.dv), dtype=torch.float32, device="cuda")
+        call = prefill_call(w, args.prefill_entry, stream, T=T)
+        for _ in range(args.launches):
+            call(d, o, S)
+    elif case == "decode":
+        w = inputs.DECODE_B256
+        B = args.B or w.B
+        S = inputs.decode_state(w, device="cuda", B=B)
+        x = inputs.decode_inputs(w, 0, device="cuda", B=B)
+        for _ in range(args.launches):
+            binding.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S)
+    elif case == "bwd":
+        w = inputs.PREFILL_4K
+        T = args.T or w.T
+        d = inputs.workload_inputs(w, device="cuda", T=T)
+        g = torch.Generator(device="cuda").manual_seed(w.seed + 7)
+        dO = torch.randn((w.B, T, w.Hv, w.dv), generator=g, device="cuda").to(w.dtype)
+        f32 = dict(dtype=torch.float32, device="cuda")
+        grads = [torch.empty((w.B, T, w.Hqk, w.dk), **f32), torch.empty((w.B, T, w.Hqk, w.dk), **f32),
+                 torch.empty((w.B, T, w.Hv, w.dv), **f32), torch.empty((w.B, T, w.Hv), **f32),
+                 torch.empty((w.B, T, w.Hv), **f32), torch.empty((w.B, w.Hv, w.dk, w.dv), **f32)]
+        ws = torch.empty(max(binding.bwd_workspace_bytes(w.B, T, w.Hv), 1), dtype=torch.uint8, device="cuda")
+        for _ in range(args.launches):
+            binding.gdn_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], dO, None, *grads,
+                            workspace=ws)
+    else:
+        raise SystemExit(f"unknown profile case {case}")
+    torch.cuda.synchronize()
+    print("ok")
 
 
 def main():
@@ -496,12 +605,26 @@ def main():
     ap.add_argument("--verify-steps", type=int, default=50)
     ap.add_argument("--varlen-steps", type=int, default=20)
     ap.add_argument("--bwd-steps", type=int, default=5)
+    ap.add_argument("--batched-steps", type=int, default=10)
+    ap.add_argument("--long-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-entry", choices=PREFILL_ENTRIES, default="split",
+                    help="prefill entry point of the timed step (default: gdn_chunk_fwd_split, the "
+                         "fastest on B=1, T=4096; the others are timed beside it)")
     ap.add_argument("--prefill-kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto",
-                    help="prefill kernel to time (default: the library's own choice)")
+                    help="kernel gdn_chunk_fwd / _split / _varlen run (default: the library's choice)")
+    ap.add_argument("--profile-case", choices=["prefill", "prefill-batched", "prefill-long", "decode",
+                                               "bwd"], default=None)
+    ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--B", type=int, default=None)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    binding.set_prefill_kernel(args.prefill_kernel)
+    if args.profile_case:
+        profile_case(args)
+        return
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
@@ -512,25 +635,25 @@ def main():
     peaks, peak_src = load_peaks()
     w = inputs.PREFILL_4K
     wd = inputs.DECODE_B256
-    binding.set_prefill_kernel(args.prefill_kernel)
+    entry = args.prefill_entry
     kernel = binding.prefill_kernel_for(w.B, w.Hv, w.dtype)
-
-    segs = binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv) > 0
-    # kernels per split step: chunk kernel + one finishing launch for two segments,
-    # chunk kernel + segment chain + output fix-up for more (same plan <=> same size)
-    two = (binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv)
-           == binding.split_workspace_bytes(w.B, w.T, w.Hv, 2, w.dk, w.dv))
-    split_launches = (2 if two else 3) if segs else 1
     with ClockSampler(local) as clocks:
-        pre = time_prefill(w, args.steps, args.warmup, world, rank, split=segs)
-        plain = time_prefill(w, max(args.steps // 5, 3), args.warmup, world, rank, split=False)
+        pre = time_prefill(w, args.steps, args.warmup, world, rank, entry=entry)
+        others = {e: time_prefill(w, max(args.steps // 5, 3), args.warmup, world, rank, entry=e)
+                  for e in PREFILL_ENTRIES if e != entry}
         dec = time_decode(wd, args.decode_steps, args.warmup, world)
+    with ClockSampler(local) as clocks3:
+        batched = prefill_leg(inputs.PREFILL_BATCH8_8K, entry, args.batched_steps, 3, world, rank,
+                              peaks, peak_src)
+        longctx = prefill_leg(inputs.PREFILL_256K, entry, args.long_steps, 3, world, rank, peaks, peak_src)
+    for leg in (batched, longctx):
+        leg["clocks"] = clocks3.summary([leg.pop("window")])
     wv, wl = inputs.VERIFY_B256_N4, inputs.PREFILL_VARLEN
     with ClockSampler(local) as clocks2:
         ver = time_verify(wv, args.verify_steps, args.warmup, world)
         vl = time_varlen(wl, args.varlen_steps, args.warmup, world)
         bw = time_backward(w, args.bwd_steps, 3, world)
-    e2e = time_prefill_e2e(w, args.e2e_steps, 3, world, split=segs)
+    e2e = time_prefill_e2e(w, args.e2e_steps, 3, world, entry=entry)
 
     tokens_per_step = w.B * w.T
     value = job_throughput(tokens_per_step, args.steps, world, pre["total_ms"])
@@ -559,25 +682,25 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "Hqk": w.Hqk, "Hv": w.Hv,
                    "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "state": "fp32",
-                   "prefill_kernel": kernel,
-                   "prefill_entry": ("gdn_chunk_fwd_split (segments chosen by the library)" if segs
-                                     else "gdn_chunk_fwd"),
-                   "plain_gdn_chunk_fwd_ms": plain["total_ms"] / max(args.steps // 5, 3),
+                   "prefill_entry": ENTRY_NAMES[entry],
+                   "other_entries_ms": {e: r["total_ms"] / r["launches"] for e, r in others.items()},
+                   "one_cta_kernel": kernel,
                    "l2": "flushed before every timed step (256 MiB write)",
                    "parallelism": f"dp{world} (independent sequences per GPU)"},
         "roofline": dict(roofline("tensor", flops_launch / t_launch / 1e12, peaks["bf16_tflops"],
-                                  "TFLOP/s", kernel_traffic("prefill_split" if segs else "prefill_" + kernel)),
-                         timed=("the whole split step: segment launch of the chunk kernel, "
-                                "segment chain, output fix-up" if segs else "the chunk kernel"),
+                                  "TFLOP/s", kernel_traffic(f"prefill_{entry}", w.name)),
+                         timed=ENTRY_TIMED[entry],
                          peak_source=f"{peak_src} bf16 burst",
                          algorithmic_flops_per_launch=flops_launch,
                          hbm_frac=bytes_launch / t_launch / 1e9 / peaks["hbm_gbs"]),
+        "batched_prefill": batched,
+        "long_context_prefill": longctx,
         "decode": {
             "metric": "decode steps/s", "workload": wd.name, "B": wd.B,
             "value": job_throughput(1, args.decode_steps, world, dec["total_ms"]), "unit": "steps/s",
             "ms_per_step": dec["total_ms"] / args.decode_steps,
             "roofline": dict(roofline("hbm", dec_bytes / t_dec / 1e9, peaks["hbm_gbs"], "GB/s",
-                                      kernel_traffic("decode")),
+                                      kernel_traffic("decode", wd.name)),
                              peak_source=f"{peak_src} copy bandwidth",
                              algorithmic_bytes_per_launch=dec_bytes),
             "gpu_launches": dec["launches"],
@@ -622,7 +745,7 @@ def main():
         "e2e": {"value": job_throughput(tokens_per_step, args.e2e_steps, world, e2e["total_ms"]),
                 "unit": "tokens/s", "h2d_bytes_per_step": e2e["h2d"],
                 "d2h_bytes_per_step": e2e["d2h"]},
-        "gpu_launches": pre["launches"] * split_launches,
+        "gpu_launches": pre["launches"] * launches_per_call(w, entry),
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:

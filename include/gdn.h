@@ -223,11 +223,18 @@ gdn_status gdn_device_status(void *stream);
  *
  * Arguments and results as gdn_chunk_fwd_split without workspace and
  * workspace_bytes.
- * - A GDN_BF16 problem whose scratch (gdn_chunk_fwd_split_workspace) is over
- *   48 MiB returns GDN_ERR_UNSUPPORTED.
- * - The first call on a device looks up the array's address
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
- *   A failed lookup returns GDN_ERR_CUDA.
+ * - A GDN_BF16 problem whose split scratch (gdn_chunk_fwd_split_workspace,
+ *   under the calling thread's kernel choice) is over 48 MiB returns
+ *   GDN_ERR_UNSUPPORTED.
+ * - Every call looks up the array's address in the current device's context
+ *   (cudaGetSymbolAddress); the current device must be the one that holds the
+ *   data.  A failed lookup returns GDN_ERR_CUDA.
+ * - With lazy module loading (CUDA_MODULE_LOADING=LAZY, the default of recent
+ *   CUDA), the module that holds the array is loaded, and its 48 MiB reserved,
+ *   by the first call on each device (or by the first use of any kernel of the
+ *   library).  A caller with a fixed memory plan makes one call as a warm-up
+ *   before the plan is fixed, and before any stream capture.  After that no
+ *   call changes the device's free memory.
  * - Every call shares the one array, so calls that overlap on the GPU (on
  *   different streams, or from different threads) race.
  * - Nothing in the array has to start at zero.
@@ -311,28 +318,25 @@ gdn_status gdn_decode_step_slots(const void *q, const void *k, const void *v,
  * Prefill kernel selection (library-specific: the page describes the method,
  * not how its evaluation is split over the GPU).
  *
- *   GDN_PREFILL_AUTO        default: GDN_BF16 runs on the tensor cores
- *                           (GDN_PREFILL_TC in this version), GDN_F32 on the
- *                           CUDA-core kernel
- *   GDN_PREFILL_SIMT        CUDA-core chunk kernel, both dtypes
- *   GDN_PREFILL_TC          tensor cores, one CTA per (sequence, V head)
- *   GDN_PREFILL_TC_CLUSTER  tensor cores, a cluster of two CTAs per
- *                           (sequence, V head): one carries the state, the
- *                           other prepares the chunks' WY factors
- * All variants compute the same function (to the dtype's rounding); the two TC
- * variants return identical bits.  The TC variants take GDN_BF16 only: with
- * another choice gdn_chunk_fwd returns GDN_ERR_UNSUPPORTED, as it does when
- * the tensor-map encoder is missing.
+ *   GDN_PREFILL_AUTO   default: GDN_BF16 runs on the tensor cores
+ *                      (GDN_PREFILL_TC), GDN_F32 on the CUDA-core kernel
+ *   GDN_PREFILL_SIMT   CUDA-core chunk kernel, both dtypes
+ *   GDN_PREFILL_TC     tensor cores, one CTA per (sequence, V head)
+ * All variants compute the same function, each to its dtype's rounding (the
+ * tensor-core kernel with bf16 operands, the CUDA-core kernel in fp32).  The TC
+ * variant takes GDN_BF16 only: with another choice gdn_chunk_fwd returns
+ * GDN_ERR_UNSUPPORTED, as it does when the tensor-map encoder is missing.
  *
- * gdn_set_prefill_kernel sets the choice for every later gdn_chunk_fwd call of
- * the process (all threads and devices); it returns GDN_ERR_INVALID_ARG for a
- * value outside the enum.  gdn_get_prefill_kernel returns the current choice.
+ * gdn_set_prefill_kernel sets the choice for the later gdn_chunk_fwd,
+ * gdn_chunk_fwd_varlen and gdn_chunk_fwd_split calls of the CALLING THREAD only
+ * (a per-thread setting; other threads keep their own, AUTO unless they set
+ * one); it returns GDN_ERR_INVALID_ARG for a value outside the enum.
+ * gdn_get_prefill_kernel returns the calling thread's current choice.
  */
 typedef enum {
     GDN_PREFILL_AUTO = 0,
     GDN_PREFILL_SIMT = 1,
-    GDN_PREFILL_TC = 2,
-    GDN_PREFILL_TC_CLUSTER = 3
+    GDN_PREFILL_TC = 2
 } gdn_prefill_kernel;
 
 gdn_status gdn_set_prefill_kernel(gdn_prefill_kernel kernel);
@@ -340,8 +344,8 @@ gdn_prefill_kernel gdn_get_prefill_kernel(void);
 
 /*
  * The kernel (a gdn_prefill_kernel value, never GDN_PREFILL_AUTO) that
- * gdn_chunk_fwd runs for B sequences of Hv V heads in `dtype` under the current
- * choice, on the calling thread's current CUDA device; -1 if that call would
+ * gdn_chunk_fwd runs for B sequences of Hv V heads in `dtype` under the calling
+ * thread's current choice, on its current CUDA device; -1 if that call would
  * return GDN_ERR_UNSUPPORTED (a forced TC kernel with GDN_F32) or the arguments
  * are invalid.  No kernel is launched.
  */

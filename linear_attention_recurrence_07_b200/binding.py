@@ -19,7 +19,7 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT 
 GDN_F32, GDN_BF16 = 0, 1
 _DTYPES = {torch.float32: GDN_F32, torch.bfloat16: GDN_BF16}
 # gdn_prefill_kernel values
-PREFILL_KERNELS = {"auto": 0, "simt": 1, "tc": 2, "tc_cluster": 3}
+PREFILL_KERNELS = {"auto": 0, "simt": 1, "tc": 2}
 
 
 class GdnError(RuntimeError):
@@ -192,8 +192,8 @@ def gdn_decode_step(q, k, v, alpha, beta, S, o, S_new, stream=None):
 
 
 def set_prefill_kernel(name):
-    """Selects the kernel of every later prefill call in this process (C entry point
-    ``gdn_set_prefill_kernel``): one of ``PREFILL_KERNELS``."""
+    """Selects the kernel of every later prefill call of this thread (C entry point
+    ``gdn_set_prefill_kernel``, a per-thread setting): one of ``PREFILL_KERNELS``."""
     if name not in PREFILL_KERNELS:
         raise GdnError(f"unknown prefill kernel {name!r}; one of {sorted(PREFILL_KERNELS)}")
     _check(library().gdn_set_prefill_kernel(PREFILL_KERNELS[name]), "gdn_set_prefill_kernel")

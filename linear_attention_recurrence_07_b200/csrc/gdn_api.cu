@@ -1,8 +1,6 @@
 // C ABI of libgdn.so: argument checks and dispatch.  See include/gdn.h.
 #include <stdint.h>
 
-#include <atomic>
-
 #include "gdn_internal.cuh"
 
 namespace {
@@ -10,7 +8,9 @@ namespace {
 thread_local int g_last_cuda_error = 0;
 constexpr int kMaxDecodeTokens = 64;   // gdn_decode_tokens: tokens per call
 constexpr int kMaxSegments = 16;       // gdn_chunk_fwd_split: segments per sequence
-std::atomic<int> g_prefill_kernel{GDN_PREFILL_AUTO};   // process-wide prefill kernel choice
+// Prefill kernel choice of the calling thread (a per-thread setting: one thread's
+// choice never changes what another thread's calls run).
+thread_local int g_prefill_kernel = GDN_PREFILL_AUTO;
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -30,22 +30,15 @@ gdn_status check_heads(int Hqk, int Hv, int dk, int dv)
     return GDN_OK;
 }
 
-// Whether the automatic choice takes the cluster kernel when all its clusters fit
-// at once.  Off while the cluster kernel is slower than the one-CTA kernel on
-// those sizes (measured on B200: 0.345 ms against 0.233 ms for B=1, T=4096,
-// 48 V heads).
-constexpr bool kPreferCluster = false;
-
 // The prefill kernel a call with these sizes runs under the current choice, or
 // -1 when a forced tensor-core kernel cannot take the call.
 int resolve_prefill_kernel(int B, int Hv, gdn_dtype dtype)
 {
-    const int kind = g_prefill_kernel.load(std::memory_order_relaxed);
+    (void)B;
+    (void)Hv;
+    const int kind = g_prefill_kernel;
     const bool tc_ok = dtype == GDN_BF16 && gdn::chunk_tc_available();
-    if (kind == GDN_PREFILL_AUTO)
-        return !tc_ok ? GDN_PREFILL_SIMT
-                      : (kPreferCluster && gdn::chunk_tc_cluster_fits(B, Hv)) ? GDN_PREFILL_TC_CLUSTER
-                                                                               : GDN_PREFILL_TC;
+    if (kind == GDN_PREFILL_AUTO) return tc_ok ? GDN_PREFILL_TC : GDN_PREFILL_SIMT;
     if (kind != GDN_PREFILL_SIMT && !tc_ok) return -1;
     return kind;
 }
@@ -86,7 +79,6 @@ gdn_status chunk_fwd_common(const void *q, const void *k, const void *v,
     cudaError_t err;
     switch (kind) {
     case GDN_PREFILL_TC: err = gdn::launch_chunk_tc(a, s); break;
-    case GDN_PREFILL_TC_CLUSTER: err = gdn::launch_chunk_tc_cluster(a, s); break;
     default: err = gdn::launch_chunk_simt(a, dtype, s); break;
     }
     return cuda_status(err);
@@ -141,14 +133,14 @@ gdn_status gdn_decode_step(const void *q, const void *k, const void *v,
 gdn_status gdn_set_prefill_kernel(gdn_prefill_kernel kernel)
 {
     const int k = (int)kernel;
-    if (k < GDN_PREFILL_AUTO || k > GDN_PREFILL_TC_CLUSTER) return GDN_ERR_INVALID_ARG;
-    g_prefill_kernel.store(k, std::memory_order_relaxed);
+    if (k < GDN_PREFILL_AUTO || k > GDN_PREFILL_TC) return GDN_ERR_INVALID_ARG;
+    g_prefill_kernel = k;
     return GDN_OK;
 }
 
 gdn_prefill_kernel gdn_get_prefill_kernel(void)
 {
-    return (gdn_prefill_kernel)g_prefill_kernel.load(std::memory_order_relaxed);
+    return (gdn_prefill_kernel)g_prefill_kernel;
 }
 
 int gdn_prefill_kernel_for(int B, int Hv, gdn_dtype dtype)
@@ -223,6 +215,26 @@ int auto_segments(int B, int Hv)
 
 }  // namespace
 
+}  // extern "C"
+
+namespace gdn {
+
+// Scratch bytes gdn_chunk_fwd_split will use for these arguments under the calling
+// thread's kernel choice: 0 when the call goes straight to gdn_chunk_fwd (not bf16,
+// the tensor cores unavailable or not chosen, or one segment covers the sequence).
+size_t split_scratch_needed(int B, int T, int Hv, int dk, int dv, int segments, gdn_dtype dtype)
+{
+    if (segments < 0 || segments > kMaxSegments) return 0;
+    if (segments == 0 && B > 0 && Hv > 0) segments = auto_segments(B, Hv);
+    const bool tc = dtype == GDN_BF16 && chunk_tc_available() && g_prefill_kernel != GDN_PREFILL_SIMT;
+    if (!tc || B <= 0 || T <= 0 || Hv <= 0 || segments <= 1 || dk != kHeadDim || dv != kHeadDim) return 0;
+    return chunk_tc_split_workspace(B, T, Hv, segments);
+}
+
+}  // namespace gdn
+
+extern "C" {
+
 size_t gdn_chunk_fwd_split_workspace(int B, int T, int Hv, int dk, int dv, int segments)
 {
     if (B <= 0 || T <= 0 || Hv <= 0 || dk != gdn::kHeadDim || dv != gdn::kHeadDim) return 0;
@@ -240,11 +252,8 @@ gdn_status gdn_chunk_fwd_split(const void *q, const void *k, const void *v,
 {
     if (segments < 0 || segments > kMaxSegments) return GDN_ERR_INVALID_ARG;
     if (segments == 0 && B > 0 && Hv > 0) segments = auto_segments(B, Hv);
-    const bool tc = dtype == GDN_BF16 && gdn::chunk_tc_available() &&
-                    g_prefill_kernel.load(std::memory_order_relaxed) != GDN_PREFILL_SIMT;
-    const size_t need = (tc && B > 0 && T > 0 && Hv > 0 && segments > 1)
-                            ? gdn::chunk_tc_split_workspace(B, T, Hv, segments) : 0;
-    if (need == 0 || dk != gdn::kHeadDim || dv != gdn::kHeadDim)   // nothing to split
+    const size_t need = gdn::split_scratch_needed(B, T, Hv, dk, dv, segments, dtype);
+    if (need == 0)   // nothing to split
         return gdn_chunk_fwd(q, k, v, alpha, beta, S0, o, S_final, B, T, Hqk, Hv, dk, dv, chunk,
                              dtype, stream);
     if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
@@ -325,7 +334,7 @@ const char *gdn_status_string(gdn_status status)
 
 int gdn_last_cuda_error(void) { return g_last_cuda_error; }
 
-int gdn_version(void) { return 100; }
+int gdn_version(void) { return 200; }
 
 }  // extern "C"
 

@@ -19,14 +19,18 @@
 //   prep CTAs   one work item = one QK head group (the Hv/Hqk V heads that share
 //               a QK head) x one chunk: TMA K, Q; the grams on the tensor core
 //               (once per group); then one warpgroup per V head computes the
-//               gates, A, P, T, Bw and Bu and writes them (bf16 operand tiles in
-//               the 128B-swizzled layout the tensor core reads, plus gamma and g)
-//               into a ring slot in global memory, then releases the slot's flag.
+//               gates, A, P, T, Bw and Bu, and W = Bw K on the tensor core, and
+//               writes W, Bu, P (bf16 operand tiles in the 128B-swizzled layout
+//               the tensor core reads) and gamma, g into a ring slot in global
+//               memory, then releases the slot's flag.
 //   chain CTAs  one (sequence, V head) at a time, all its chunks in order: TMA
 //               K, Q, V from the inputs and the ring slot from the prep; the
-//               state S^T (fp32) stays in TMEM; per chunk W^T = K^T Bw^T,
-//               U~^T = V^T Bu^T, U^T = U~^T - S^T W^T, O^T = S^T Q~^T + U^T P^T,
-//               S^T <- gamma_{C-1} S^T + (U^T diag(g)) K, as in the one-CTA kernel.
+//               state S^T (fp32) stays in TMEM; per chunk U~^T = V^T Bu^T,
+//               U^T = U~^T - S^T W^T, O^T = (S^T Q^T) diag(gamma) + U^T P^T,
+//               S^T <- gamma_{C-1} S^T + (U^T diag(g)) K.  The two diagonal
+//               scalings act on TMEM values (a g-scaled bf16 copy of U^T, and the
+//               S-part of O^T scaled by the helper warpgroup), so the K and Q tiles
+//               go to the tensor core as loaded.
 //
 // The ring has kRing slots per chain CTA.  A prep warpgroup writes slot n % kRing
 // for the chain's n-th chunk only after the chain has loaded chunk n - kRing
@@ -45,7 +49,7 @@ namespace {
 
 __device__ unsigned int g_pipe_error = 0;   // bit 0: a bounded wait of this kernel gave up
 
-constexpr int NT = 448;                     // 14 warps, both roles
+constexpr int NT = 512;                     // 16 warps, both roles
 
 // Optional event trace (build with -DGDN_TRACE): %globaltimer stamps of chain CTA 0's
 // roles and of the prep warpgroups that serve it, for its first kPTraceN chunks.
@@ -62,81 +66,116 @@ __device__ __forceinline__ void ptrace(int n, int slot, bool on) {
     }
 }
 #define PTRACE(n, slot, on) ptrace((n), (slot), (on))
+// whole grid: each CTA's start and end, each chain CTA's conversion start per chunk
+constexpr int kGridCTAs = 160, kGridChunks = 64;
+__device__ unsigned long long g_pcta[kGridCTAs][4];             // start, end, smid, SM clocks start..end
+// per chain CTA and chunk: conversion start, ring flag seen, slot landed, prep release,
+// S^T bf16 ready, U^T done (seen), U^T bf16 ready, O epilogue done
+__device__ unsigned long long g_pchain[kGridCTAs][kGridChunks][8];
+__device__ __forceinline__ unsigned long long gtimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ long long g_pclk0[kGridCTAs];
+#define PCTA(slot) do { if (threadIdx.x == 0 && blockIdx.x < kGridCTAs) { g_pcta[blockIdx.x][(slot)] = gtimer(); \
+    unsigned sid; asm volatile("mov.u32 %0, %%smid;" : "=r"(sid)); g_pcta[blockIdx.x][2] = sid; \
+    if ((slot) == 0) g_pclk0[blockIdx.x] = clock64(); else g_pcta[blockIdx.x][3] = clock64() - g_pclk0[blockIdx.x]; } } while (0)
+#define PCHAIN(x, n, k, on) do { if ((on) && (x) < kGridCTAs && (n) < kGridChunks) g_pchain[(x)][(n)][(k)] = gtimer(); } while (0)
 // clock64 stamps inside the MMA issuer's groups (chain CTA 0, chunks 8..15)
 __device__ long long g_pmma[8][24];
 #define PMMA(n, slot, on) do { if ((on) && (n) >= 8 && (n) < 16) g_pmma[(n) - 8][(slot)] = clock64(); } while (0)
 #else
 #define PTRACE(n, slot, on) ((void)0)
 #define PMMA(n, slot, on) ((void)0)
+#define PCTA(slot) ((void)0)
+#define PCHAIN(x, n, k, on) ((void)0)
 #endif
 
 // ---------------------------------------------------------------- ring slot
-constexpr uint32_t RS_BW = 0, RS_BU = TILE, RS_P = 2 * TILE, RS_GATE = 3 * TILE;
-constexpr uint32_t RS_LOAD = 3 * TILE + 512;          // bytes loaded per chunk
-constexpr uint32_t RS_BYTES = 25600;                  // slot stride (1024-multiple)
+constexpr uint32_t RS_W = 0;                          // W [d][r] bf16, MN-major B operand (16 KB)
+constexpr uint32_t RS_BU = 2 * TILE, RS_P = 3 * TILE; // T diag(beta), masked decay P (8 KB each)
+constexpr uint32_t RS_GATE = 4 * TILE;                // gamma[64], g[64] fp32
+constexpr uint32_t RS_TILES = 4 * TILE;               // operand tiles of a slot (loaded as one copy)
+constexpr uint32_t RS_GATE_BYTES = 512;               // the gate vectors (a second copy)
+constexpr uint32_t RS_BYTES = 33 * 1024;              // slot stride in the ring (1024-multiple)
 constexpr int kRing = 8;                              // slots per chain CTA
+constexpr int kFlagWords = 32;                        // one 128-byte line per chain CTA's flags
 
 // ---------------------------------------------------------------- chain role
 constexpr uint32_t COL_S = 0;      // S^T fp32, 128 columns
-constexpr uint32_t COL_W = 128;    // W^T fp32; after the chain read it: S^T bf16 (64 packed)
-constexpr uint32_t COL_U = 192;    // U^T, two buffers; then U^T bf16 in place (32 packed)
-constexpr uint32_t COL_O = 320;    // O^T, two buffers
-constexpr uint32_t COL_UG = 448;   // U^T diag(g) bf16 (32 packed columns), two buffers
+constexpr uint32_t COL_SB = 128;   // S^T bf16 (64 packed columns), two buffers
+constexpr uint32_t COL_U = 256;    // U^T fp32, two buffers; then U^T bf16 in place (32 packed)
+constexpr uint32_t COL_O = 384;    // O^T, two buffers
 constexpr uint32_t CH_TMEM_COLS = 512;
 
-constexpr int NKQ = 3;
+constexpr int NKQ = 3;                                // K/Q stages, chunk n uses n % NKQ
+constexpr int NRB = 3;                                // ring buffers, chunk n uses n % NRB
 constexpr uint32_t KQ_STAGE = 4 * TILE;               // [K d0-63][Q d0-63][K d64-127][Q d64-127]
 constexpr uint32_t OFF_KQ = 0;
 constexpr uint32_t OFF_V = OFF_KQ + NKQ * KQ_STAGE;    // 2 x [V j0-63][V j64-127]
-constexpr uint32_t OFF_RB = OFF_V + 4 * TILE;          // 2 ring buffers (RS_BYTES each)
-constexpr uint32_t OFF_W = OFF_RB + 2 * RS_BYTES;      // W stored [d][r] (MN-major B)
-constexpr uint32_t OFF_OST = OFF_W + 2 * TILE;         // O staging [r][j] for the TMA store
-constexpr uint32_t OFF_CBAR = OFF_OST + 2 * TILE;
-constexpr uint32_t CH_NBAR = 32;
-constexpr uint32_t OFF_CMISC = OFF_CBAR + CH_NBAR * 8;
+constexpr uint32_t OFF_RB = OFF_V + 4 * TILE;          // NRB ring buffers: operand tiles (32 KB each)
+constexpr uint32_t OFF_RG = OFF_RB + NRB * RS_TILES;   // NRB ring buffers: gate vectors (512 B each)
+constexpr uint32_t OFF_CBAR = OFF_RG + NRB * RS_GATE_BYTES;
+constexpr uint32_t CH_NBAR = 38;
+constexpr uint32_t OFF_CMISC = OFF_CBAR + CH_NBAR * 8;   // TMEM base, local abort flag
 constexpr uint32_t CH_SMEM_USED = OFF_CMISC + 16;
-static_assert(OFF_RB % 1024 == 0 && RS_BYTES % 1024 == 0 && OFF_W % 1024 == 0 &&
-              OFF_OST % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(OFF_RB % 1024 == 0 && RS_TILES % 1024 == 0 && RS_BYTES % 1024 == 0,
+              "swizzled tiles need 1024-byte alignment");
 
+// Chain CTA warps: 0 input TMA, 1 and 3 MMA issuers, 2 ring loader, 4-7 and 8-11
+// the two conversion warpgroups (state columns 0-63 / 64-127; U columns 0-31 /
+// 32-63), 12-15 the helper warpgroup (gamma scaling of the S-part of O, O epilogue).
 enum : int {
-    C_KQ_FULL = 0,    // x3
-    C_KQ_EMPTY = 3,   // x3 (YS MMAs of the chunk done)
+    C_KQ_FULL = 0,    // x3 (K/Q stage landed)
+    C_KQ_EMPTY = 3,   // x3 (S and O MMAs of the chunk done: one commit of each issuer)
     C_V_FULL = 6,     // x2
-    C_V_EMPTY = 8,    // x2 (WU MMAs done)
-    C_RB_FULL = 10,   // x2 (ring slot landed)
-    C_RB_EMPTY = 12,  // x2 (1 MMA commit + 128 chain + 128 helper)
-    C_W_FULL = 14,    // x2 (W^T, U~^T done)
-    C_S_READY = 16,   // chain: S^T bf16 in TMEM, W bf16 in SMEM (128)
-    C_QT_READY = 17,  // x2 helper: Q~ scaled in place (128)
-    C_U_FULL = 19,    // U^T done
-    C_X_FULL = 20,    // S-part of O^T done
-    C_U_READY = 21,   // x2 chain: U^T bf16 written (128)
+    C_V_EMPTY = 8,    // x2 (U~ MMAs done)
+    C_RB_FULL = 10,   // x3 (ring slot landed)
+    C_RB_EMPTY = 13,  // x3 (a commit of each issuer + 12 warps)
+    C_S_READY = 16,   // x2 (per S^T bf16 buffer): both conversion warpgroups (8 warps)
+    C_XS_READY = 18,  // x2 helper: S-part of O^T scaled by gamma (4 warps)
+    C_U_FULL = 20,    // U^T done
+    C_U_READY = 21,   // x2 conversion warpgroups: U^T bf16 written (8 warps)
     C_S_FULL = 23,    // state update done
-    C_O_FULL = 24,    // x2 O^T complete
-    C_O_FREE = 26,    // x2 helper: O^T read out (128)
-    C_DRAIN = 28,
+    C_X_FULL = 24,    // x2 (per S^T bf16 buffer): S-part of O^T done
+    C_O_FULL = 26,    // x2 O^T complete
+    C_O_FREE = 28,    // x2 helper: O^T read out (4 warps)
+    C_DRAIN = 30,     // both issuing threads' MMAs done (2 commits)
+    C_UT_FULL = 31,   // x2 U~^T of the chunk done (its U buffer)
+    C_X_GO = 33,      // x2 critical issuer: UG(n) issued (per S^T bf16 buffer)
+    C_O_GO = 35,      // x2 critical issuer: SG(n) issued (per U buffer)
 };
+// Arrival counts: a tcgen05.commit counts one, a warp (warp_arrive) one.
 __host__ __device__ constexpr uint32_t chain_bar_count(int i) {
-    return (i == C_RB_EMPTY || i == C_RB_EMPTY + 1) ? 257u
-         : (i == C_S_READY || i == C_QT_READY || i == C_QT_READY + 1 || i == C_U_READY ||
-            i == C_U_READY + 1 || i == C_O_FREE || i == C_O_FREE + 1) ? 128u : 1u;
+    return (i >= C_RB_EMPTY && i < C_RB_EMPTY + NRB) ? 14u
+         : ((i >= C_KQ_EMPTY && i < C_KQ_EMPTY + NKQ) || i == C_DRAIN) ? 2u
+         : (i == C_S_READY || i == C_S_READY + 1 || i == C_U_READY || i == C_U_READY + 1) ? 8u
+         : (i == C_XS_READY || i == C_XS_READY + 1 || i == C_O_FREE || i == C_O_FREE + 1) ? 4u : 1u;
 }
-static_assert(C_DRAIN < (int)CH_NBAR, "barrier count");
+static_assert(C_O_GO + 1 < (int)CH_NBAR, "barrier count");
 
 // ---------------------------------------------------------------- prep role
 constexpr int NPKQ = 2;
 constexpr int kPrepWG = 3;
 constexpr uint32_t P_OFF_KQ = 0;
+constexpr uint32_t P_OFF_BW = P_OFF_KQ + NPKQ * KQ_STAGE;   // per warpgroup: Bw tile (8 KB)
 constexpr uint32_t P_SA = 64 * LDA * 4, P_SY = 32 * LDY * 4;
 constexpr uint32_t P_WG_BYTES = P_SA + P_SY + GATE_BUF;
-constexpr uint32_t P_OFF_WG = P_OFF_KQ + NPKQ * KQ_STAGE;
+constexpr uint32_t P_OFF_WG = P_OFF_BW + kPrepWG * TILE;
 constexpr uint32_t P_OFF_BAR = P_OFF_WG + kPrepWG * P_WG_BYTES;
-constexpr uint32_t P_NBAR = 9;
+constexpr uint32_t P_NBAR = 16;
 constexpr uint32_t P_OFF_MISC = P_OFF_BAR + P_NBAR * 8;
 constexpr uint32_t P_SMEM_USED = P_OFF_MISC + 16;
-constexpr uint32_t P_TMEM_COLS = 128;   // two gram buffers
-enum : int { P_KQ_FULL = 0, P_KQ_EMPTY = 2, P_G_FULL = 4, P_G_FREE = 6, P_DRAIN = 8 };   // x2 but DRAIN
-static_assert(P_WG_BYTES % 16 == 0, "per-warpgroup scratch alignment");
+constexpr uint32_t P_TMEM_COLS = 512;   // two gram buffers (0-127), W^T per warpgroup (128 + 64 w)
+enum : int {
+    P_KQ_FULL = 0, P_KQ_EMPTY = 2, P_G_FULL = 4, P_G_FREE = 6,   // x2 each
+    P_BW_READY = 8,   // x3 (per warpgroup): Bw tile written (4 warps)
+    P_WT_FULL = 11,   // x3 (per warpgroup): W^T = K^T Bw^T done
+    P_DRAIN = 14,
+};
+static_assert(P_WG_BYTES % 16 == 0 && P_OFF_BW % 1024 == 0, "prep shared-memory alignment");
+static_assert(P_DRAIN < (int)P_NBAR, "barrier count");
 
 constexpr uint32_t SMEM_USED = CH_SMEM_USED > P_SMEM_USED ? CH_SMEM_USED : P_SMEM_USED;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
@@ -150,17 +189,12 @@ struct PipeParams {
     int nchunks;                  // ceil(T / 64)
     int n_chain, n_prep;          // CTA roles: blockIdx.x < n_chain is a chain CTA
     unsigned char *ring;          // [n_chain][kRing][RS_BYTES]
-    unsigned *ready;              // [n_chain][kRing]: chunk counter + 1 once the slot is filled
-    unsigned *consumed;           // [n_chain]: chunks whose slot the chain has loaded
-    unsigned *abort;              // launch-wide abort word
+    unsigned *ready;              // [n_chain][kFlagWords], first kRing used: chunk counter + 1 once the slot is filled
+    unsigned *consumed;           // [n_chain][kFlagWords], first used: chunks whose slot the chain has loaded
+    unsigned *abort;              // launch-wide abort word (a line of its own)
     long long wait_limit;         // SM clocks a wait may take before giving up
 };
 
-__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
 __device__ __forceinline__ void st_release(unsigned *p, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -174,39 +208,90 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t b
         ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
-// Bounded waits that also give up once any CTA of the launch has aborted.
+__device__ __forceinline__ unsigned ld_relaxed(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_acquire_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// Bounded waits that also give up once any CTA of the launch has aborted.  The
+// CTA's own abort flag (shared memory) is checked on every pass; the launch-wide
+// word (global memory, a round trip of about a microsecond) only every kGlobalPoll
+// clocks, so that a waiting thread is never stuck in that load when its phase
+// completes.
+constexpr long long kGlobalPoll = 16384;
 struct PCtl {
     uint64_t *bar;
     volatile int *abort_local;
     volatile unsigned *abort_global;
     long long limit;
-    __device__ __forceinline__ bool aborted() const { return *abort_local != 0 || *abort_global != 0; }
+    __device__ __forceinline__ bool aborted() const { return *abort_local != 0; }
+    // Reads the launch-wide word; if another CTA aborted, marks this CTA too.
+    __device__ __forceinline__ bool poll_global() const {
+        if (*abort_global == 0) return false;
+        *abort_local = 1;
+        return true;
+    }
     __device__ __noinline__ bool fail() const {
         *abort_local = 1;
         atomicOr(const_cast<unsigned *>(abort_global), 1u);
         atomicOr(&g_pipe_error, 1u);
         return false;
     }
+    __device__ __forceinline__ long long poll_every() const { return limit < 4 * kGlobalPoll ? limit / 4 + 1 : kGlobalPoll; }
     __device__ __forceinline__ bool wait(int i, uint32_t parity) const {
         if (mbar_try_wait(&bar[i], parity)) return true;
         const long long t0 = clock64();
+        long long next_poll = t0 + poll_every();
         const uint32_t hint = limit < (1ll << 24) ? 200u : 20000u;
         for (;;) {
             if (mbar_try_wait_suspend(&bar[i], parity, hint)) return true;
             if (aborted()) return false;
-            if (clock64() - t0 > limit) return fail();
+            const long long now = clock64();
+            if (now >= next_poll) {
+                if (poll_global()) return false;
+                next_poll = now + poll_every();
+            }
+            if (now - t0 > limit) return fail();
         }
     }
-    // Waits until *p >= target (one thread; acquire).
-    __device__ __forceinline__ bool wait_flag(const unsigned *p, unsigned target) const {
-        if (ld_acquire(p) >= target) return true;
+    // Waits until *p >= target (one thread; acquire once seen).  The pause between
+    // polls doubles from 32 ns up to max_sleep ns, so that many waiters do not load
+    // the memory system with polls while they have long to wait.
+    __device__ __forceinline__ bool wait_flag(const unsigned *p, unsigned target, unsigned max_sleep) const {
+        if (ld_relaxed(p) >= target) { fence_acquire_gpu(); return true; }
         const long long t0 = clock64();
+        long long next_poll = t0 + poll_every();
+        unsigned pause = 32;
         for (;;) {
-            __nanosleep(64);
-            if (ld_acquire(p) >= target) return true;
+            __nanosleep(pause);
+            pause = min(2 * pause, max_sleep);
+            if (ld_relaxed(p) >= target) { fence_acquire_gpu(); return true; }
             if (aborted()) return false;
-            if (clock64() - t0 > limit) return fail();
+            const long long now = clock64();
+            if (now >= next_poll) {
+                if (poll_global()) return false;
+                next_poll = now + poll_every();
+            }
+            if (now - t0 > limit) return fail();
         }
+    }
+    // For polling loops: true once this CTA or (checked every kGlobalPoll clocks)
+    // the launch has aborted.
+    __device__ __forceinline__ bool aborted_polled(long long &next_poll) const {
+        if (aborted()) return true;
+        const long long now = clock64();
+        if (now < next_poll) return false;
+        next_poll = now + poll_every();
+        return poll_global();
     }
 };
 
@@ -221,6 +306,13 @@ __device__ __forceinline__ void load_gates_pipe(const PipeParams &p, int b, int 
     b0 = r < Ln ? p.beta[gi] : 0.f;
     a1 = r + 1 < Ln ? p.alpha[gi + p.Hv] : 1.f;
     b1 = r + 1 < Ln ? p.beta[gi + p.Hv] : 0.f;
+}
+
+// One arrival per warp (after the warp's lanes are done): an mbarrier serialises
+// arrivals, so 128 or 256 thread arrivals would add hundreds of clocks to a hand-off.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
 // Where chunk counter n of chain CTA x lives: head wave k = n / nchunks, chunk c.
@@ -246,8 +338,7 @@ __device__ __forceinline__ int chain_units(const PipeParams &p, int x) {
 
 // ============================================================================ chain
 __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorMap *tm_q,
-                                           const CUtensorMap *tm_v, const CUtensorMap *tm_o,
-                                           const PipeParams &p, unsigned char *sm)
+                                        const CUtensorMap *tm_v, const PipeParams &p, unsigned char *sm)
 {
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_CBAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_CMISC);
@@ -263,7 +354,6 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         prefetch_tensormap(tm_k);
         prefetch_tensormap(tm_q);
         prefetch_tensormap(tm_v);
-        prefetch_tensormap(tm_o);
         for (int i = 0; i < (int)CH_NBAR; ++i) mbar_init(&bar[i], chain_bar_count(i));
         *abort_local = 0;
         fence_mbar_init();
@@ -281,9 +371,9 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         // ============================================================ input TMA
         if (lane == 0) {
             int nkq = 0, nv = 0;
-            long long idle_since = clock64();
+            long long idle_since = clock64(), next_poll = idle_since;
             while (nkq < N || nv < N) {
-                if (ctl.aborted()) break;
+                if (ctl.aborted_polled(next_poll)) break;
                 bool issued = false;
                 if (nkq < N && (nkq < NKQ || mbar_test(&bar[C_KQ_EMPTY + nkq % NKQ], ((nkq / NKQ) - 1) & 1))) {
                     const Unit u = unit_of(p, x, nkq);
@@ -326,260 +416,179 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     mbar_wait(&bar[C_V_FULL + (m & 1)], (m >> 1) & 1, 1ll << 28);
             }
         }
-    } else if (warp == 1) {
-        // ============================================================ MMA issuer
-        //   YS(n): S^T += (U^T diag(g)) K, O^T += U^T P^T        needs U^T bf16 of n
-        //   UO(n): U^T += S^T (-W)^T, O^T = S^T Q~^T             needs S^T bf16, W, Q~ of n
-        //   WU(n): W^T = K^T Bw^T, U~^T = V^T Bu^T              needs K, V, ring slot of n
-        if (lane == 0) {
-            int nwu = 0, nuo = 0, nys = 0;
-            long long idle_since = clock64();
-            while (nys < N) {
-                if (ctl.aborted()) break;
-                bool issued = false;
-                if (nys < nuo && mbar_test(&bar[C_U_READY + (nys & 1)], (nys >> 1) & 1)) {
-                    const int n = nys, s = n & 1;
-                    tc_fence_after();
-                    // (compact loops: the issuing warp's code stays in the instruction cache)
-                    const uint64_t bk = smem_desc_sw128(sbase + OFF_KQ + (n % NKQ) * KQ_STAGE, 2 * TILE, 1024);
-#pragma unroll 1
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16_ts(tmem + COL_S, tmem + COL_UG + s * 32 + k * 8, bk + (uint64_t)(k * 128),
-                                    ID_S, true);
-                    mma_commit(&bar[C_S_FULL]);
-                    mma_commit(&bar[C_KQ_EMPTY + n % NKQ]);
-                    const uint64_t bp = smem_desc_sw128(sbase + OFF_RB + s * RS_BYTES + RS_P, 16, 1024);
-#pragma unroll 1
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16_ts(tmem + COL_O + s * 64, tmem + COL_U + s * 64 + k * 8, bp + (uint64_t)(k * 2),
-                                    ID_O, true);
-                    mma_commit(&bar[C_O_FULL + s]);
-                    mma_commit(&bar[C_RB_EMPTY + s]);
-                    PTRACE(n, 4, x == 0);
-                    ++nys;
-                    issued = true;
-                } else if (nuo < nwu && mbar_test(&bar[C_S_READY], nuo & 1) &&
-                           mbar_test(&bar[C_QT_READY + (nuo & 1)], (nuo >> 1) & 1) &&
-                           (nuo < 2 || mbar_test(&bar[C_O_FREE + (nuo & 1)], ((nuo >> 1) - 1) & 1))) {
-                    const int n = nuo, s = n & 1;
-                    const uint32_t st = sbase + OFF_KQ + (n % NKQ) * KQ_STAGE;
-                    tc_fence_after();
-                    const uint64_t bw = smem_desc_sw128(sbase + OFF_W, 2 * TILE, 1024);
-                    PMMA(n, 0, x == 0);
-#pragma unroll 1
-                    for (int k = 0; k < 8; ++k) {
-                        mma_bf16_ts(tmem + COL_U + s * 64, tmem + COL_W + k * 8, bw + (uint64_t)(k * 128), ID_U, true);
-                        PMMA(n, 1 + k, x == 0);
-                    }
-                    mma_commit(&bar[C_U_FULL]);
-                    PMMA(n, 9, x == 0);
-                    const uint64_t bq = smem_desc_sw128(st + TILE, 16, 1024);
-#pragma unroll 1
-                    for (int k = 0; k < 8; ++k) {
-                        mma_bf16_ts(tmem + COL_O + s * 64, tmem + COL_W + k * 8,
-                                    bq + (uint64_t)(((k >> 2) * 2 * TILE + (k & 3) * 32) >> 4), ID_O, k > 0);
-                        PMMA(n, 10 + k, x == 0);
-                    }
-                    mma_commit(&bar[C_X_FULL]);
-                    PMMA(n, 18, x == 0);
-                    PTRACE(n, 3, x == 0);
-                    ++nuo;
-                    issued = true;
-                } else if (nwu < N && mbar_test(&bar[C_KQ_FULL + nwu % NKQ], (nwu / NKQ) & 1) &&
-                           mbar_test(&bar[C_V_FULL + (nwu & 1)], (nwu >> 1) & 1) &&
-                           mbar_test(&bar[C_RB_FULL + (nwu & 1)], (nwu >> 1) & 1) &&
-                           // UO of n-1 (last reader of the S^T bf16 in the W^T columns) done;
-                           // so are the YS MMAs of n-2 (readers of this U^T buffer), issued before it
-                           (nwu < 1 || mbar_test(&bar[C_X_FULL], (nwu - 1) & 1))) {
-                    const int n = nwu, s = n & 1;
-                    const uint32_t st = sbase + OFF_KQ + (n % NKQ) * KQ_STAGE;
-                    const uint32_t rb = sbase + OFF_RB + s * RS_BYTES;
-                    const uint32_t vb = sbase + OFF_V + s * 2 * TILE;
-                    tc_fence_after();
-                    const uint64_t ak = smem_desc_sw128(st, 2 * TILE, 1024);
-                    const uint64_t bbw = smem_desc_sw128(rb + RS_BW, 16, 1024);
-#pragma unroll 1
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16(tmem + COL_W, ak + (uint64_t)(k * 128), bbw + (uint64_t)(k * 2), ID_W, k > 0);
-                    const uint64_t av = smem_desc_sw128(vb, TILE, 1024);
-                    const uint64_t bbu = smem_desc_sw128(rb + RS_BU, 16, 1024);
-#pragma unroll 1
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16(tmem + COL_U + s * 64, av + (uint64_t)(k * 128), bbu + (uint64_t)(k * 2), ID_UT, k > 0);
-                    mma_commit(&bar[C_W_FULL + s]);
-                    mma_commit(&bar[C_V_EMPTY + s]);
-                    PTRACE(n, 2, x == 0);
-                    ++nwu;
-                    issued = true;
-                }
-                if (issued) {
-                    idle_since = clock64();
-                } else {
-                    __nanosleep(32);
-                    if (clock64() - idle_since > p.wait_limit) {
-                        ctl.fail();
-                        break;
-                    }
-                }
+    } else if (warp == 1 || warp == 3) {
+        // ============================================================ MMA issuers
+        // Two threads issue, so that issuing one group never waits behind another:
+        //   warp 1 (critical chain)  UG(n)   U^T += S^T (-W)^T   8 MMAs
+        //                            SG(n)   S^T += (U diag(g))^T K  4 MMAs
+        //   warp 3 (the rest)        XG(n)   O^T  = S^T Q^T      8 MMAs  after UG(n) is issued
+        //                            OG(n)   O^T += U^T P^T      4 MMAs  after SG(n) is issued
+        //                            UT(n+2) U~^T = V^T Bu^T     4 MMAs  once S and O MMAs of n are done
+        // U~ of a chunk is so computed two chunks ahead of its UG, and XG / OG queue
+        // behind UG / SG in the tensor pipe.  Every barrier waited on here is one of a
+        // pair (or a ring), so that no wait can miss its phase: the next phase of each
+        // depends on the group the wait gates.  Both threads wait by suspending
+        // (try_wait), which leaves the shared-memory pipe to the other warps.
+        if (lane == 0 && warp == 1) {
+            bool ok = true;
+            for (int n = 0; n < N && ok; ++n) {
+                const int s = n & 1;
+                const uint32_t st = sbase + OFF_KQ + (n % NKQ) * KQ_STAGE;
+                const uint32_t rb = sbase + OFF_RB + (n % NRB) * RS_TILES;
+                // UG(n): S^T bf16 of n, U~^T of n done (its ring slot is then loaded too)
+                if (!(ok = ctl.wait(C_UT_FULL + s, (n >> 1) & 1))) break;
+                if (!(ok = ctl.wait(C_S_READY + s, (n >> 1) & 1))) break;
+                PTRACE(n, 13, x == 0);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    mma_bf16_ts(tmem + COL_U + s * 64, tmem + COL_SB + s * 64 + k * 8,
+                                smem_desc_sw128(rb + RS_W + k * 2048, 2 * TILE, 1024), ID_U, true);
+                mma_commit(&bar[C_U_FULL]);
+                mbar_arrive(&bar[C_X_GO + s]);
+                PTRACE(n, 3, x == 0);
+                // SG(n): (U diag(g))^T bf16 of n
+                if (!(ok = ctl.wait(C_U_READY + s, (n >> 1) & 1))) break;
+                PTRACE(n, 24, x == 0);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ts(tmem + COL_S, tmem + COL_U + s * 64 + 32 + k * 8,
+                                smem_desc_sw128(st + k * 2048, 2 * TILE, 1024), ID_S, true);
+                mma_commit(&bar[C_S_FULL]);
+                mma_commit(&bar[C_KQ_EMPTY + n % NKQ]);
+                mma_commit(&bar[C_RB_EMPTY + n % NRB]);
+                mbar_arrive(&bar[C_O_GO + s]);
+                PTRACE(n, 4, x == 0);
             }
             mma_commit(&bar[C_DRAIN]);
-            mbar_wait(&bar[C_DRAIN], 0, 1ll << 30);
+        } else if (lane == 0 && warp == 3) {
+            bool ok = true;
+            auto issue_ut = [&](int n) -> bool {       // U~^T of chunk n into U buffer n & 1
+                const int s = n & 1;
+                if (!ctl.wait(C_V_FULL + s, (n >> 1) & 1) || !ctl.wait(C_RB_FULL + n % NRB, (n / NRB) & 1))
+                    return false;
+                // the buffer's last readers, SG(n-2) and OG(n-2), are done
+                if (n >= 2 && !ctl.wait(C_KQ_EMPTY + (n - 2) % NKQ, ((n - 2) / NKQ) & 1)) return false;
+                tc_fence_after();
+                const uint32_t vb = sbase + OFF_V + s * 2 * TILE;
+                const uint32_t rb = sbase + OFF_RB + (n % NRB) * RS_TILES;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem + COL_U + s * 64, smem_desc_sw128(vb + k * 2048, TILE, 1024),
+                             smem_desc_sw128(rb + RS_BU + k * 32, 16, 1024), ID_UT, k > 0);
+                mma_commit(&bar[C_V_EMPTY + s]);
+                mma_commit(&bar[C_UT_FULL + s]);
+                PTRACE(n, 2, x == 0);
+                return true;
+            };
+            if (N > 0) ok = issue_ut(0);
+            if (N > 1 && ok) ok = issue_ut(1);
+            for (int n = 0; n < N && ok; ++n) {
+                const int s = n & 1;
+                const uint32_t st = sbase + OFF_KQ + (n % NKQ) * KQ_STAGE;
+                const uint32_t rb = sbase + OFF_RB + (n % NRB) * RS_TILES;
+                // XG(n): after UG(n) is issued; S^T bf16 of n, O buffer read out
+                if (!(ok = ctl.wait(C_X_GO + s, (n >> 1) & 1))) break;
+                if (!(ok = ctl.wait(C_S_READY + s, (n >> 1) & 1))) break;
+                if (n >= 2 && !(ok = ctl.wait(C_O_FREE + s, ((n >> 1) - 1) & 1))) break;
+                PTRACE(n, 14, x == 0);
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t koff = (k >> 2) * 2 * TILE + (k & 3) * 32;
+                    mma_bf16_ts(tmem + COL_O + s * 64, tmem + COL_SB + s * 64 + k * 8,
+                                smem_desc_sw128(st + TILE + koff, 16, 1024), ID_O, k > 0);
+                }
+                mma_commit(&bar[C_X_FULL + s]);
+                PTRACE(n, 15, x == 0);
+                // OG(n): after SG(n) is issued; U^T bf16 of n, S-part scaled by gamma
+                if (!(ok = ctl.wait(C_O_GO + s, (n >> 1) & 1))) break;
+                if (!(ok = ctl.wait(C_U_READY + s, (n >> 1) & 1))) break;
+                if (!(ok = ctl.wait(C_XS_READY + s, (n >> 1) & 1))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ts(tmem + COL_O + s * 64, tmem + COL_U + s * 64 + k * 8,
+                                smem_desc_sw128(rb + RS_P + k * 32, 16, 1024), ID_O, true);
+                mma_commit(&bar[C_O_FULL + s]);
+                mma_commit(&bar[C_RB_EMPTY + n % NRB]);
+                mma_commit(&bar[C_KQ_EMPTY + n % NKQ]);
+                PTRACE(n, 26, x == 0);
+                // UT(n+2), ahead of its UG
+                if (n + 2 < N && !(ok = issue_ut(n + 2))) break;
+            }
+            mma_commit(&bar[C_DRAIN]);
         }
+        if (lane == 0) mbar_wait(&bar[C_DRAIN], 0, 1ll << 30);
     } else if (warp == 2) {
         // ============================================================ ring loader
+        // The ready flag of chunk n is read (acquire) before waiting for its buffer,
+        // so that its round trip overlaps that wait; chunk n's slot is handed back to
+        // the prep (consumed counter) once its copy has landed, checked one chunk later.
         if (lane == 0) {
             const unsigned char *ring = p.ring + (size_t)x * kRing * RS_BYTES;
-            const unsigned *ready = p.ready + (size_t)x * kRing;
-            int pending = -1;        // a load issued but not yet seen landed
-            for (int n = 0; n < N; ++n) {
-                const int s = n & 1;
-                if (n >= 2 && !ctl.wait(C_RB_EMPTY + s, ((n >> 1) - 1) & 1)) break;
+            const unsigned *ready = p.ready + (size_t)x * kFlagWords;
+            int issued = 0;          // copies issued
+            bool ok = true;
+            for (int n = 0; n < N && ok; ++n) {
+                const int r = n % NRB;
+                const unsigned flag = ld_acquire(&ready[n % kRing]);
+                if (n >= NRB && !(ok = ctl.wait(C_RB_EMPTY + r, ((n / NRB) - 1) & 1))) break;
                 PTRACE(n, 12, x == 0);
-                if (!ctl.wait_flag(&ready[n % kRing], (unsigned)n + 1u)) break;
+                if (flag < (unsigned)n + 1u && !(ok = ctl.wait_flag(&ready[n % kRing], (unsigned)n + 1u, 64))) break;
                 PTRACE(n, 0, x == 0);
+                PCHAIN(x, n, 1, true);
                 fence_proxy_async_global();
-                mbar_arrive_expect_tx(&bar[C_RB_FULL + s], RS_LOAD);
-                bulk_load(sm + OFF_RB + s * RS_BYTES, ring + (size_t)(n % kRing) * RS_BYTES, RS_LOAD,
-                          &bar[C_RB_FULL + s]);
-                pending = n;
-                if (!ctl.wait(C_RB_FULL + s, (n >> 1) & 1)) break;
-                pending = -1;
-                PTRACE(n, 1, x == 0);
-                st_release(&p.consumed[x], (unsigned)n + 1u);   // the slot may be refilled
-            }
-            if (pending >= 0) mbar_wait(&bar[C_RB_FULL + (pending & 1)], (pending >> 1) & 1, 1ll << 28);
-        }
-    } else if (warp >= 4 && warp < 8) {
-        // ============================================================ helper warpgroup
-        // Q~ = diag(gamma) Q in place for the UO MMAs, and the O epilogue (TMEM ->
-        // bf16 tile [r][j] by stmatrix -> one TMA store per chunk; row stores for a
-        // chunk cut by the end of the sequence).
-        const int pt = tid - 128;
-        const int q4 = warp & 3;
-        const int j = q4 * 32 + lane;
-        const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
-        const bool leader = pt == 0;
-        const size_t row_stride = (size_t)p.Hv * kHeadDim;
-        bool ok = true;
-        auto epilogue = [&](int n) -> bool {
-            if (leader) bulk_wait_group_read0();     // the previous store has read the staging tile
-            if (!named_and(1, 128, ctl.wait(C_O_FULL + (n & 1), (n >> 1) & 1))) return false;
-            tc_fence_after();
-            const Unit u = unit_of(p, x, n);
-            const uint32_t col_o = COL_O + (n & 1) * 64;
-            const int rows = min(C, p.T - u.c * C);
-            if (rows == C) {
-                const uint32_t stage = smem_u32(sm + OFF_OST);
-                const int mt = lane >> 3, mi = lane & 7;
-                auto emit = [&](const uint32_t *rr, int sl, int cb) {
-#pragma unroll
-                    for (int kk = 0; kk < 2; ++kk) {
-                        uint32_t m[4];
-#pragma unroll
-                        for (int mm = 0; mm < 4; ++mm) {
-                            const int k = 2 * kk + (mm >> 1), g = mm & 1;
-                            m[mm] = pack_bf16x2(__uint_as_float(rr[4 * k + 2 * g]),
-                                                __uint_as_float(rr[4 * k + 2 * g + 1]));
-                        }
-                        const int k = 2 * kk + (mt >> 1), g = mt & 1;
-                        const int orow = 32 * cb + 8 * k + mi;
-                        const int jst = q4 * 32 + 16 * sl + 8 * g;
-                        stmatrix_x4_trans(stage + (jst >> 6) * TILE + sw128_chunk(orow, (jst & 63) >> 3),
-                                          m[0], m[1], m[2], m[3]);
-                    }
-                };
-#pragma unroll 1
-                for (int sl = 0; sl < 2; ++sl) {
-                    uint32_t ra[16], rb[16];
-                    const uint32_t ta = tmem + ((uint32_t)(q4 * 32 + 16 * sl) << 16) + col_o;
-                    tmem_ld16x256b_x4(ta, ra);
-                    tmem_ld16x256b_x4(ta + 32, rb);
-                    tmem_wait_ld();
-                    emit(ra, sl, 0);
-                    emit(rb, sl, 1);
+                const unsigned char *src = ring + (size_t)(n % kRing) * RS_BYTES;
+                mbar_arrive_expect_tx(&bar[C_RB_FULL + r], RS_TILES + RS_GATE_BYTES);
+                bulk_load(sm + OFF_RB + r * RS_TILES, src, RS_TILES, &bar[C_RB_FULL + r]);
+                bulk_load(sm + OFF_RG + r * RS_GATE_BYTES, src + RS_GATE, RS_GATE_BYTES, &bar[C_RB_FULL + r]);
+                issued = n + 1;
+                if (n >= 1) {                        // chunk n - 1's copy has landed: free its slot
+                    if (!(ok = ctl.wait(C_RB_FULL + (n - 1) % NRB, ((n - 1) / NRB) & 1))) break;
+                    PTRACE(n - 1, 1, x == 0);
+                    PCHAIN(x, n - 1, 2, true);
+                    st_release(&p.consumed[(size_t)x * kFlagWords], (unsigned)n);
                 }
-                tc_fence_before();
-                mbar_arrive(&bar[C_O_FREE + (n & 1)]);
-                fence_proxy_async_smem();
-                named_sync(1, 128);
-                if (leader) {
-                    tma_store_4d(tm_o, sm + OFF_OST, 0, u.h, u.c * C, u.b);
-                    tma_store_4d(tm_o, sm + OFF_OST + TILE, 64, u.h, u.c * C, u.b);
-                    bulk_commit_group();
-                }
-                return true;
             }
-            __nv_bfloat16 *dst = p.o + ((size_t)u.b * p.T + (size_t)u.c * C) * row_stride +
-                                 (size_t)u.h * kHeadDim + j;
-#pragma unroll 1
-            for (int r0 = 0; r0 < C; r0 += 32) {
-                float ov[32];
-                tmem_ld32(t_row + col_o + r0, ov);
-                tmem_wait_ld();
-#pragma unroll
-                for (int xx = 0; xx < 32; ++xx)
-                    if (r0 + xx < rows) dst[(size_t)(r0 + xx) * row_stride] = __float2bfloat16_rn(ov[xx]);
-            }
-            tc_fence_before();
-            mbar_arrive(&bar[C_O_FREE + (n & 1)]);
-            return true;
-        };
-        for (int n = 0; n < N && ok; ++n) {
-            const int s = n & 1;
-            ok = ctl.wait(C_KQ_FULL + n % NKQ, (n / NKQ) & 1) && ctl.wait(C_RB_FULL + s, (n >> 1) & 1);
-            ok = named_and(1, 128, ok);
-            if (!ok) break;
-            {
-                const float *gam = reinterpret_cast<const float *>(sm + OFF_RB + s * RS_BYTES + RS_GATE);
-                const int i = pt >> 1, half = pt & 1;
-                unsigned char *qt = sm + OFF_KQ + (n % NKQ) * KQ_STAGE + (2 * half + 1) * TILE;
-                scale_row_bf16(qt, qt, i, gam[i]);
-            }
-            fence_proxy_async_smem();
-            PTRACE(n, 9, x == 0 && pt == 0);
-            mbar_arrive(&bar[C_QT_READY + s]);
-            mbar_arrive(&bar[C_RB_EMPTY + s]);
-            if (n > 0 && !(ok = epilogue(n - 1))) break;
-            PTRACE(n - 1, 10, x == 0 && pt == 0);
+            if (ok && issued > 0 && ctl.wait(C_RB_FULL + (issued - 1) % NRB, ((issued - 1) / NRB) & 1))
+                st_release(&p.consumed[(size_t)x * kFlagWords], (unsigned)issued);
+            // on an abort, let the copies in flight land before the CTA's memory goes away
+            for (int m = issued - 1; m >= 0 && m >= issued - NRB; --m)
+                mbar_wait(&bar[C_RB_FULL + m % NRB], (m / NRB) & 1, 1ll << 28);
         }
-        if (ok && N > 0) ok = epilogue(N - 1);
-        if (leader) bulk_wait_group0();
-    } else if (warp >= 8 && warp < 12) {
-        // ============================================================ chain warpgroup
+    } else if (warp >= 4 && warp < 12) {
+        // ============================================================ conversion warpgroups
+        // Warpgroup h (0: warps 4-7, 1: warps 8-11) owns state columns (key dims)
+        // 64h .. 64h+63 and U^T columns (chunk rows) 32h .. 32h+31.
+        const int h2 = (warp - 4) >> 2;
         const int q4 = warp & 3;
-        const int j = q4 * 32 + lane;                 // TMEM lane = value column j (W^T: key dim d)
+        const int j = q4 * 32 + lane;                 // TMEM lane = value column j
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
+        const int nb = 1 + h2;                        // this warpgroup's named barrier
         const size_t hstate = (size_t)kHeadDim * kHeadDim;
+        const int d0 = 64 * h2;
         bool ok = true;
         for (int n = 0; n < N && ok; ++n) {
             const int s = n & 1;
             const Unit u = unit_of(p, x, n);
-            const float *gv = reinterpret_cast<const float *>(sm + OFF_RB + s * RS_BYTES + RS_GATE);
-            // W^T (TMEM, lane d) -> W [d][r] bf16 (MN-major B of the U MMAs); the U MMAs
-            // of n-1, the last readers of the W tile, have completed (U_FULL, waited in n-1)
-            ok = named_and(2, 128, ctl.wait(C_W_FULL + s, (n >> 1) & 1));
-            if (!ok) break;
-            PTRACE(n, 5, x == 0 && j == 0);
-            tc_fence_after();
-            {
-                float w0[32], w1[32];
-                tmem_ld32(t_row + COL_W, w0);
-                tmem_ld32(t_row + COL_W + 32, w1);
-                tmem_wait_ld();
-                store_half_row_bf16(sm + OFF_W, j, 0, w0);
-                store_half_row_bf16(sm + OFF_W, j, 1, w1);
-            }
+            const float *gv = reinterpret_cast<const float *>(sm + OFF_RG + (n % NRB) * RS_GATE_BYTES);
+            // S^T bf16 buffer s was last read by UG(n-2) (U_FULL, waited then) and XG(n-2);
             // the previous chunk's state update is done (for a new head: the previous
             // head's last one, whose final state was stored below)
-            if (n > 0) ok = ctl.wait(C_S_FULL, (n - 1) & 1);
-            ok = ok && ctl.wait(C_RB_FULL + s, (n >> 1) & 1);
-            ok = named_and(2, 128, ok);
+            if (n >= 2) ok = ctl.wait(C_X_FULL + s, ((n >> 1) - 1) & 1);
+            if (n > 0) ok = ok && ctl.wait(C_S_FULL, (n - 1) & 1);
+            ok = ok && ctl.wait(C_RB_FULL + n % NRB, (n / NRB) & 1);
+            ok = named_and(nb, 128, ok);
             if (!ok) break;
             tc_fence_after();
+            PTRACE(n, 5, x == 0 && j == 0 && h2 == 0);
+            PCHAIN(x, n, 0, j == 0 && h2 == 0);
             if (u.c == 0) {   // a new head: S^T[j][d] = S0[d][j] (zeros without S0)
                 const float *src = p.S0 ? p.S0 + ((size_t)u.b * p.Hv + u.h) * hstate : nullptr;
 #pragma unroll 1
-                for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
+                for (int c0 = d0; c0 < d0 + 64; c0 += 32) {
                     float v[32];
 #pragma unroll
                     for (int xx = 0; xx < 32; ++xx) v[xx] = src ? src[(size_t)(c0 + xx) * kHeadDim + j] : 0.f;
@@ -587,63 +596,72 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 }
                 tmem_wait_st();
             }
-            // S^T -> packed bf16 A operand in the (read) W^T columns; S^T <- gamma_{C-1} S^T
-            const float glast = gv[C - 1];
-#pragma unroll 1
-            for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
-                float v[32];
-                uint32_t pk[16];
-                tmem_ld32(t_row + COL_S + c0, v);
+            // S^T -> packed bf16 A operand (buffer s); S^T <- gamma_{C-1} S^T
+            {
+                const float glast = gv[C - 1];
+                float v[64];
+                uint32_t pk[32];
+                tmem_ld32(t_row + COL_S + d0, v);
+                tmem_ld32(t_row + COL_S + d0 + 32, v + 32);
                 tmem_wait_ld();
 #pragma unroll
-                for (int xx = 0; xx < 16; ++xx) pk[xx] = pack_bf16x2(v[2 * xx], v[2 * xx + 1]);
-                tmem_st16u(t_row + COL_W + (c0 >> 1), pk);
+                for (int xx = 0; xx < 32; ++xx) pk[xx] = pack_bf16x2(v[2 * xx], v[2 * xx + 1]);
+                tmem_st32u(t_row + COL_SB + s * 64 + (d0 >> 1), pk);
 #pragma unroll
-                for (int xx = 0; xx < 32; ++xx) v[xx] *= glast;
-                tmem_st32(t_row + COL_S + c0, v);
+                for (int xx = 0; xx < 64; ++xx) v[xx] *= glast;
+                tmem_st32(t_row + COL_S + d0, v);
+                tmem_st32(t_row + COL_S + d0 + 32, v + 32);
             }
             tmem_wait_st();
-            fence_proxy_async_smem();                // the W tile, for the tensor core
             tc_fence_before();
-            mbar_arrive(&bar[C_S_READY]);
-            PTRACE(n, 6, x == 0 && j == 0);
-            // U^T -> packed bf16 A operands in place: U^T (columns 0-31 of its buffer)
-            // for the O update, U^T diag(g) (columns 32-63) for the state update
-            ok = named_and(2, 128, ctl.wait(C_U_FULL, n & 1));
+            warp_arrive(&bar[C_S_READY + s]);
+            PTRACE(n, 6, x == 0 && j == 0 && h2 == 0);
+            PCHAIN(x, n, 4, j == 0 && h2 == 0);
+            PTRACE(n, 27, x == 0 && j == 127 && h2 == 1);
+            // U^T (fp32, 64 columns) -> two packed bf16 copies in place: U^T (columns
+            // 0-31, for the O MMAs) and (U diag(g))^T (columns 32-63, for the state
+            // update, so that K needs no scaling).  Both warpgroups load their half
+            // before either writes (the packed copies overlap the fp32 halves).  The
+            // wait is agreed by both warpgroups together, so that either both reach the
+            // barrier between loads and stores or neither does.
+            ok = named_and(3, 256, ctl.wait(C_U_FULL, n & 1));
             if (!ok) break;
-            PTRACE(n, 7, x == 0 && j == 0);
+            PTRACE(n, 7, x == 0 && j == 0 && h2 == 0);
+            PCHAIN(x, n, 5, j == 0 && h2 == 0);
             tc_fence_after();
-#pragma unroll 1
-            for (int c0 = 0; c0 < C; c0 += 32) {   // packed U^T in place: writes trail reads
+            {
                 float uu[32];
                 uint32_t pk[16];
-                tmem_ld32(t_row + COL_U + s * 64 + c0, uu);
+                tmem_ld32(t_row + COL_U + s * 64 + 32 * h2, uu);
                 tmem_wait_ld();
+                named_sync(3, 256);
 #pragma unroll
                 for (int xx = 0; xx < 16; ++xx) pk[xx] = pack_bf16x2(uu[2 * xx], uu[2 * xx + 1]);
-                tmem_st16u(t_row + COL_U + s * 64 + (c0 >> 1), pk);
-                const float4 *g4 = reinterpret_cast<const float4 *>(gv + C + c0);
+                tmem_st16u(t_row + COL_U + s * 64 + 16 * h2, pk);
+                const float *gg = gv + C + 32 * h2;   // g_r of this half's rows r
 #pragma unroll
-                for (int xx = 0; xx < 8; ++xx) {
-                    const float4 g = g4[xx];
-                    pk[2 * xx] = pack_bf16x2(uu[4 * xx] * g.x, uu[4 * xx + 1] * g.y);
-                    pk[2 * xx + 1] = pack_bf16x2(uu[4 * xx + 2] * g.z, uu[4 * xx + 3] * g.w);
-                }
-                tmem_st16u(t_row + COL_UG + s * 32 + (c0 >> 1), pk);
+                for (int xx = 0; xx < 16; ++xx)
+                    pk[xx] = pack_bf16x2(uu[2 * xx] * gg[2 * xx], uu[2 * xx + 1] * gg[2 * xx + 1]);
+                tmem_st16u(t_row + COL_U + s * 64 + 32 + 16 * h2, pk);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&bar[C_U_READY + s]);
-            mbar_arrive(&bar[C_RB_EMPTY + s]);      // gamma, g of n no longer read
-            PTRACE(n, 8, x == 0 && j == 0);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar[C_U_READY + s]);
+                mbar_arrive(&bar[C_RB_EMPTY + n % NRB]);   // gamma of n no longer read here
+            }
+            PTRACE(n, 8, x == 0 && j == 0 && h2 == 0);
+            PCHAIN(x, n, 6, j == 0 && h2 == 0);
+            PTRACE(n, 28, x == 0 && j == 127 && h2 == 1);
             // last chunk of a head: store its final state once the update is done
             if (u.c == nck - 1 && p.S_final) {
-                ok = named_and(2, 128, ctl.wait(C_S_FULL, n & 1));
+                ok = named_and(nb, 128, ctl.wait(C_S_FULL, n & 1));
                 if (!ok) break;
                 tc_fence_after();
                 float *dst = p.S_final + ((size_t)u.b * p.Hv + u.h) * hstate;
 #pragma unroll 1
-                for (int c0 = 0; c0 < kHeadDim; c0 += 32) {
+                for (int c0 = d0; c0 < d0 + 64; c0 += 32) {
                     float v[32];
                     tmem_ld32(t_row + COL_S + c0, v);
                     tmem_wait_ld();
@@ -652,6 +670,70 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 }
                 tc_fence_before();
             }
+        }
+    } else if (warp >= 12) {
+        // ============================================================ helper warpgroup
+        // Per chunk: the S-part of O^T (S^T Q^T, from XG) scaled by gamma_r in TMEM, so
+        // that OG adds P U to diag(gamma) Q S; then the O epilogue (TMEM -> registers
+        // -> bf16 stores of the chunk's rows).  Neither step is on the state chain.
+        const int q4 = warp & 3;
+        const int j = q4 * 32 + lane;
+        const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
+        const size_t row_stride = (size_t)p.Hv * kHeadDim;
+        bool ok = true;
+        for (int n = 0; n < N && ok; ++n) {
+            const int s = n & 1;
+            const uint32_t col_o = COL_O + s * 64;
+            // ---- O^T[j][r] *= gamma_r (XG of n done; OG of n waits for it)
+            ok = named_and(4, 128, ctl.wait(C_X_FULL + s, (n >> 1) & 1) &&
+                                   ctl.wait(C_RB_FULL + n % NRB, (n / NRB) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            PTRACE(n, 9, x == 0 && j == 0);
+            {
+                const float *gam = reinterpret_cast<const float *>(sm + OFF_RG + (n % NRB) * RS_GATE_BYTES);
+                float ov[64];
+                tmem_ld32(t_row + col_o, ov);
+                tmem_ld32(t_row + col_o + 32, ov + 32);
+                tmem_wait_ld();
+#pragma unroll
+                for (int r = 0; r < C; ++r) ov[r] *= gam[r];
+                tmem_st32(t_row + col_o, ov);
+                tmem_st32(t_row + col_o + 32, ov + 32);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar[C_XS_READY + s]);
+                mbar_arrive(&bar[C_RB_EMPTY + n % NRB]);   // gamma of n no longer read here
+            }
+            // ---- epilogue of n
+            ok = named_and(4, 128, ctl.wait(C_O_FULL + s, (n >> 1) & 1));
+            if (!ok) break;
+            tc_fence_after();
+            const Unit u = unit_of(p, x, n);
+            const int rows = min(C, p.T - u.c * C);
+            float ov[64];
+            tmem_ld32(t_row + col_o, ov);
+            tmem_ld32(t_row + col_o + 32, ov + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            warp_arrive(&bar[C_O_FREE + s]);            // the O buffer is free once read out
+            // thread j writes o[t][h][j] of the chunk's rows: each warp store covers 32
+            // consecutive j (64 contiguous bytes)
+            __nv_bfloat16 *dst = p.o + ((size_t)u.b * p.T + (size_t)u.c * C) * row_stride +
+                                 (size_t)u.h * kHeadDim + j;
+            if (rows == C) {
+#pragma unroll
+                for (int r = 0; r < C; ++r) dst[(size_t)r * row_stride] = __float2bfloat16_rn(ov[r]);
+            } else {
+#pragma unroll
+                for (int r = 0; r < C; ++r)
+                    if (r < rows) dst[(size_t)r * row_stride] = __float2bfloat16_rn(ov[r]);
+            }
+            PTRACE(n, 10, x == 0 && j == 0);
+            PCHAIN(x, n, 7, j == 0);
         }
     }
 
@@ -694,8 +776,10 @@ __device__ __forceinline__ int total_items(const PipeParams &p, int g) {
     return total;
 }
 
+// Prep CTA warps: 0 K/Q TMA, 1 MMA issuer (grams per item, W^T per V head), 4-15
+// three V-head warpgroups (warpgroup w takes V heads w, w + 3, ... of each group).
 __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMap *tm_q,
-                                          const PipeParams &p, unsigned char *sm)
+                                       const PipeParams &p, unsigned char *sm)
 {
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_OFF_MISC);
@@ -712,7 +796,8 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
         prefetch_tensormap(tm_k);
         prefetch_tensormap(tm_q);
         for (int i = 0; i < (int)P_NBAR; ++i)
-            mbar_init(&bar[i], (i == P_G_FREE || i == P_G_FREE + 1) ? 128u * kPrepWG : 1u);
+            mbar_init(&bar[i], (i == P_G_FREE || i == P_G_FREE + 1) ? 4u * kPrepWG   // warps
+                               : (i >= P_BW_READY && i < P_BW_READY + kPrepWG) ? 4u : 1u);
         *abort_local = 0;
         fence_mbar_init();
     }
@@ -747,46 +832,110 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
                     mbar_wait(&bar[P_KQ_FULL + (m & 1)], (m >> 1) & 1, 1ll << 28);
         }
     } else if (warp == 1) {
-        // ============================================================ grams
+        // ============================================================ MMA issuer
+        // Polls for work: the grams G = [K;Q] K^T of the next item once its K/Q tiles
+        // have landed and its gram buffer is free, and the W^T = K^T Bw^T product of
+        // any warpgroup whose Bw tile is ready (its heads in item order).  An item's
+        // K/Q stage is released after its last W^T product.
         if (lane == 0) {
-            for (int jj = 0; jj < nmine; ++jj) {
-                const int s = jj & 1;
-                if (!ctl.wait(P_KQ_FULL + s, (jj >> 1) & 1)) break;
-                if (jj >= 2 && !ctl.wait(P_G_FREE + s, ((jj >> 1) - 1) & 1)) break;
-                tc_fence_after();
-                const uint32_t st = sbase + P_OFF_KQ + s * KQ_STAGE;
+            int ng = 0;                                  // items whose grams are issued
+            int wt_item[kPrepWG] = {0, 0, 0};            // per warpgroup: item and head of
+            int wt_head[kPrepWG] = {0, 1, 2};            //   its next W^T product
+            int oldest = 0;                              // oldest item whose stage is held
+            long long idle_since = clock64(), next_poll = idle_since;
+            while (oldest < nmine) {
+                if (ctl.aborted_polled(next_poll)) break;
+                bool issued = false;
+                if (ng < nmine && ng < oldest + NPKQ && mbar_test(&bar[P_KQ_FULL + (ng & 1)], (ng >> 1) & 1) &&
+                    (ng < 2 || mbar_test(&bar[P_G_FREE + (ng & 1)], ((ng >> 1) - 1) & 1))) {
+                    const uint32_t st = sbase + P_OFF_KQ + (ng & 1) * KQ_STAGE;
+                    tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const uint32_t koff = (k >> 2) * 2 * TILE + (k & 3) * 32;
-                    mma_bf16(tmem + s * 64, smem_desc_sw128(st + koff, 16, 1024),
-                             smem_desc_sw128(st + koff, 16, 1024), ID_G, k > 0);
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t koff = (k >> 2) * 2 * TILE + (k & 3) * 32;
+                        mma_bf16(tmem + (ng & 1) * 64, smem_desc_sw128(st + koff, 16, 1024),
+                                 smem_desc_sw128(st + koff, 16, 1024), ID_G, k > 0);
+                    }
+                    mma_commit(&bar[P_G_FULL + (ng & 1)]);
+                    ++ng;
+                    issued = true;
                 }
-                mma_commit(&bar[P_G_FULL + s]);
-                mma_commit(&bar[P_KQ_EMPTY + s]);
+#pragma unroll
+                for (int w = 0; w < kPrepWG; ++w) {
+                    const int jj = wt_item[w], i = wt_head[w];
+                    if (jj >= nmine || jj >= ng || jj >= oldest + NPKQ) continue;
+                    // the (heads_per_wg(w) * jj + i / 3)-th W^T product of warpgroup w
+                    const int use = ((g - w + kPrepWG - 1) / kPrepWG) * jj + i / kPrepWG;
+                    if (!mbar_test(&bar[P_BW_READY + w], use & 1)) continue;
+                    const uint32_t st = sbase + P_OFF_KQ + (jj & 1) * KQ_STAGE;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16(tmem + 128 + 64 * w, smem_desc_sw128(st + k * 2048, 2 * TILE, 1024),
+                                 smem_desc_sw128(sbase + P_OFF_BW + w * TILE + k * 32, 16, 1024), ID_W, k > 0);
+                    mma_commit(&bar[P_WT_FULL + w]);
+                    if (i + kPrepWG < g) {
+                        wt_head[w] = i + kPrepWG;
+                    } else {
+                        wt_item[w] = jj + 1;
+                        wt_head[w] = w;
+                    }
+                    issued = true;
+                }
+                // the oldest item is done once every warpgroup has moved past it
+                bool past = true;
+#pragma unroll
+                for (int w = 0; w < kPrepWG; ++w) past = past && (w >= g || wt_item[w] > oldest);
+                if (past && oldest < ng) {
+                    mma_commit(&bar[P_KQ_EMPTY + (oldest & 1)]);
+                    ++oldest;
+                    issued = true;
+                }
+                if (issued) {
+                    idle_since = clock64();
+                } else {
+                    __nanosleep(32);
+                    if (clock64() - idle_since > p.wait_limit) {
+                        ctl.fail();
+                        break;
+                    }
+                }
             }
             // drain: every issued MMA has completed before TMEM is released
             mma_commit(&bar[P_DRAIN]);
             mbar_wait(&bar[P_DRAIN], 0, 1ll << 30);
         }
-    } else if (warp >= 2) {
+    } else if (warp >= 4) {
         // ============================================================ V-head warpgroups
-        // (warps 2-5, 6-9, 10-13: each four consecutive warps, one per TMEM lane quarter)
-        const int wg = (warp - 2) >> 2;               // 0 .. kPrepWG-1
-        const int pt = tid - 64 - 128 * wg;           // 0 .. 127
+        const int wg = (warp - 4) >> 2;               // 0 .. kPrepWG-1
+        const int pt = tid - 128 - 128 * wg;          // 0 .. 127
         const int nb = 1 + wg;                        // named barrier of this warpgroup
         const int q4 = warp & 3;
-        const int row = q4 * 32 + lane;               // TMEM lane = gram row
+        const int row = q4 * 32 + lane;               // TMEM lane = gram row (W^T: key dim d)
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
         unsigned char *mine = sm + P_OFF_WG + wg * P_WG_BYTES;
         float *sA = reinterpret_cast<float *>(mine);
         float *sY = reinterpret_cast<float *>(mine + P_SA);
         float *gv = reinterpret_cast<float *>(mine + P_SA + P_SY);
+        unsigned char *bw_tile = sm + P_OFF_BW + wg * TILE;
         const bool gate_warp = pt < 32;
+        const int heads_here = (g - wg + kPrepWG - 1) / kPrepWG;   // V heads per item on this warpgroup
+        // The next head's gates (gate warp) and its ring slot's consumed counter
+        // (thread 0) are loaded one head ahead, so their latency overlaps this head.
+        float na0 = 1.f, na1 = 1.f, nb0 = 0.f, nb1 = 0.f;
+        unsigned ncons = 0;
+        auto prefetch = [&](int jj, int i) {
+            if (jj >= nmine || wg >= g) return;
+            const Item it = item_of(p, pidx + jj * p.n_prep, g);
+            const int b = it.hh0 / p.Hv, h = it.hh0 - b * p.Hv + i;
+            if (gate_warp) load_gates_pipe(p, b, h, it.c, lane, na0, na1, nb0, nb1);
+            if (pt == 0) ncons = ld_relaxed(&p.consumed[(size_t)(it.gi * g + i) * kFlagWords]);
+        };
+        prefetch(0, wg);
         bool ok = true;
         for (int jj = 0; jj < nmine && ok; ++jj) {
             const int s = jj & 1;
             const Item it = item_of(p, pidx + jj * p.n_prep, g);
-            const int b = it.hh0 / p.Hv, h0 = it.hh0 - b * p.Hv;
             const int n = it.k * p.nchunks + it.c;     // chunk counter of the chain CTAs
             PTRACE(n, 22, it.gi == 0 && pt == 0 && wg == 0);
             ok = named_and(nb, 128, ctl.wait(P_G_FULL + s, (jj >> 1) & 1));
@@ -795,70 +944,133 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
             tc_fence_after();
             if (wg >= g) {                            // no V head of this group here
                 tc_fence_before();
-                mbar_arrive(&bar[P_G_FREE + s]);
+                warp_arrive(&bar[P_G_FREE + s]);
                 continue;
             }
             for (int i = wg; i < g && ok; i += kPrepWG) {
-                const int h = h0 + i, x = it.gi * g + i;
+                const int x = it.gi * g + i;
                 const bool tr = x == 0 && pt == 0;
+                (void)tr;
                 PTRACE(n, 16, tr);
+                const float a0 = na0, a1 = na1, be0 = nb0, be1 = nb1;
+                const unsigned cons = ncons;
+                if (i + kPrepWG < g) prefetch(jj, i + kPrepWG);
+                else prefetch(jj + 1, wg);
                 // ---- the ring slot of chain CTA x for its chunk n is free once the
                 //      chain has loaded chunk n - kRing
                 bool free_ok = true;
-                if (pt == 0 && n >= kRing) free_ok = ctl.wait_flag(&p.consumed[x], (unsigned)(n - kRing + 1));
+                if (pt == 0 && n >= kRing) {
+                    if (cons >= (unsigned)(n - kRing + 1)) fence_acquire_gpu();
+                    else free_ok = ctl.wait_flag(&p.consumed[(size_t)x * kFlagWords], (unsigned)(n - kRing + 1), 1024);
+                }
                 ok = named_and(nb, 128, free_ok);
                 if (!ok) break;
                 PTRACE(n, 20, tr);
                 unsigned char *slot = p.ring + ((size_t)x * kRing + n % kRing) * RS_BYTES;
                 // ---- gates of (b, h, chunk c)
-                if (gate_warp) {
-                    float a0, a1, b0, b1;
-                    load_gates_pipe(p, b, h, it.c, lane, a0, a1, b0, b1);
-                    compute_gates(gv, a0, a1, b0, b1, lane);
-                }
+                if (gate_warp) compute_gates(gv, a0, a1, be0, be1, lane);
                 named_sync(nb, 128);
                 PTRACE(n, 17, tr);
-                // ---- grams -> A rows (fp32, sA) and P rows (bf16, straight into the slot)
+                // ---- grams -> A rows (fp32, sA) and P rows (bf16, straight into the slot).
+                //      Row r of A is beta_r Gam[r][i] k_r.k_i (i < r), of P Gam[r][i] q_r.k_i
+                //      (i <= r); the decays are running products of alpha along the row from
+                //      column r down (Gam[r][x-1] = Gam[r][x] alpha_x), continued into columns
+                //      below 32 by d31[x] = Gam[31][x].  One 32-column half at a time: the
+                //      high half first, whose running product the low half continues.
                 {
-                    float g0[32], g1[32];
-                    tmem_ld32(t_row + s * 64, g0);
-                    tmem_ld32(t_row + s * 64 + 32, g1);
+                    const int r = row & 63;
+                    const bool is_a = row < 64;
+                    const bool low = r < 32;          // warp-uniform
+                    float run = is_a ? gv[GV_BETA + r] : 1.f;
+                    float gg[32];
+                    tmem_ld32(t_row + s * 64 + 32, gg);
+                    tmem_wait_ld();
+                    if (low) {
+#pragma unroll
+                        for (int xx = 0; xx < 32; ++xx) gg[xx] = 0.f;
+                    } else {
+#pragma unroll
+                        for (int xx = 31; xx >= 0; --xx) {
+                            const int ci = 32 + xx;
+                            const bool on = ci <= r;
+                            const bool keep = is_a ? ci < r : on;
+                            const float val = run * gg[xx];
+                            gg[xx] = keep ? val : 0.f;
+                            run = on ? run * gv[GV_ALPHA + ci] : run;
+                        }
+                    }
+                    if (is_a) {
+                        float4 *dst = reinterpret_cast<float4 *>(sA + r * LDA + 32);
+#pragma unroll
+                        for (int xx = 0; xx < 8; ++xx)
+                            dst[xx] = make_float4(gg[4 * xx], gg[4 * xx + 1], gg[4 * xx + 2], gg[4 * xx + 3]);
+                    } else {
+                        store_half_row_bf16(slot + RS_P, r, 1, gg);
+                    }
+                    tmem_ld32(t_row + s * 64, gg);
                     tmem_wait_ld();
                     if (i + kPrepWG >= g) {           // this warpgroup's last read of the grams
                         tc_fence_before();
-                        mbar_arrive(&bar[P_G_FREE + s]);
+                        warp_arrive(&bar[P_G_FREE + s]);
                     }
-                    ap_row_values(gv, row, g0, g1);
-                    if (row < 64) {
-                        float4 *dst = reinterpret_cast<float4 *>(sA + row * LDA);
+                    if (low) {
+#pragma unroll
+                        for (int xx = 31; xx >= 0; --xx) {
+                            const bool on = xx <= r;
+                            const bool keep = is_a ? xx < r : on;
+                            const float val = run * gg[xx];
+                            gg[xx] = keep ? val : 0.f;
+                            run = on ? run * gv[GV_ALPHA + xx] : run;
+                        }
+                    } else {                          // run = scale * Gam[r][31]
+#pragma unroll
+                        for (int xx = 0; xx < 32; ++xx) gg[xx] = run * gv[GV_D31 + xx] * gg[xx];
+                    }
+                    if (is_a) {
+                        float4 *dst = reinterpret_cast<float4 *>(sA + r * LDA);
 #pragma unroll
                         for (int xx = 0; xx < 8; ++xx)
-                            dst[xx] = make_float4(g0[4 * xx], g0[4 * xx + 1], g0[4 * xx + 2], g0[4 * xx + 3]);
-#pragma unroll
-                        for (int xx = 0; xx < 8; ++xx)
-                            dst[8 + xx] = make_float4(g1[4 * xx], g1[4 * xx + 1], g1[4 * xx + 2], g1[4 * xx + 3]);
+                            dst[xx] = make_float4(gg[4 * xx], gg[4 * xx + 1], gg[4 * xx + 2], gg[4 * xx + 3]);
                     } else {
-                        store_half_row_bf16(slot + RS_P, row - 64, 0, g0);
-                        store_half_row_bf16(slot + RS_P, row - 64, 1, g1);
+                        store_half_row_bf16(slot + RS_P, r, 0, gg);
                     }
                 }
                 named_sync(nb, 128);
                 PTRACE(n, 18, tr);
-                // ---- T = (I + A)^-1
+                // ---- T = (I + A)^-1; Bw = T diag(beta gamma) into this warpgroup's tile
+                //      (the W^T product of its previous head has read it: WT_FULL waited
+                //      there), Bu = T diag(beta) into the slot
                 unit_lower_inverse(sA, sY, pt, nb);
                 PTRACE(n, 19, tr);
-                write_bw_bu(gv, sA, pt, slot + RS_BW, slot + RS_BU);
+                write_bw_bu(gv, sA, pt, bw_tile, slot + RS_BU);
+                fence_proxy_async_smem();
+                warp_arrive(&bar[P_BW_READY + wg]);
+                PTRACE(n, 25, tr);
                 {
                     float *sg = reinterpret_cast<float *>(slot + RS_GATE);
                     sg[pt] = pt < 64 ? gv[GV_GAM + pt] : gv[GV_G + pt - 64];
                 }
-                fence_proxy_async_global();
-                named_sync(nb, 128);
-                if (pt == 0) {
-                    __threadfence();
-                    st_release(&p.ready[(size_t)x * kRing + n % kRing], (unsigned)n + 1u);
+                // ---- W^T (TMEM, lane d) -> W [d][r] bf16 rows into the slot
+                ok = named_and(nb, 128, ctl.wait(P_WT_FULL + wg, (heads_here * jj + i / kPrepWG) & 1));
+                if (!ok) break;
+                PTRACE(n, 29, tr);
+                tc_fence_after();
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float w0[32];
+                    tmem_ld32(t_row + 128 + 64 * wg + 32 * half, w0);
+                    tmem_wait_ld();
+                    store_half_row_bf16(slot + RS_W, row, half, w0);
                 }
+                tc_fence_before();
+                PTRACE(n, 30, tr);
+                // every thread's slot writes come before thread 0's release (the barrier
+                // orders them at CTA scope; the release is cumulative); the chain acquires
+                // the flag and fences the async proxy before its bulk copy reads the slot
+                named_sync(nb, 128);
+                if (pt == 0) st_release(&p.ready[(size_t)x * kFlagWords + n % kRing], (unsigned)n + 1u);
                 PTRACE(n, 21, tr);
+                PCHAIN(x, n, 3, pt == 0);
             }
         }
     }
@@ -873,16 +1085,17 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
 
 __global__ void __launch_bounds__(NT, 1)
 chunk_pipe_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                  const __grid_constant__ PipeParams p)
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ PipeParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     PTRACE(0, 31, blockIdx.x == 0 && threadIdx.x == 0);
+    PCTA(0);
     if ((int)blockIdx.x < p.n_chain)
-        chain_role(&tm_k, &tm_q, &tm_v, &tm_o, p, sm);
+        chain_role(&tm_k, &tm_q, &tm_v, p, sm);
     else
         prep_role(&tm_k, &tm_q, p, sm);
+    PCTA(1);
 }
 
 }  // namespace
@@ -892,10 +1105,11 @@ namespace gdn {
 
 namespace {
 
-// Workspace: [ready: n_chain * kRing][consumed: n_chain][abort] as 32-bit words,
-// then the ring (256-byte aligned).
+// Workspace: 32-bit flag words, one 128-byte line per use (ready flags of each chain
+// CTA, its consumed counter, the abort word: lines that many threads poll share no
+// cache line with one another), then the ring (256-byte aligned).
 constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
-size_t flag_bytes(int n_chain) { return align256(((size_t)n_chain * (kRing + 1) + 1) * sizeof(unsigned)); }
+size_t flag_bytes(int n_chain) { return align256(((size_t)2 * n_chain + 1) * kFlagWords * sizeof(unsigned)); }
 
 int device_sms()
 {
@@ -973,9 +1187,9 @@ cudaError_t launch_chunk_pipe(const ChunkArgs &a, int chain_ctas, long long wait
     if (err != cudaSuccess) return err;
     if ((long long)per_sm * sms < n_chain + n_prep) return cudaErrorCooperativeLaunchTooLarge;
 
-    CUtensorMap tk, tq, tv, to;
+    CUtensorMap tk, tq, tv;
     if (!make_map(&tk, a.k, a.B, a.T, a.Hqk) || !make_map(&tq, a.q, a.B, a.T, a.Hqk) ||
-        !make_map(&tv, a.v, a.B, a.T, a.Hv) || !make_map(&to, a.o, a.B, a.T, a.Hv))
+        !make_map(&tv, a.v, a.B, a.T, a.Hv))
         return cudaErrorInvalidValue;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     unsigned *flags = reinterpret_cast<unsigned *>(ws);
@@ -995,11 +1209,11 @@ cudaError_t launch_chunk_pipe(const ChunkArgs &a, int chain_ctas, long long wait
     p.n_chain = n_chain;
     p.n_prep = n_prep;
     p.ready = flags;
-    p.consumed = flags + (size_t)n_chain * kRing;
-    p.abort = flags + (size_t)n_chain * (kRing + 1);
+    p.consumed = flags + (size_t)n_chain * kFlagWords;
+    p.abort = flags + (size_t)2 * n_chain * kFlagWords;
     p.ring = ws + fb;
     p.wait_limit = wait_limit > 0 ? wait_limit : (1ll << 32);
-    void *args[] = {&tk, &tq, &tv, &to, &p};
+    void *args[] = {&tk, &tq, &tv, &p};
     return cudaLaunchCooperativeKernel((const void *)chunk_pipe_kernel, dim3((unsigned)(n_chain + n_prep)),
                                        dim3(NT), args, SMEM_BYTES, stream);
 }
@@ -1014,6 +1228,12 @@ extern "C" int gdn_pipe_mma_read(long long *host, int n)
 {
     if (n < 8 * 24) return -1;
     return (int)cudaMemcpyFromSymbol(host, g_pmma, sizeof(g_pmma));
+}
+extern "C" int gdn_pipe_grid_read(unsigned long long *cta, unsigned long long *chain)
+{
+    cudaError_t e = cudaMemcpyFromSymbol(cta, g_pcta, sizeof(g_pcta));
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(chain, g_pchain, sizeof(g_pchain));
+    return (int)e;
 }
 extern "C" int gdn_pipe_clock_read(long long *host, int n)
 {

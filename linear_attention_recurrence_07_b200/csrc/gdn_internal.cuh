@@ -41,13 +41,13 @@ cudaError_t launch_decode(const DecodeArgs &a, gdn_dtype dtype, cudaStream_t str
 cudaError_t launch_chunk_simt(const ChunkArgs &a, gdn_dtype dtype, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const ChunkArgs &a, cudaStream_t stream);
 bool chunk_tc_available();
-cudaError_t launch_chunk_tc_cluster(const ChunkArgs &a, cudaStream_t stream);
-bool chunk_tc_cluster_fits(int B, int Hv);   // all B * Hv clusters resident at once
 // Segment-parallel prefill (bf16, tensor cores): each sequence in up to `segments`
 // pieces; workspace of chunk_tc_split_workspace bytes (0: no split needed).
 size_t chunk_tc_split_workspace(int B, int T, int Hv, int segments);
 cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *workspace,
                                   cudaStream_t stream);
+// Scratch gdn_chunk_fwd_split uses for these arguments (0: it will not split).
+size_t split_scratch_needed(int B, int T, int Hv, int dk, int dv, int segments, gdn_dtype dtype);
 // Backward pass (gdn_bwd.cu): gradients of q, k, v, alpha, beta, S0.
 struct BwdLaunch {
     const void *q, *k, *v, *dO;

@@ -9,36 +9,21 @@
 // allocates.  Every call shares that one array, so calls that overlap on the GPU
 // race; nothing in it has to start at zero (every byte the split reads was written
 // earlier in the same call).
-#include <mutex>
-
 #include "gdn_internal.cuh"
 
 namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(48) << 20;   // 48 MiB
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_split_scratch[kStaticScratchBytes];
 
-std::mutex g_scratch_mutex;
-void *g_scratch_addr[kMaxDevices];   // device address of g_split_scratch, per device
-
-// Address of the array on the current device: looked up once per device.
+// Device address of the array in the current device's context.  Looked up on every
+// call (cheap once the module is loaded), so it is never stale: after a context is
+// torn down and created again (cudaDeviceReset), the module and its array may sit
+// at another address.
 cudaError_t scratch_address(void **out)
 {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_addr[dev]) {
-        void *p = nullptr;
-        err = cudaGetSymbolAddress(&p, g_split_scratch);
-        if (err != cudaSuccess) return err;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
-    return cudaSuccess;
+    return cudaGetSymbolAddress(out, g_split_scratch);
 }
 
 }  // namespace
@@ -50,8 +35,8 @@ extern "C" gdn_status gdn_chunk_fwd_split_noalloc(const void *q, const void *k, 
                                                   int chunk, int segments, gdn_dtype dtype,
                                                   void *stream)
 {
-    // only bf16 calls split (and need scratch); the others go straight through
-    const size_t need = dtype == GDN_BF16 ? gdn_chunk_fwd_split_workspace(B, T, Hv, dk, dv, segments) : 0;
+    // the scratch the split itself will use (0 when it goes straight to gdn_chunk_fwd)
+    const size_t need = gdn::split_scratch_needed(B, T, Hv, dk, dv, segments, dtype);
     if (need > kStaticScratchBytes) return GDN_ERR_UNSUPPORTED;
     void *scratch = nullptr;
     if (need > 0) {

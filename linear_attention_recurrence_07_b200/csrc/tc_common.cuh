@@ -1,5 +1,5 @@
-// Device code shared by the tensor-core prefill kernels (single CTA per head and
-// cluster per head): constants, bf16 operand writers, barrier helpers, the blocked
+// Device code shared by the tensor-core prefill kernels (one CTA per head, and the
+// pipelined kernel's prep and chain CTAs): constants, bf16 operand writers, barrier helpers, the blocked
 // triangular inverse, gate loading, and the host-side TMA descriptor builder.
 // Everything is in an anonymous namespace: each kernel file gets its own copy.
 #pragma once
@@ -29,20 +29,8 @@ __device__ __forceinline__ void trace(int c, int slot, bool leader) {
     }
 }
 #define GDN_TRACE_AT(c, slot, leader) trace((c), (slot), (leader))
-// Cluster kernels: both CTAs of cluster (0, 0), chunks kTraceBase .. kTraceBase + 15.
-constexpr int kTraceBase = 24;
-__device__ __forceinline__ void trace_cluster(int c, int slot, bool leader) {
-    const int cc = c - kTraceBase;
-    if (leader && blockIdx.x < 2 && blockIdx.y == 0 && cc >= 0 && cc < kTraceChunks) {
-        unsigned long long t;
-        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-        g_trace[cc][slot] = t;
-    }
-}
-#define GDN_TRACE_CL(c, slot, leader) trace_cluster((c), (slot), (leader))
 #else
 #define GDN_TRACE_AT(c, slot, leader) ((void)0)
-#define GDN_TRACE_CL(c, slot, leader) ((void)0)
 #endif
 
 

@@ -121,14 +121,14 @@ def test_prefill_kernel_selection(lib):
             assert lib.gdn_get_prefill_kernel() == code
             assert binding.get_prefill_kernel() == name
         assert binding.get_prefill_kernel() == "auto"
-    assert lib.gdn_set_prefill_kernel(4) == binding.GDN_ERR_INVALID_ARG
+    assert lib.gdn_set_prefill_kernel(3) == binding.GDN_ERR_INVALID_ARG
     assert lib.gdn_set_prefill_kernel(-1) == binding.GDN_ERR_INVALID_ARG
     assert binding.get_prefill_kernel() == "auto"
     with pytest.raises(binding.GdnError, match="unknown prefill kernel"):
         binding.set_prefill_kernel("wgmma")
     # the tensor-core kernels take bf16 only: fp32 with a forced TC kernel is refused
     # on the host, before any launch
-    for name in ("tc", "tc_cluster"):
+    for name in ("tc",):
         with binding.prefill_kernel(name):
             assert chunk(lib, dtype=0) == binding.GDN_ERR_UNSUPPORTED
             assert chunk(lib, dtype=0, T=0) == binding.GDN_OK   # nothing to launch
@@ -140,7 +140,7 @@ def test_prefill_kernel_for_without_device_work(lib):
     assert binding.prefill_kernel_for(1, 48, torch.float32) == "simt"
     with binding.prefill_kernel("simt"):
         assert binding.prefill_kernel_for(4, 48, torch.bfloat16) == "simt"
-    for name in ("tc", "tc_cluster"):
+    for name in ("tc",):
         with binding.prefill_kernel(name):
             with pytest.raises(binding.GdnError, match="no prefill kernel"):
                 binding.prefill_kernel_for(1, 48, torch.float32)

@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import oracle
+from conftest import record_parity
 from linear_attention_recurrence_07_b200 import binding, inputs
 
 pytestmark = pytest.mark.gpu
@@ -33,6 +34,7 @@ def rel_err(got, ref):
 def check(got, ref, tau, what):
     e = rel_err(got, ref)
     print(f"{what}: max rel err {e:.3e} (tau {tau})")
+    record_parity(what, e, tau)
     assert e <= tau, f"{what}: max|err| / max|ref| = {e:.3e} > {tau}"
 
 
@@ -41,8 +43,8 @@ def to_dev(d):
 
 
 # Prefill kernels a bf16 input can run on; fp32 inputs always take "simt".
-BF16_KERNELS = ["tc", "tc_cluster", "simt"]
-TC_KERNELS = ["tc", "tc_cluster"]
+BF16_KERNELS = ["tc", "simt"]
+TC_KERNELS = ["tc"]
 
 
 def kernels_for(dtype):
@@ -100,7 +102,7 @@ def test_prefill_one_v_head_per_qk_head(dtype):
 @pytest.mark.parametrize("kernel", TC_KERNELS)
 def test_prefill_tc_kernels_beyond_one_wave(kernel):
     """More (sequence, V head) pairs than the GPU holds at once (B=7, Hv=48: 336
-    CTAs, 1008 in clusters): later waves reuse SMs and TMEM of finished ones."""
+    CTAs): later waves reuse SMs and TMEM of finished ones."""
     d = to_dev(inputs.prefill_inputs(7, 130, 16, 48, dtype=torch.bfloat16, s0_std=0.1, seed=11))
     o, S = run_chunk(d, kernel=kernel)
     o_a, S_a = run_chunk(d, kernel="simt")
@@ -116,14 +118,17 @@ def test_prefill_tc_kernels_beyond_one_wave(kernel):
 
 @pytest.mark.parametrize("B,T,Hqk,Hv,seed", [(1, 385, 2, 6, 21), (2, 4096, 16, 48, 22)])
 def test_prefill_tc_kernels_agree(B, T, Hqk, Hv, seed):
-    """The two tensor-core kernels round the decay factors into their bf16 operands
-    at different points: the one-CTA kernel rounds Q~ = diag(gamma) Q and
-    U^T diag(g), the cluster kernel scales the fp32 product gamma_r (S^T q_r) and
-    rounds K~ = diag(g) K.  Each of those roundings is one bf16 ulp (2^-8
-    relative), so the two agree to a few ulp of the largest value."""
+    """The one-CTA and the pipelined tensor-core kernels round the decay factors
+    into their bf16 operands at different points: the one-CTA kernel rounds
+    U^T diag(g) for the state update, the pipelined one rounds K~ = diag(g) K.
+    Each of those roundings is one bf16 ulp (2^-8 relative), so the two agree to
+    a few ulp of the largest value."""
     d = to_dev(inputs.prefill_inputs(B, T, Hqk, Hv, dtype=torch.bfloat16, s0_std=0.3, seed=seed))
     o1, S1 = run_chunk(d, kernel="tc")
-    o2, S2 = run_chunk(d, kernel="tc_cluster")
+    o2 = torch.empty_like(o1)
+    S2 = torch.empty_like(S1)
+    binding.gdn_chunk_fwd_pipelined(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o2, S2)
+    torch.cuda.synchronize()
     err_s = (S1 - S2).abs().max().item()
     assert err_s <= 2 ** -6 * S2.abs().max().item(), err_s
     err = (o1.float() - o2.float()).abs().max().item()
@@ -174,7 +179,12 @@ def test_prefill_batched_workload_sampled():
     first and last sequence on the first and last QK group (all their tokens)."""
     w = inputs.PREFILL_BATCH8_8K
     d = inputs.workload_inputs(w, device=DEV)
-    outs = {kernel: run_chunk(d, kernel=kernel) for kernel in ["auto", "tc_cluster"]}
+    outs = {kernel: run_chunk(d, kernel=kernel) for kernel in ["auto"]}
+    o = torch.empty_like(d["v"])
+    S = torch.empty_like(d["S0"])
+    binding.gdn_chunk_fwd_pipelined(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S)
+    torch.cuda.synchronize()
+    outs["pipelined"] = (o, S)
     for b, (h0, h1) in [(0, (0, 3)), (7, (45, 48)), (3, (21, 24))]:
         o_ref, S_ref = oracle_ref(_sub_problem(d, b, h0, h1, w.Hv, w.Hqk))
         for kernel, (o, S) in outs.items():
@@ -191,6 +201,11 @@ def test_prefill_long_context_workload_sampled():
     d = inputs.workload_inputs(w, device=DEV)
     outs = {kernel: run_chunk(d, kernel=kernel) for kernel in TC_KERNELS}
     outs["split"] = run_split(d)
+    o = torch.empty_like(d["v"])
+    S = torch.empty((w.B, w.Hv, w.dk, w.dv), device=DEV)
+    binding.gdn_chunk_fwd_pipelined(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o, S)
+    torch.cuda.synchronize()
+    outs["pipelined"] = (o, S)
     for h in (0, 47):
         o_ref, S_ref = oracle_ref(_sub_problem(d, 0, h, h + 1, w.Hv, w.Hqk))
         for kernel, (o, S) in outs.items():
@@ -220,9 +235,8 @@ def test_prefill_in_place_state():
     assert torch.equal(S, S_ref)
 
 
-@pytest.mark.parametrize("dtype,kernel", [(torch.bfloat16, "tc"), (torch.bfloat16, "tc_cluster"),
-                                          (torch.float32, "simt")],
-                         ids=["bf16-tc", "bf16-tc_cluster", "fp32-simt"])
+@pytest.mark.parametrize("dtype,kernel", [(torch.bfloat16, "tc"), (torch.float32, "simt")],
+                         ids=["bf16-tc", "fp32-simt"])
 def test_prefill_split_invariance(dtype, kernel):
     """T1 tokens, then T2 tokens from the saved state, equals one call over T1+T2."""
     d = to_dev(inputs.prefill_inputs(2, 300, 2, 6, dtype=dtype, s0_std=0.2, seed=5))

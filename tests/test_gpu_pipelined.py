@@ -8,6 +8,7 @@ import pytest
 import torch
 
 import oracle
+from conftest import record_parity
 from linear_attention_recurrence_07_b200 import binding, inputs
 
 pytestmark = pytest.mark.gpu
@@ -25,6 +26,7 @@ def rel_err(got, ref):
 def check(got, ref, tau, what):
     e = rel_err(got, ref)
     print(f"{what}: max rel err {e:.3e} (tau {tau})")
+    record_parity(what, e, tau)
     assert e <= tau, f"{what}: max|err| / max|ref| = {e:.3e} > {tau}"
 
 
@@ -91,8 +93,9 @@ def test_pipelined_strong_and_no_decay():
 
 def test_pipelined_model_dims_workload():
     """B=1, T=4096, 16/48 heads (the bench workload): every output against the
-    oracle, and against the one-CTA tensor-core kernel (same products, same
-    precisions)."""
+    oracle, and against the one-CTA tensor-core kernel (the same products, rounded
+    to bf16 at slightly different points, e.g. gamma applied to the fp32 S-part of
+    O here and to the bf16 Q operand there, so they agree to a few bf16 ulp)."""
     w = inputs.PREFILL_4K
     d = inputs.workload_inputs(w, device=DEV)
     o, S = run_pipe(d)
