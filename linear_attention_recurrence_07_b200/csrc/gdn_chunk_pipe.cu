@@ -65,23 +65,36 @@ __device__ __forceinline__ void ptrace(int n, int slot, bool on) {
         g_pclock[n][slot] = clock64();
     }
 }
+#ifdef GDN_TRACE_CLKONLY
+#define PTRACE(n, slot, on) ((void)0)
+#else
 #define PTRACE(n, slot, on) ptrace((n), (slot), (on))
+#endif
 // whole grid: each CTA's start and end, each chain CTA's conversion start per chunk
 constexpr int kGridCTAs = 160, kGridChunks = 64;
 __device__ unsigned long long g_pcta[kGridCTAs][4];             // start, end, smid, SM clocks start..end
 // per chain CTA and chunk: conversion start, ring flag seen, slot landed, prep release,
-// S^T bf16 ready, U^T done (seen), U^T bf16 ready, O epilogue done
-__device__ unsigned long long g_pchain[kGridCTAs][kGridChunks][8];
+// S^T bf16 ready, U^T done (seen), U^T bf16 ready, O epilogue done, U~ issued, UG
+// started, V load issued, V landed (seen by the U~ issuer), K/Q load issued
+__device__ unsigned long long g_pchain[kGridCTAs][kGridChunks][16];
 __device__ __forceinline__ unsigned long long gtimer() {
     unsigned long long t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
     return t;
 }
 __device__ long long g_pclk0[kGridCTAs];
+// clock64 stamps of the chain's MMA issuer: UG start / issued / done, SG start / issued /
+// done (the done stamps only in builds that spin on the completion, GDN_TRACE_MMA)
+__device__ long long g_pmclk[kGridCTAs][kGridChunks][16];
+#define PMCLK(x, n, k) do { if ((x) < kGridCTAs && (n) < kGridChunks) g_pmclk[(x)][(n)][(k)] = clock64(); } while (0)
 #define PCTA(slot) do { if (threadIdx.x == 0 && blockIdx.x < kGridCTAs) { g_pcta[blockIdx.x][(slot)] = gtimer(); \
     unsigned sid; asm volatile("mov.u32 %0, %%smid;" : "=r"(sid)); g_pcta[blockIdx.x][2] = sid; \
     if ((slot) == 0) g_pclk0[blockIdx.x] = clock64(); else g_pcta[blockIdx.x][3] = clock64() - g_pclk0[blockIdx.x]; } } while (0)
+#ifdef GDN_TRACE_CLKONLY
+#define PCHAIN(x, n, k, on) ((void)0)
+#else
 #define PCHAIN(x, n, k, on) do { if ((on) && (x) < kGridCTAs && (n) < kGridChunks) g_pchain[(x)][(n)][(k)] = gtimer(); } while (0)
+#endif
 // clock64 stamps inside the MMA issuer's groups (chain CTA 0, chunks 8..15)
 __device__ long long g_pmma[8][24];
 #define PMMA(n, slot, on) do { if ((on) && (n) >= 8 && (n) < 16) g_pmma[(n) - 8][(slot)] = clock64(); } while (0)
@@ -90,15 +103,17 @@ __device__ long long g_pmma[8][24];
 #define PMMA(n, slot, on) ((void)0)
 #define PCTA(slot) ((void)0)
 #define PCHAIN(x, n, k, on) ((void)0)
+#define PMCLK(x, n, k) ((void)0)
 #endif
 
 // ---------------------------------------------------------------- ring slot
 constexpr uint32_t RS_W = 0;                          // W [d][r] bf16, MN-major B operand (16 KB)
 constexpr uint32_t RS_BU = 2 * TILE, RS_P = 3 * TILE; // T diag(beta), masked decay P (8 KB each)
-constexpr uint32_t RS_GATE = 4 * TILE;                // gamma[64], g[64] fp32
-constexpr uint32_t RS_TILES = 4 * TILE;               // operand tiles of a slot (loaded as one copy)
+constexpr uint32_t RS_QT = 4 * TILE;                  // diag(gamma) Q [r][d] bf16, two d-halves (16 KB)
+constexpr uint32_t RS_GATE = 6 * TILE;                // gamma[64], g[64] fp32
+constexpr uint32_t RS_TILES = 6 * TILE;               // operand tiles of a slot (loaded as one copy)
 constexpr uint32_t RS_GATE_BYTES = 512;               // the gate vectors (a second copy)
-constexpr uint32_t RS_BYTES = 33 * 1024;              // slot stride in the ring (1024-multiple)
+constexpr uint32_t RS_BYTES = 49 * 1024;              // slot stride in the ring (1024-multiple)
 constexpr int kRing = 8;                              // slots per chain CTA
 constexpr int kFlagWords = 32;                        // one 128-byte line per chain CTA's flags
 
@@ -109,34 +124,37 @@ constexpr uint32_t COL_U = 256;    // U^T fp32, two buffers; then U^T bf16 in pl
 constexpr uint32_t COL_O = 384;    // O^T, two buffers
 constexpr uint32_t CH_TMEM_COLS = 512;
 
-constexpr int NKQ = 3;                                // K/Q stages, chunk n uses n % NKQ
+constexpr int NKQ = 3;                                // K stages, chunk n uses n % NKQ
 constexpr int NRB = 3;                                // ring buffers, chunk n uses n % NRB
-constexpr uint32_t KQ_STAGE = 4 * TILE;               // [K d0-63][Q d0-63][K d64-127][Q d64-127]
+constexpr uint32_t KQ_STAGE = 4 * TILE;               // prep: [K d0-63][Q d0-63][K d64-127][Q d64-127]
+constexpr uint32_t K_STAGE = 2 * TILE;                // chain: [K d0-63][K d64-127]
 constexpr uint32_t OFF_KQ = 0;
-constexpr uint32_t OFF_V = OFF_KQ + NKQ * KQ_STAGE;    // 2 x [V j0-63][V j64-127]
+constexpr uint32_t OFF_V = OFF_KQ + NKQ * K_STAGE;     // 2 x [V j0-63][V j64-127]
 constexpr uint32_t OFF_RB = OFF_V + 4 * TILE;          // NRB ring buffers: operand tiles (32 KB each)
 constexpr uint32_t OFF_RG = OFF_RB + NRB * RS_TILES;   // NRB ring buffers: gate vectors (512 B each)
 constexpr uint32_t OFF_CBAR = OFF_RG + NRB * RS_GATE_BYTES;
 constexpr uint32_t CH_NBAR = 38;
+// named barriers of the chain CTA: the state chain (conversion warpgroups + the
+// chain issuer warp), the conversion warpgroups alone, the helper warpgroup
+constexpr int kChainBar = 3, kChainThreads = 288, kConvBar = 5;
 constexpr uint32_t OFF_CMISC = OFF_CBAR + CH_NBAR * 8;   // TMEM base, local abort flag
 constexpr uint32_t CH_SMEM_USED = OFF_CMISC + 16;
 static_assert(OFF_RB % 1024 == 0 && RS_TILES % 1024 == 0 && RS_BYTES % 1024 == 0,
               "swizzled tiles need 1024-byte alignment");
 
-// Chain CTA warps: 0 input TMA, 1 and 3 MMA issuers, 2 ring loader, 4-7 and 8-11
-// the two conversion warpgroups (state columns 0-63 / 64-127; U columns 0-31 /
-// 32-63), 12-15 the helper warpgroup (gamma scaling of the S-part of O, O epilogue).
+// Chain CTA warps: 0 input TMA, 2 ring loader, 3 the MMA issuer off the chain,
+// 4-7 and 8-11 the two conversion warpgroups (state columns 0-63 / 64-127; U
+// columns 0-31 / 32-63), one thread of which issues the chain's MMAs, 12-15 the
+// helper warpgroup (gamma scaling of the S-part of O, O epilogue); warp 1 idles.
 enum : int {
-    C_KQ_FULL = 0,    // x3 (K/Q stage landed)
-    C_KQ_EMPTY = 3,   // x3 (S and O MMAs of the chunk done: one commit of each issuer)
+    C_KQ_FULL = 0,    // x3 (K stage landed)
+    C_KQ_EMPTY = 3,   // x3 (S and O MMAs of the chunk done: one commit of each issuer; frees
+                      //     the K stage and, for U~ two chunks on, the U buffer)
     C_V_FULL = 6,     // x2
     C_V_EMPTY = 8,    // x2 (U~ MMAs done)
     C_RB_FULL = 10,   // x3 (ring slot landed)
-    C_RB_EMPTY = 13,  // x3 (a commit of each issuer + 12 warps)
-    C_S_READY = 16,   // x2 (per S^T bf16 buffer): both conversion warpgroups (8 warps)
-    C_XS_READY = 18,  // x2 helper: S-part of O^T scaled by gamma (4 warps)
+    C_RB_EMPTY = 13,  // x3 (a commit of each issuer + the 8 conversion warps)
     C_U_FULL = 20,    // U^T done
-    C_U_READY = 21,   // x2 conversion warpgroups: U^T bf16 written (8 warps)
     C_S_FULL = 23,    // state update done
     C_X_FULL = 24,    // x2 (per S^T bf16 buffer): S-part of O^T done
     C_O_FULL = 26,    // x2 O^T complete
@@ -148,10 +166,9 @@ enum : int {
 };
 // Arrival counts: a tcgen05.commit counts one, a warp (warp_arrive) one.
 __host__ __device__ constexpr uint32_t chain_bar_count(int i) {
-    return (i >= C_RB_EMPTY && i < C_RB_EMPTY + NRB) ? 14u
+    return (i >= C_RB_EMPTY && i < C_RB_EMPTY + NRB) ? 10u
          : ((i >= C_KQ_EMPTY && i < C_KQ_EMPTY + NKQ) || i == C_DRAIN) ? 2u
-         : (i == C_S_READY || i == C_S_READY + 1 || i == C_U_READY || i == C_U_READY + 1) ? 8u
-         : (i == C_XS_READY || i == C_XS_READY + 1 || i == C_O_FREE || i == C_O_FREE + 1) ? 4u : 1u;
+         : (i == C_O_FREE || i == C_O_FREE + 1) ? 4u : 1u;
 }
 static_assert(C_O_GO + 1 < (int)CH_NBAR, "barrier count");
 
@@ -247,8 +264,12 @@ struct PCtl {
         return false;
     }
     __device__ __forceinline__ long long poll_every() const { return limit < 4 * kGlobalPoll ? limit / 4 + 1 : kGlobalPoll; }
+    // The first try inline; the bounded loop out of line (the waiting code of the
+    // many call sites then costs the hot loops no instruction-cache room).
     __device__ __forceinline__ bool wait(int i, uint32_t parity) const {
-        if (mbar_try_wait(&bar[i], parity)) return true;
+        return mbar_try_wait(&bar[i], parity) || wait_loop(i, parity);
+    }
+    __device__ __noinline__ bool wait_loop(int i, uint32_t parity) const {
         const long long t0 = clock64();
         long long next_poll = t0 + poll_every();
         const uint32_t hint = limit < (1ll << 24) ? 200u : 20000u;
@@ -263,10 +284,21 @@ struct PCtl {
             if (now - t0 > limit) return fail();
         }
     }
+    // Polls a few times before falling back to wait(): for waits that usually end
+    // within a few hundred clocks, where waking from a suspended try_wait is slower.
+    __device__ __forceinline__ bool wait_fast(int i, uint32_t parity) const {
+        return mbar_test(&bar[i], parity) || wait_fast_loop(i, parity);
+    }
+    __device__ __noinline__ bool wait_fast_loop(int i, uint32_t parity) const {
+#pragma unroll 1
+        for (int k = 0; k < 64; ++k)
+            if (mbar_test(&bar[i], parity)) return true;
+        return wait(i, parity);
+    }
     // Waits until *p >= target (one thread; acquire once seen).  The pause between
     // polls doubles from 32 ns up to max_sleep ns, so that many waiters do not load
     // the memory system with polls while they have long to wait.
-    __device__ __forceinline__ bool wait_flag(const unsigned *p, unsigned target, unsigned max_sleep) const {
+    __device__ __noinline__ bool wait_flag(const unsigned *p, unsigned target, unsigned max_sleep) const {
         if (ld_relaxed(p) >= target) { fence_acquire_gpu(); return true; }
         const long long t0 = clock64();
         long long next_poll = t0 + poll_every();
@@ -336,6 +368,45 @@ __device__ __forceinline__ int chain_units(const PipeParams &p, int x) {
     return heads * p.nchunks;
 }
 
+// Rare steps of the state chain, out of line so that the per-chunk loop stays small:
+// S^T[j][d] = S0[d][j] of a new head (zeros without S0), and the final state
+// S_final[d][j] = S^T[j][d] of a finished one, for the thread's value column j and
+// its warpgroup's 64 key dims d0 ...
+__device__ __noinline__ void chain_load_s0(const float *src, uint32_t t_row, int d0, int j) {
+#pragma unroll 1
+    for (int c0 = d0; c0 < d0 + 64; c0 += 32) {
+        float v[32];
+#pragma unroll
+        for (int xx = 0; xx < 32; ++xx) v[xx] = src ? src[(size_t)(c0 + xx) * kHeadDim + j] : 0.f;
+        tmem_st32(t_row + COL_S + c0, v);
+    }
+    tmem_wait_st();
+}
+__device__ __noinline__ void chain_store_final(float *dst, uint32_t t_row, int d0, int j) {
+#pragma unroll 1
+    for (int c0 = d0; c0 < d0 + 64; c0 += 32) {
+        float w[32];
+        tmem_ld32(t_row + COL_S + c0, w);
+        tmem_wait_ld();
+#pragma unroll
+        for (int xx = 0; xx < 32; ++xx) dst[(size_t)(c0 + xx) * kHeadDim + j] = w[xx];
+    }
+}
+__device__ __noinline__ Unit unit_of_ool(const PipeParams &p, int x, int n) { return unit_of(p, x, n); }
+// O rows of a chunk cut by the end of its sequence (rows < C of them exist), from the
+// warp's TMEM lanes at t_col.
+__device__ __noinline__ void store_o_rows(__nv_bfloat16 *dst, uint32_t t_col, int rows, size_t row_stride) {
+#pragma unroll 1
+    for (int r0 = 0; r0 < C; r0 += 32) {
+        float ov[32];
+        tmem_ld32(t_col + r0, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int xx = 0; xx < 32; ++xx)
+            if (r0 + xx < rows) dst[(size_t)(r0 + xx) * row_stride] = __float2bfloat16_rn(ov[xx]);
+    }
+}
+
 // ============================================================================ chain
 __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorMap *tm_q,
                                         const CUtensorMap *tm_v, const PipeParams &p, unsigned char *sm)
@@ -378,13 +449,12 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 if (nkq < N && (nkq < NKQ || mbar_test(&bar[C_KQ_EMPTY + nkq % NKQ], ((nkq / NKQ) - 1) & 1))) {
                     const Unit u = unit_of(p, x, nkq);
                     const int s = nkq % NKQ, t0 = u.c * C;
-                    unsigned char *st = sm + OFF_KQ + s * KQ_STAGE;
-                    mbar_arrive_expect_tx(&bar[C_KQ_FULL + s], KQ_STAGE);
-                    tma_load_4d(st + 0 * TILE, tm_k, &bar[C_KQ_FULL + s], 0, u.hq, t0, u.b);
-                    tma_load_4d(st + 1 * TILE, tm_q, &bar[C_KQ_FULL + s], 0, u.hq, t0, u.b);
-                    tma_load_4d(st + 2 * TILE, tm_k, &bar[C_KQ_FULL + s], 64, u.hq, t0, u.b);
-                    tma_load_4d(st + 3 * TILE, tm_q, &bar[C_KQ_FULL + s], 64, u.hq, t0, u.b);
+                    unsigned char *st = sm + OFF_KQ + s * K_STAGE;
+                    mbar_arrive_expect_tx(&bar[C_KQ_FULL + s], K_STAGE);
+                    tma_load_4d(st, tm_k, &bar[C_KQ_FULL + s], 0, u.hq, t0, u.b);
+                    tma_load_4d(st + TILE, tm_k, &bar[C_KQ_FULL + s], 64, u.hq, t0, u.b);
                     PTRACE(nkq, 11, x == 0);
+                    PCHAIN(x, nkq, 12, true);
                     ++nkq;
                     issued = true;
                 }
@@ -395,6 +465,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     mbar_arrive_expect_tx(&bar[C_V_FULL + s], 2 * TILE);
                     tma_load_4d(vb, tm_v, &bar[C_V_FULL + s], 0, u.h, t0, u.b);
                     tma_load_4d(vb + TILE, tm_v, &bar[C_V_FULL + s], 64, u.h, t0, u.b);
+                    PCHAIN(x, nv, 10, true);
                     ++nv;
                     issued = true;
                 }
@@ -416,60 +487,25 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     mbar_wait(&bar[C_V_FULL + (m & 1)], (m >> 1) & 1, 1ll << 28);
             }
         }
-    } else if (warp == 1 || warp == 3) {
-        // ============================================================ MMA issuers
-        // Two threads issue, so that issuing one group never waits behind another:
-        //   warp 1 (critical chain)  UG(n)   U^T += S^T (-W)^T   8 MMAs
-        //                            SG(n)   S^T += (U diag(g))^T K  4 MMAs
-        //   warp 3 (the rest)        XG(n)   O^T  = S^T Q^T      8 MMAs  after UG(n) is issued
-        //                            OG(n)   O^T += U^T P^T      4 MMAs  after SG(n) is issued
-        //                            UT(n+2) U~^T = V^T Bu^T     4 MMAs  once S and O MMAs of n are done
+    } else if (warp == 3) {
+        // ============================================================ MMA issuer (off the chain)
+        //   XG(n)   O^T  = S^T Q^T      8 MMAs  after UG(n) is issued
+        //   OG(n)   O^T += U^T P^T      4 MMAs  after SG(n) is issued
+        //   UT(n+2) U~^T = V^T Bu^T     4 MMAs  once the S and O MMAs of n are done
         // U~ of a chunk is so computed two chunks ahead of its UG, and XG / OG queue
         // behind UG / SG in the tensor pipe.  Every barrier waited on here is one of a
         // pair (or a ring), so that no wait can miss its phase: the next phase of each
-        // depends on the group the wait gates.  Both threads wait by suspending
-        // (try_wait), which leaves the shared-memory pipe to the other warps.
-        if (lane == 0 && warp == 1) {
-            bool ok = true;
-            for (int n = 0; n < N && ok; ++n) {
-                const int s = n & 1;
-                const uint32_t st = sbase + OFF_KQ + (n % NKQ) * KQ_STAGE;
-                const uint32_t rb = sbase + OFF_RB + (n % NRB) * RS_TILES;
-                // UG(n): S^T bf16 of n, U~^T of n done (its ring slot is then loaded too)
-                if (!(ok = ctl.wait(C_UT_FULL + s, (n >> 1) & 1))) break;
-                if (!(ok = ctl.wait(C_S_READY + s, (n >> 1) & 1))) break;
-                PTRACE(n, 13, x == 0);
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_bf16_ts(tmem + COL_U + s * 64, tmem + COL_SB + s * 64 + k * 8,
-                                smem_desc_sw128(rb + RS_W + k * 2048, 2 * TILE, 1024), ID_U, true);
-                mma_commit(&bar[C_U_FULL]);
-                mbar_arrive(&bar[C_X_GO + s]);
-                PTRACE(n, 3, x == 0);
-                // SG(n): (U diag(g))^T bf16 of n
-                if (!(ok = ctl.wait(C_U_READY + s, (n >> 1) & 1))) break;
-                PTRACE(n, 24, x == 0);
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16_ts(tmem + COL_S, tmem + COL_U + s * 64 + 32 + k * 8,
-                                smem_desc_sw128(st + k * 2048, 2 * TILE, 1024), ID_S, true);
-                mma_commit(&bar[C_S_FULL]);
-                mma_commit(&bar[C_KQ_EMPTY + n % NKQ]);
-                mma_commit(&bar[C_RB_EMPTY + n % NRB]);
-                mbar_arrive(&bar[C_O_GO + s]);
-                PTRACE(n, 4, x == 0);
-            }
-            mma_commit(&bar[C_DRAIN]);
-        } else if (lane == 0 && warp == 3) {
+        // depends on the group the wait gates.
+        if (lane == 0) {
             bool ok = true;
             auto issue_ut = [&](int n) -> bool {       // U~^T of chunk n into U buffer n & 1
                 const int s = n & 1;
-                if (!ctl.wait(C_V_FULL + s, (n >> 1) & 1) || !ctl.wait(C_RB_FULL + n % NRB, (n / NRB) & 1))
-                    return false;
+                if (!ctl.wait(C_V_FULL + s, (n >> 1) & 1)) return false;
+                PCHAIN(x, n, 11, true);
+                if (!ctl.wait(C_RB_FULL + n % NRB, (n / NRB) & 1)) return false;
                 // the buffer's last readers, SG(n-2) and OG(n-2), are done
                 if (n >= 2 && !ctl.wait(C_KQ_EMPTY + (n - 2) % NKQ, ((n - 2) / NKQ) & 1)) return false;
+                PCHAIN(x, n, 8, true);
                 tc_fence_after();
                 const uint32_t vb = sbase + OFF_V + s * 2 * TILE;
                 const uint32_t rb = sbase + OFF_RB + (n % NRB) * RS_TILES;
@@ -486,26 +522,22 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             if (N > 1 && ok) ok = issue_ut(1);
             for (int n = 0; n < N && ok; ++n) {
                 const int s = n & 1;
-                const uint32_t st = sbase + OFF_KQ + (n % NKQ) * KQ_STAGE;
                 const uint32_t rb = sbase + OFF_RB + (n % NRB) * RS_TILES;
-                // XG(n): after UG(n) is issued; S^T bf16 of n, O buffer read out
+                // XG(n): after UG(n) is issued (S^T bf16 of n written); O buffer read out
                 if (!(ok = ctl.wait(C_X_GO + s, (n >> 1) & 1))) break;
-                if (!(ok = ctl.wait(C_S_READY + s, (n >> 1) & 1))) break;
                 if (n >= 2 && !(ok = ctl.wait(C_O_FREE + s, ((n >> 1) - 1) & 1))) break;
                 PTRACE(n, 14, x == 0);
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    const uint32_t koff = (k >> 2) * 2 * TILE + (k & 3) * 32;
+                    const uint32_t koff = (k >> 2) * TILE + (k & 3) * 32;
                     mma_bf16_ts(tmem + COL_O + s * 64, tmem + COL_SB + s * 64 + k * 8,
-                                smem_desc_sw128(st + TILE + koff, 16, 1024), ID_O, k > 0);
+                                smem_desc_sw128(rb + RS_QT + koff, 16, 1024), ID_O, k > 0);
                 }
                 mma_commit(&bar[C_X_FULL + s]);
                 PTRACE(n, 15, x == 0);
-                // OG(n): after SG(n) is issued; U^T bf16 of n, S-part scaled by gamma
+                // OG(n): after SG(n) is issued (U^T bf16 of n written)
                 if (!(ok = ctl.wait(C_O_GO + s, (n >> 1) & 1))) break;
-                if (!(ok = ctl.wait(C_U_READY + s, (n >> 1) & 1))) break;
-                if (!(ok = ctl.wait(C_XS_READY + s, (n >> 1) & 1))) break;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
@@ -558,74 +590,158 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             for (int m = issued - 1; m >= 0 && m >= issued - NRB; --m)
                 mbar_wait(&bar[C_RB_FULL + m % NRB], (m / NRB) & 1, 1ll << 28);
         }
+    } else if (warp == 1) {
+        // ============================================================ chain MMA issuer
+        // Meets the conversion warpgroups at their named barrier (kChainBar, 288 threads:
+        // 8 conversion warps and this one) and issues, right after
+        //   #2 (S^T bf16 of n written):           UG(n)  U^T += S^T (-W)^T       8 MMAs
+        //   #4 (U^T bf16 copies, decayed S^T):     SG(n)  S^T += (U diag(g))^T K  4 MMAs
+        // The commits that release the K stage and the ring slot of n are issued after
+        // UG(n+1) (they then also cover it), off the hand-off to the conversion.
+        bool ok = true;
+        for (int n = 0; n < N && ok; ++n) {
+            const int s = n & 1, nk = n % NKQ, nr = n % NRB;
+            const uint32_t st = sbase + OFF_KQ + nk * K_STAGE;
+            const uint32_t rb = sbase + OFF_RB + nr * RS_TILES;
+            bool ut_ready = false;
+            if (lane == 0) ut_ready = mbar_test(&bar[C_UT_FULL + s], (n >> 1) & 1);
+            ok = named_and(kChainBar, kChainThreads, true);           // #1
+            if (!ok) break;
+            named_sync(kChainBar, kChainThreads);                     // #2
+            if (lane == 0) {   // UG(n): its U~^T is done too
+                tc_fence_after();
+                if (ut_ready || ctl.wait(C_UT_FULL + s, (n >> 1) & 1)) {
+                    PMCLK(x, n, 0);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16_ts(tmem + COL_U + s * 64, tmem + COL_SB + s * 64 + k * 8,
+                                    smem_desc_sw128(rb + RS_W + k * 2048, 2 * TILE, 1024), ID_U, true);
+                    PMCLK(x, n, 1);
+                    mma_commit(&bar[C_U_FULL]);
+#ifdef GDN_TRACE_MMA
+                    for (int it = 0; it < (1 << 22) && !mbar_test(&bar[C_U_FULL], n & 1); ++it) {}
+                    PMCLK(x, n, 2);
+#endif
+                    tc_fence_before();
+                    mbar_arrive(&bar[C_X_GO + s]);
+                    if (n > 0) {
+                        mma_commit(&bar[C_KQ_EMPTY + (n - 1) % NKQ]);
+                        mma_commit(&bar[C_RB_EMPTY + (n - 1) % NRB]);
+                    }
+                }
+                PTRACE(n, 3, x == 0);
+            }
+            __syncwarp();
+            ok = named_and(kChainBar, kChainThreads, true);           // #3
+            if (!ok) break;
+            named_sync(kChainBar, kChainThreads);                     // #4
+            if (lane == 0) {   // SG(n)
+                tc_fence_after();
+                PMCLK(x, n, 3);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ts(tmem + COL_S, tmem + COL_U + s * 64 + 32 + k * 8,
+                                smem_desc_sw128(st + k * 2048, TILE, 1024), ID_S, true);
+                PMCLK(x, n, 4);
+                mma_commit(&bar[C_S_FULL]);
+#ifdef GDN_TRACE_MMA
+                for (int it = 0; it < (1 << 22) && !mbar_test(&bar[C_S_FULL], n & 1); ++it) {}
+                PMCLK(x, n, 5);
+#endif
+                tc_fence_before();
+                mbar_arrive(&bar[C_O_GO + s]);
+                PTRACE(n, 4, x == 0);
+            }
+            __syncwarp();
+        }
+        if (lane == 0) {
+            mma_commit(&bar[C_DRAIN]);
+            mbar_wait(&bar[C_DRAIN], 0, 1ll << 30);
+        }
     } else if (warp >= 4 && warp < 12) {
-        // ============================================================ conversion warpgroups
-        // Warpgroup h (0: warps 4-7, 1: warps 8-11) owns state columns (key dims)
-        // 64h .. 64h+63 and U^T columns (chunk rows) 32h .. 32h+31.
+        // ============================================================ state chain
+        // Two conversion warpgroups (h = 0: warps 4-7, 1: warps 8-11) own state
+        // columns (key dims) 64h .. 64h+63 and U^T columns (chunk rows) 32h .. 32h+31.
+        // Per chunk, with the issuer warp at the named barriers #1-#4:
+        //   #1 the chunk's inputs are in: S^T -> bf16 copy;  #2 (UG issued) the decay
+        //   S^T <- gamma_{C-1} S^T while UG runs (UG reads the bf16 copy);  #3 U^T done:
+        //   U^T -> two bf16 copies;  #4 (SG issued).
         const int h2 = (warp - 4) >> 2;
         const int q4 = warp & 3;
         const int j = q4 * 32 + lane;                 // TMEM lane = value column j
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
-        const int nb = 1 + h2;                        // this warpgroup's named barrier
+        const bool tr0 = warp == 4 && lane == 0;      // trace stamps
         const size_t hstate = (size_t)kHeadDim * kHeadDim;
         const int d0 = 64 * h2;
         bool ok = true;
+        Unit u = unit_of(p, x, 0);
         for (int n = 0; n < N && ok; ++n) {
             const int s = n & 1;
-            const Unit u = unit_of(p, x, n);
-            const float *gv = reinterpret_cast<const float *>(sm + OFF_RG + (n % NRB) * RS_GATE_BYTES);
-            // S^T bf16 buffer s was last read by UG(n-2) (U_FULL, waited then) and XG(n-2);
-            // the previous chunk's state update is done (for a new head: the previous
-            // head's last one, whose final state was stored below)
-            if (n >= 2) ok = ctl.wait(C_X_FULL + s, ((n >> 1) - 1) & 1);
-            if (n > 0) ok = ok && ctl.wait(C_S_FULL, (n - 1) & 1);
-            ok = ok && ctl.wait(C_RB_FULL + n % NRB, (n / NRB) & 1);
-            ok = named_and(nb, 128, ok);
+            if (n > 0) {                              // the next chunk of this head, or the next head
+                if (u.c + 1 < nck) ++u.c;
+                else u = unit_of_ool(p, x, n);
+            }
+            const int nr = n % NRB;
+            const float *gv = reinterpret_cast<const float *>(sm + OFF_RG + nr * RS_GATE_BYTES);
+            // S^T bf16 buffer s was last read by UG(n-2) and XG(n-2); the previous
+            // chunk's state update is done (for a new head: the previous head's last
+            // one, whose final state was stored below); the ring slot has landed.
+            // One lane per warp waits (the named barrier then orders the others after
+            // it); the three are tested at once first, as they are usually complete.
+            if (lane == 0) {
+                const bool a = n < 2 || mbar_test(&bar[C_X_FULL + s], ((n >> 1) - 1) & 1);
+                const bool b = n == 0 || mbar_test(&bar[C_S_FULL], (n - 1) & 1);
+                const bool c = mbar_test(&bar[C_RB_FULL + nr], (n / NRB) & 1);
+                if (tr0) PMCLK(x, n, 6);
+                if (!(a && b && c))
+                    ok = (a || ctl.wait(C_X_FULL + s, ((n >> 1) - 1) & 1)) &&
+                         (b || ctl.wait_fast(C_S_FULL, (n - 1) & 1)) &&
+                         (c || ctl.wait(C_RB_FULL + nr, (n / NRB) & 1));
+                if (tr0) PMCLK(x, n, 7);
+                if (tr0) PMCLK(x, n, 8);
+            }
+            ok = named_and(kChainBar, kChainThreads, ok);             // #1
             if (!ok) break;
             tc_fence_after();
+            if (tr0) PMCLK(x, n, 9);
             PTRACE(n, 5, x == 0 && j == 0 && h2 == 0);
             PCHAIN(x, n, 0, j == 0 && h2 == 0);
-            if (u.c == 0) {   // a new head: S^T[j][d] = S0[d][j] (zeros without S0)
-                const float *src = p.S0 ? p.S0 + ((size_t)u.b * p.Hv + u.h) * hstate : nullptr;
-#pragma unroll 1
-                for (int c0 = d0; c0 < d0 + 64; c0 += 32) {
-                    float v[32];
-#pragma unroll
-                    for (int xx = 0; xx < 32; ++xx) v[xx] = src ? src[(size_t)(c0 + xx) * kHeadDim + j] : 0.f;
-                    tmem_st32(t_row + COL_S + c0, v);
-                }
-                tmem_wait_st();
-            }
-            // S^T -> packed bf16 A operand (buffer s); S^T <- gamma_{C-1} S^T
+            if (u.c == 0)     // a new head
+                chain_load_s0(p.S0 ? p.S0 + ((size_t)u.b * p.Hv + u.h) * hstate : nullptr, t_row, d0, j);
+            // S^T -> packed bf16 A operand (buffer s)
+            float v[64];
             {
-                const float glast = gv[C - 1];
-                float v[64];
                 uint32_t pk[32];
                 tmem_ld32(t_row + COL_S + d0, v);
                 tmem_ld32(t_row + COL_S + d0 + 32, v + 32);
                 tmem_wait_ld();
+                if (tr0) PMCLK(x, n, 10);
 #pragma unroll
                 for (int xx = 0; xx < 32; ++xx) pk[xx] = pack_bf16x2(v[2 * xx], v[2 * xx + 1]);
                 tmem_st32u(t_row + COL_SB + s * 64 + (d0 >> 1), pk);
+            }
+            tmem_wait_st();
+            if (tr0) PMCLK(x, n, 11);
+            tc_fence_before();
+            named_sync(kChainBar, kChainThreads);                     // #2
+            if (tr0) PMCLK(x, n, 12);
+            PTRACE(n, 6, x == 0 && j == 0 && h2 == 0);
+            PCHAIN(x, n, 4, j == 0 && h2 == 0);
+            {   // S^T <- gamma_{C-1} S^T
+                const float glast = gv[C - 1];
 #pragma unroll
                 for (int xx = 0; xx < 64; ++xx) v[xx] *= glast;
                 tmem_st32(t_row + COL_S + d0, v);
                 tmem_st32(t_row + COL_S + d0 + 32, v + 32);
             }
-            tmem_wait_st();
-            tc_fence_before();
-            warp_arrive(&bar[C_S_READY + s]);
-            PTRACE(n, 6, x == 0 && j == 0 && h2 == 0);
-            PCHAIN(x, n, 4, j == 0 && h2 == 0);
-            PTRACE(n, 27, x == 0 && j == 127 && h2 == 1);
             // U^T (fp32, 64 columns) -> two packed bf16 copies in place: U^T (columns
             // 0-31, for the O MMAs) and (U diag(g))^T (columns 32-63, for the state
             // update, so that K needs no scaling).  Both warpgroups load their half
-            // before either writes (the packed copies overlap the fp32 halves).  The
-            // wait is agreed by both warpgroups together, so that either both reach the
-            // barrier between loads and stores or neither does.
-            ok = named_and(3, 256, ctl.wait(C_U_FULL, n & 1));
+            // before either writes (the packed copies overlap the fp32 halves).
+            if (tr0) PMCLK(x, n, 13);
+            ok = named_and(kChainBar, kChainThreads, lane != 0 || ctl.wait_fast(C_U_FULL, n & 1));   // #3
             if (!ok) break;
+            if (tr0) PMCLK(x, n, 14);
             PTRACE(n, 7, x == 0 && j == 0 && h2 == 0);
             PCHAIN(x, n, 5, j == 0 && h2 == 0);
             tc_fence_after();
@@ -634,7 +750,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 uint32_t pk[16];
                 tmem_ld32(t_row + COL_U + s * 64 + 32 * h2, uu);
                 tmem_wait_ld();
-                named_sync(3, 256);
+                named_sync(kConvBar, 256);
 #pragma unroll
                 for (int xx = 0; xx < 16; ++xx) pk[xx] = pack_bf16x2(uu[2 * xx], uu[2 * xx + 1]);
                 tmem_st16u(t_row + COL_U + s * 64 + 16 * h2, pk);
@@ -644,93 +760,61 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     pk[xx] = pack_bf16x2(uu[2 * xx] * gg[2 * xx], uu[2 * xx + 1] * gg[2 * xx + 1]);
                 tmem_st16u(t_row + COL_U + s * 64 + 32 + 16 * h2, pk);
             }
-            tmem_wait_st();
+            tmem_wait_st();                       // the bf16 copies and the decayed state
+            if (tr0) PMCLK(x, n, 15);
             tc_fence_before();
+            named_sync(kChainBar, kChainThreads);                     // #4
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bar[C_U_READY + s]);
-                mbar_arrive(&bar[C_RB_EMPTY + n % NRB]);   // gamma of n no longer read here
-            }
+            if (lane == 0) mbar_arrive(&bar[C_RB_EMPTY + nr]);   // gates of n no longer read here
             PTRACE(n, 8, x == 0 && j == 0 && h2 == 0);
             PCHAIN(x, n, 6, j == 0 && h2 == 0);
-            PTRACE(n, 28, x == 0 && j == 127 && h2 == 1);
             // last chunk of a head: store its final state once the update is done
             if (u.c == nck - 1 && p.S_final) {
-                ok = named_and(nb, 128, ctl.wait(C_S_FULL, n & 1));
+                ok = named_and(kConvBar, 256, lane != 0 || ctl.wait(C_S_FULL, n & 1));
                 if (!ok) break;
                 tc_fence_after();
-                float *dst = p.S_final + ((size_t)u.b * p.Hv + u.h) * hstate;
-#pragma unroll 1
-                for (int c0 = d0; c0 < d0 + 64; c0 += 32) {
-                    float v[32];
-                    tmem_ld32(t_row + COL_S + c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int xx = 0; xx < 32; ++xx) dst[(size_t)(c0 + xx) * kHeadDim + j] = v[xx];
-                }
+                chain_store_final(p.S_final + ((size_t)u.b * p.Hv + u.h) * hstate, t_row, d0, j);
                 tc_fence_before();
             }
         }
     } else if (warp >= 12) {
         // ============================================================ helper warpgroup
-        // Per chunk: the S-part of O^T (S^T Q^T, from XG) scaled by gamma_r in TMEM, so
-        // that OG adds P U to diag(gamma) Q S; then the O epilogue (TMEM -> registers
-        // -> bf16 stores of the chunk's rows).  Neither step is on the state chain.
+        // The O epilogue of each chunk (TMEM -> registers -> bf16 stores of its rows).
         const int q4 = warp & 3;
         const int j = q4 * 32 + lane;
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
         const size_t row_stride = (size_t)p.Hv * kHeadDim;
         bool ok = true;
+        Unit u = unit_of(p, x, 0);
         for (int n = 0; n < N && ok; ++n) {
             const int s = n & 1;
             const uint32_t col_o = COL_O + s * 64;
-            // ---- O^T[j][r] *= gamma_r (XG of n done; OG of n waits for it)
-            ok = named_and(4, 128, ctl.wait(C_X_FULL + s, (n >> 1) & 1) &&
-                                   ctl.wait(C_RB_FULL + n % NRB, (n / NRB) & 1));
-            if (!ok) break;
-            tc_fence_after();
-            PTRACE(n, 9, x == 0 && j == 0);
-            {
-                const float *gam = reinterpret_cast<const float *>(sm + OFF_RG + (n % NRB) * RS_GATE_BYTES);
-                float ov[64];
-                tmem_ld32(t_row + col_o, ov);
-                tmem_ld32(t_row + col_o + 32, ov + 32);
-                tmem_wait_ld();
-#pragma unroll
-                for (int r = 0; r < C; ++r) ov[r] *= gam[r];
-                tmem_st32(t_row + col_o, ov);
-                tmem_st32(t_row + col_o + 32, ov + 32);
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bar[C_XS_READY + s]);
-                mbar_arrive(&bar[C_RB_EMPTY + n % NRB]);   // gamma of n no longer read here
-            }
             // ---- epilogue of n
-            ok = named_and(4, 128, ctl.wait(C_O_FULL + s, (n >> 1) & 1));
+            ok = named_and(4, 128, lane != 0 || ctl.wait(C_O_FULL + s, (n >> 1) & 1));
             if (!ok) break;
             tc_fence_after();
-            const Unit u = unit_of(p, x, n);
+            if (n > 0) {                              // the next chunk of this head, or the next head
+                if (u.c + 1 < nck) ++u.c;
+                else u = unit_of_ool(p, x, n);
+            }
             const int rows = min(C, p.T - u.c * C);
-            float ov[64];
-            tmem_ld32(t_row + col_o, ov);
-            tmem_ld32(t_row + col_o + 32, ov + 32);
-            tmem_wait_ld();
-            tc_fence_before();
-            warp_arrive(&bar[C_O_FREE + s]);            // the O buffer is free once read out
             // thread j writes o[t][h][j] of the chunk's rows: each warp store covers 32
             // consecutive j (64 contiguous bytes)
             __nv_bfloat16 *dst = p.o + ((size_t)u.b * p.T + (size_t)u.c * C) * row_stride +
                                  (size_t)u.h * kHeadDim + j;
             if (rows == C) {
+                float ov[64];
+                tmem_ld32(t_row + col_o, ov);
+                tmem_ld32(t_row + col_o + 32, ov + 32);
+                tmem_wait_ld();
+                tc_fence_before();
+                warp_arrive(&bar[C_O_FREE + s]);        // the O buffer is free once read out
 #pragma unroll
                 for (int r = 0; r < C; ++r) dst[(size_t)r * row_stride] = __float2bfloat16_rn(ov[r]);
             } else {
-#pragma unroll
-                for (int r = 0; r < C; ++r)
-                    if (r < rows) dst[(size_t)r * row_stride] = __float2bfloat16_rn(ov[r]);
+                store_o_rows(dst, t_row + col_o, rows, row_stride);
+                tc_fence_before();
+                warp_arrive(&bar[C_O_FREE + s]);
             }
             PTRACE(n, 10, x == 0 && j == 0);
             PCHAIN(x, n, 7, j == 0);
@@ -971,6 +1055,12 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
                 if (gate_warp) compute_gates(gv, a0, a1, be0, be1, lane);
                 named_sync(nb, 128);
                 PTRACE(n, 17, tr);
+                {   // ---- Q~ = diag(gamma) Q: thread pt scales row i of d-half `half` of the
+                    //      item's Q tile into the slot, in the tile layout it was loaded in
+                    const int i = pt & 63, half = pt >> 6;
+                    const unsigned char *qt = sm + P_OFF_KQ + s * KQ_STAGE + (2 * half + 1) * TILE;
+                    scale_row_bf16(qt, slot + RS_QT + half * TILE, i, gv[GV_GAM + i]);
+                }
                 // ---- grams -> A rows (fp32, sA) and P rows (bf16, straight into the slot).
                 //      Row r of A is beta_r Gam[r][i] k_r.k_i (i < r), of P Gam[r][i] q_r.k_i
                 //      (i <= r); the decays are running products of alpha along the row from
@@ -1234,6 +1324,10 @@ extern "C" int gdn_pipe_grid_read(unsigned long long *cta, unsigned long long *c
     cudaError_t e = cudaMemcpyFromSymbol(cta, g_pcta, sizeof(g_pcta));
     if (e == cudaSuccess) e = cudaMemcpyFromSymbol(chain, g_pchain, sizeof(g_pchain));
     return (int)e;
+}
+extern "C" int gdn_pipe_mclk_read(long long *host)
+{
+    return (int)cudaMemcpyFromSymbol(host, g_pmclk, sizeof(g_pmclk));
 }
 extern "C" int gdn_pipe_clock_read(long long *host, int n)
 {
