@@ -7,7 +7,7 @@
 A step is one pass of the hot path over one batch of synthetic input: the
 prefill of the model-dims workload (B=1, T=4096, 16 QK heads, 48 V heads, head
 dim 128, bf16 q/k/v, fp32 gates and state, chunk 64) through the library's
-prefill entry point (default gdn_chunk_fwd_split, its workspace allocated
+prefill entry point (default gdn_chunk_fwd_pipelined, its workspace allocated
 once).  The headline ``value`` is prefill tokens/s over all ranks with inputs
 resident in HBM; L2 is flushed (256 MiB write) before every timed step and each
 step is timed with CUDA events on the launching stream.  Measured in the same
@@ -608,9 +608,9 @@ def main():
     ap.add_argument("--batched-steps", type=int, default=10)
     ap.add_argument("--long-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--prefill-entry", choices=PREFILL_ENTRIES, default="split",
-                    help="prefill entry point of the timed step (default: gdn_chunk_fwd_split, the "
-                         "fastest on B=1, T=4096; the others are timed beside it)")
+    ap.add_argument("--prefill-entry", choices=PREFILL_ENTRIES, default="pipelined",
+                    help="prefill entry point of the timed step (default: gdn_chunk_fwd_pipelined, "
+                         "the fastest on B=1, T=4096; the others are timed beside it)")
     ap.add_argument("--prefill-kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto",
                     help="kernel gdn_chunk_fwd / _split / _varlen run (default: the library's choice)")
     ap.add_argument("--profile-case", choices=["prefill", "prefill-batched", "prefill-long", "decode",

@@ -133,7 +133,7 @@ constexpr uint32_t OFF_V = OFF_KQ + NKQ * K_STAGE;     // 2 x [V j0-63][V j64-12
 constexpr uint32_t OFF_RB = OFF_V + 4 * TILE;          // NRB ring buffers: operand tiles (32 KB each)
 constexpr uint32_t OFF_RG = OFF_RB + NRB * RS_TILES;   // NRB ring buffers: gate vectors (512 B each)
 constexpr uint32_t OFF_CBAR = OFF_RG + NRB * RS_GATE_BYTES;
-constexpr uint32_t CH_NBAR = 38;
+constexpr uint32_t CH_NBAR = 40;
 // named barriers of the chain CTA: the state chain (conversion warpgroups + the
 // chain issuer warp), the conversion warpgroups alone, the helper warpgroup
 constexpr int kChainBar = 3, kChainThreads = 288, kConvBar = 5;
@@ -163,6 +163,7 @@ enum : int {
     C_UT_FULL = 31,   // x2 U~^T of the chunk done (its U buffer)
     C_X_GO = 33,      // x2 critical issuer: UG(n) issued (per S^T bf16 buffer)
     C_O_GO = 35,      // x2 critical issuer: SG(n) issued (per U buffer)
+    C_K_FREE = 37,    // x3 helper: the O store staged in the K stage has read it
 };
 // Arrival counts: a tcgen05.commit counts one, a warp (warp_arrive) one.
 __host__ __device__ constexpr uint32_t chain_bar_count(int i) {
@@ -170,7 +171,7 @@ __host__ __device__ constexpr uint32_t chain_bar_count(int i) {
          : ((i >= C_KQ_EMPTY && i < C_KQ_EMPTY + NKQ) || i == C_DRAIN) ? 2u
          : (i == C_O_FREE || i == C_O_FREE + 1) ? 4u : 1u;
 }
-static_assert(C_O_GO + 1 < (int)CH_NBAR, "barrier count");
+static_assert(C_K_FREE + NKQ <= (int)CH_NBAR, "barrier count");
 
 // ---------------------------------------------------------------- prep role
 constexpr int NPKQ = 2;
@@ -409,7 +410,8 @@ __device__ __noinline__ void store_o_rows(__nv_bfloat16 *dst, uint32_t t_col, in
 
 // ============================================================================ chain
 __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorMap *tm_q,
-                                        const CUtensorMap *tm_v, const PipeParams &p, unsigned char *sm)
+                                        const CUtensorMap *tm_v, const CUtensorMap *tm_o,
+                                        const PipeParams &p, unsigned char *sm)
 {
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_CBAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_CMISC);
@@ -425,6 +427,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         prefetch_tensormap(tm_k);
         prefetch_tensormap(tm_q);
         prefetch_tensormap(tm_v);
+        prefetch_tensormap(tm_o);
         for (int i = 0; i < (int)CH_NBAR; ++i) mbar_init(&bar[i], chain_bar_count(i));
         *abort_local = 0;
         fence_mbar_init();
@@ -446,7 +449,8 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             while (nkq < N || nv < N) {
                 if (ctl.aborted_polled(next_poll)) break;
                 bool issued = false;
-                if (nkq < N && (nkq < NKQ || mbar_test(&bar[C_KQ_EMPTY + nkq % NKQ], ((nkq / NKQ) - 1) & 1))) {
+                if (nkq < N && (nkq < NKQ || (mbar_test(&bar[C_KQ_EMPTY + nkq % NKQ], ((nkq / NKQ) - 1) & 1) &&
+                                              mbar_test(&bar[C_K_FREE + nkq % NKQ], ((nkq / NKQ) - 1) & 1)))) {
                     const Unit u = unit_of(p, x, nkq);
                     const int s = nkq % NKQ, t0 = u.c * C;
                     unsigned char *st = sm + OFF_KQ + s * K_STAGE;
@@ -597,14 +601,18 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         //   #2 (S^T bf16 of n written):           UG(n)  U^T += S^T (-W)^T       8 MMAs
         //   #4 (U^T bf16 copies, decayed S^T):     SG(n)  S^T += (U diag(g))^T K  4 MMAs
         // The commits that release the K stage and the ring slot of n are issued after
-        // UG(n+1) (they then also cover it), off the hand-off to the conversion.
+        // UG(n+1) (they then also cover it; the last chunk's after the loop), off the
+        // hand-off to the conversion.
         bool ok = true;
         for (int n = 0; n < N && ok; ++n) {
             const int s = n & 1, nk = n % NKQ, nr = n % NRB;
             const uint32_t st = sbase + OFF_KQ + nk * K_STAGE;
             const uint32_t rb = sbase + OFF_RB + nr * RS_TILES;
-            bool ut_ready = false;
-            if (lane == 0) ut_ready = mbar_test(&bar[C_UT_FULL + s], (n >> 1) & 1);
+            bool ut_ready = false, k_ready = false;
+            if (lane == 0) {
+                ut_ready = mbar_test(&bar[C_UT_FULL + s], (n >> 1) & 1);
+                k_ready = mbar_test(&bar[C_KQ_FULL + nk], (n / NKQ) & 1);
+            }
             ok = named_and(kChainBar, kChainThreads, true);           // #1
             if (!ok) break;
             named_sync(kChainBar, kChainThreads);                     // #2
@@ -635,7 +643,9 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             ok = named_and(kChainBar, kChainThreads, true);           // #3
             if (!ok) break;
             named_sync(kChainBar, kChainThreads);                     // #4
-            if (lane == 0) {   // SG(n)
+            if (lane == 0 && (k_ready || ctl.wait(C_KQ_FULL + nk, (n / NKQ) & 1))) {
+                // SG(n), once the chunk's K stage has landed (a wait that gave up leaves
+                // the chunk unissued; every waiter then sees the abort)
                 tc_fence_after();
                 PMCLK(x, n, 3);
 #pragma unroll
@@ -655,6 +665,10 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             __syncwarp();
         }
         if (lane == 0) {
+            if (ok && N > 0) {   // the last chunk's releases (the O epilogue waits for its K stage)
+                mma_commit(&bar[C_KQ_EMPTY + (N - 1) % NKQ]);
+                mma_commit(&bar[C_RB_EMPTY + (N - 1) % NRB]);
+            }
             mma_commit(&bar[C_DRAIN]);
             mbar_wait(&bar[C_DRAIN], 0, 1ll << 30);
         }
@@ -674,6 +688,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         const size_t hstate = (size_t)kHeadDim * kHeadDim;
         const int d0 = 64 * h2;
         bool ok = true;
+        bool pre_ready = false;                       // lane 0: X and ring tested for this chunk
         Unit u = unit_of(p, x, 0);
         for (int n = 0; n < N && ok; ++n) {
             const int s = n & 1;
@@ -687,17 +702,16 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             // chunk's state update is done (for a new head: the previous head's last
             // one, whose final state was stored below); the ring slot has landed.
             // One lane per warp waits (the named barrier then orders the others after
-            // it); the three are tested at once first, as they are usually complete.
+            // it).  The first and last were usually tested already, while the
+            // previous chunk's UG ran (pre_ready), so that only the state update is
+            // waited for here.
             if (lane == 0) {
-                const bool a = n < 2 || mbar_test(&bar[C_X_FULL + s], ((n >> 1) - 1) & 1);
-                const bool b = n == 0 || mbar_test(&bar[C_S_FULL], (n - 1) & 1);
-                const bool c = mbar_test(&bar[C_RB_FULL + nr], (n / NRB) & 1);
                 if (tr0) PMCLK(x, n, 6);
-                if (!(a && b && c))
-                    ok = (a || ctl.wait(C_X_FULL + s, ((n >> 1) - 1) & 1)) &&
-                         (b || ctl.wait_fast(C_S_FULL, (n - 1) & 1)) &&
-                         (c || ctl.wait(C_RB_FULL + nr, (n / NRB) & 1));
+                if (!pre_ready)
+                    ok = ctl.wait(C_RB_FULL + nr, (n / NRB) & 1) &&
+                         (n < 2 || ctl.wait(C_X_FULL + s, ((n >> 1) - 1) & 1));
                 if (tr0) PMCLK(x, n, 7);
+                ok = ok && (n == 0 || ctl.wait_fast(C_S_FULL, (n - 1) & 1));
                 if (tr0) PMCLK(x, n, 8);
             }
             ok = named_and(kChainBar, kChainThreads, ok);             // #1
@@ -739,6 +753,11 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             // update, so that K needs no scaling).  Both warpgroups load their half
             // before either writes (the packed copies overlap the fp32 halves).
             if (tr0) PMCLK(x, n, 13);
+            if (lane == 0) {   // the next chunk's ring slot and S^T bf16 buffer, while UG runs
+                const int m = n + 1;
+                pre_ready = m < N && mbar_test(&bar[C_RB_FULL + m % NRB], (m / NRB) & 1) &&
+                            (m < 2 || mbar_test(&bar[C_X_FULL + (m & 1)], ((m >> 1) - 1) & 1));
+            }
             ok = named_and(kChainBar, kChainThreads, lane != 0 || ctl.wait_fast(C_U_FULL, n & 1));   // #3
             if (!ok) break;
             if (tr0) PMCLK(x, n, 14);
@@ -760,12 +779,13 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     pk[xx] = pack_bf16x2(uu[2 * xx] * gg[2 * xx], uu[2 * xx + 1] * gg[2 * xx + 1]);
                 tmem_st16u(t_row + COL_U + s * 64 + 32 + 16 * h2, pk);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[C_RB_EMPTY + nr]);   // gates of n no longer read here
             tmem_wait_st();                       // the bf16 copies and the decayed state
             if (tr0) PMCLK(x, n, 15);
             tc_fence_before();
             named_sync(kChainBar, kChainThreads);                     // #4
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[C_RB_EMPTY + nr]);   // gates of n no longer read here
+            if (tr0) PMCLK(x, n, 2);
             PTRACE(n, 8, x == 0 && j == 0 && h2 == 0);
             PCHAIN(x, n, 6, j == 0 && h2 == 0);
             // last chunk of a head: store its final state once the update is done
@@ -779,17 +799,42 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         }
     } else if (warp >= 12) {
         // ============================================================ helper warpgroup
-        // The O epilogue of each chunk (TMEM -> registers -> bf16 stores of its rows).
+        // The O epilogue of each chunk: O^T (TMEM) -> registers, after which the O
+        // buffer is free; the bf16 tile O[r][j] goes by stmatrix into the chunk's K
+        // stage (free once the chunk's S and O MMAs are done: KQ_EMPTY) and out by two
+        // TMA stores; the stage returns to the K loads (C_K_FREE) once the store has
+        // read it, checked at the next chunk.  A chunk cut by the end of its sequence
+        // is stored row by row.
+        const int pt = tid - 384;
         const int q4 = warp & 3;
         const int j = q4 * 32 + lane;
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
+        const bool leader = pt == 0;
         const size_t row_stride = (size_t)p.Hv * kHeadDim;
+        const int mt = lane >> 3, mi = lane & 7;
         bool ok = true;
+        int pending = -1;                             // leader: K stage a store may still read
         Unit u = unit_of(p, x, 0);
+        // 16 lanes (j) x 32 columns (r) of O^T from tmem_ld16x256b_x4 -> O[r][j] bf16 in
+        // the 128B-swizzled staging tiles (j 0-63, j 64-127)
+        auto emit = [&](uint32_t stage, const uint32_t *rr, int sl, int cb) {
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+                uint32_t m[4];
+#pragma unroll
+                for (int mm = 0; mm < 4; ++mm) {
+                    const int k = 2 * kk + (mm >> 1), g = mm & 1;
+                    m[mm] = pack_bf16x2(__uint_as_float(rr[4 * k + 2 * g]), __uint_as_float(rr[4 * k + 2 * g + 1]));
+                }
+                const int k = 2 * kk + (mt >> 1), g = mt & 1;
+                const int orow = 32 * cb + 8 * k + mi;
+                const int jst = q4 * 32 + 16 * sl + 8 * g;
+                stmatrix_x4_trans(stage + (jst >> 6) * TILE + sw128_chunk(orow, (jst & 63) >> 3), m[0], m[1], m[2], m[3]);
+            }
+        };
         for (int n = 0; n < N && ok; ++n) {
-            const int s = n & 1;
+            const int s = n & 1, nk = n % NKQ;
             const uint32_t col_o = COL_O + s * 64;
-            // ---- epilogue of n
             ok = named_and(4, 128, lane != 0 || ctl.wait(C_O_FULL + s, (n >> 1) & 1));
             if (!ok) break;
             tc_fence_after();
@@ -798,27 +843,56 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 else u = unit_of_ool(p, x, n);
             }
             const int rows = min(C, p.T - u.c * C);
-            // thread j writes o[t][h][j] of the chunk's rows: each warp store covers 32
-            // consecutive j (64 contiguous bytes)
-            __nv_bfloat16 *dst = p.o + ((size_t)u.b * p.T + (size_t)u.c * C) * row_stride +
-                                 (size_t)u.h * kHeadDim + j;
             if (rows == C) {
-                float ov[64];
-                tmem_ld32(t_row + col_o, ov);
-                tmem_ld32(t_row + col_o + 32, ov + 32);
+                uint32_t a0[16], b0[16], a1[16], b1[16];
+                const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + col_o;
+                const uint32_t tb = tmem + ((uint32_t)(q4 * 32 + 16) << 16) + col_o;
+                tmem_ld16x256b_x4(ta, a0);
+                tmem_ld16x256b_x4(ta + 32, b0);
+                tmem_ld16x256b_x4(tb, a1);
+                tmem_ld16x256b_x4(tb + 32, b1);
                 tmem_wait_ld();
                 tc_fence_before();
-                warp_arrive(&bar[C_O_FREE + s]);        // the O buffer is free once read out
-#pragma unroll
-                for (int r = 0; r < C; ++r) dst[(size_t)r * row_stride] = __float2bfloat16_rn(ov[r]);
+                warp_arrive(&bar[C_O_FREE + s]);      // the O buffer is free once read out
+                if (leader && pending >= 0) {
+                    bulk_wait_group_read0();
+                    mbar_arrive(&bar[C_K_FREE + pending]);
+                    pending = -1;
+                }
+                ok = named_and(4, 128, lane != 0 || ctl.wait(C_KQ_EMPTY + nk, (n / NKQ) & 1));
+                if (!ok) break;
+                const uint32_t stage = sbase + OFF_KQ + nk * K_STAGE;
+                emit(stage, a0, 0, 0);
+                emit(stage, b0, 0, 1);
+                emit(stage, a1, 1, 0);
+                emit(stage, b1, 1, 1);
+                fence_proxy_async_smem();
+                named_sync(4, 128);
+                if (leader) {
+                    tma_store_4d(tm_o, sm + OFF_KQ + nk * K_STAGE, 0, u.h, u.c * C, u.b);
+                    tma_store_4d(tm_o, sm + OFF_KQ + nk * K_STAGE + TILE, 64, u.h, u.c * C, u.b);
+                    bulk_commit_group();
+                    pending = nk;
+                }
             } else {
+                __nv_bfloat16 *dst = p.o + ((size_t)u.b * p.T + (size_t)u.c * C) * row_stride +
+                                     (size_t)u.h * kHeadDim + j;
                 store_o_rows(dst, t_row + col_o, rows, row_stride);
                 tc_fence_before();
                 warp_arrive(&bar[C_O_FREE + s]);
+                if (leader) {
+                    if (pending >= 0) {
+                        bulk_wait_group_read0();
+                        mbar_arrive(&bar[C_K_FREE + pending]);
+                        pending = -1;
+                    }
+                    mbar_arrive(&bar[C_K_FREE + nk]);
+                }
             }
             PTRACE(n, 10, x == 0 && j == 0);
             PCHAIN(x, n, 7, j == 0);
         }
+        if (leader) bulk_wait_group0();               // the stores have read this CTA's memory
     }
 
     tc_fence_before();
@@ -1175,14 +1249,15 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
 
 __global__ void __launch_bounds__(NT, 1)
 chunk_pipe_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ PipeParams p)
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const __grid_constant__ PipeParams p)
 {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     PTRACE(0, 31, blockIdx.x == 0 && threadIdx.x == 0);
     PCTA(0);
     if ((int)blockIdx.x < p.n_chain)
-        chain_role(&tm_k, &tm_q, &tm_v, p, sm);
+        chain_role(&tm_k, &tm_q, &tm_v, &tm_o, p, sm);
     else
         prep_role(&tm_k, &tm_q, p, sm);
     PCTA(1);
@@ -1277,9 +1352,9 @@ cudaError_t launch_chunk_pipe(const ChunkArgs &a, int chain_ctas, long long wait
     if (err != cudaSuccess) return err;
     if ((long long)per_sm * sms < n_chain + n_prep) return cudaErrorCooperativeLaunchTooLarge;
 
-    CUtensorMap tk, tq, tv;
+    CUtensorMap tk, tq, tv, to;
     if (!make_map(&tk, a.k, a.B, a.T, a.Hqk) || !make_map(&tq, a.q, a.B, a.T, a.Hqk) ||
-        !make_map(&tv, a.v, a.B, a.T, a.Hv))
+        !make_map(&tv, a.v, a.B, a.T, a.Hv) || !make_map(&to, a.o, a.B, a.T, a.Hv))
         return cudaErrorInvalidValue;
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     unsigned *flags = reinterpret_cast<unsigned *>(ws);
@@ -1303,7 +1378,7 @@ cudaError_t launch_chunk_pipe(const ChunkArgs &a, int chain_ctas, long long wait
     p.abort = flags + (size_t)2 * n_chain * kFlagWords;
     p.ring = ws + fb;
     p.wait_limit = wait_limit > 0 ? wait_limit : (1ll << 32);
-    void *args[] = {&tk, &tq, &tv, &p};
+    void *args[] = {&tk, &tq, &tv, &to, &p};
     return cudaLaunchCooperativeKernel((const void *)chunk_pipe_kernel, dim3((unsigned)(n_chain + n_prep)),
                                        dim3(NT), args, SMEM_BYTES, stream);
 }
