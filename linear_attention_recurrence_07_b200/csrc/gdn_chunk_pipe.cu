@@ -545,7 +545,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16_ts(tmem + COL_O + s * 64, tmem + COL_U + s * 64 + k * 8,
+                    mma_bf16_ts(tmem + COL_O + s * 64, tmem + COL_U + s * 64 + 32 * (k >> 1) + 8 * (k & 1),
                                 smem_desc_sw128(rb + RS_P + k * 32, 16, 1024), ID_O, true);
                 mma_commit(&bar[C_O_FULL + s]);
                 mma_commit(&bar[C_RB_EMPTY + n % NRB]);
@@ -613,6 +613,9 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 ut_ready = mbar_test(&bar[C_UT_FULL + s], (n >> 1) & 1);
                 k_ready = mbar_test(&bar[C_KQ_FULL + nk], (n / NKQ) & 1);
             }
+            uint64_t wdesc[8];                        // UG's B operands, ready before the barrier
+#pragma unroll
+            for (int k = 0; k < 8; ++k) wdesc[k] = smem_desc_sw128(rb + RS_W + k * 2048, 2 * TILE, 1024);
             ok = named_and(kChainBar, kChainThreads, true);           // #1
             if (!ok) break;
             named_sync(kChainBar, kChainThreads);                     // #2
@@ -622,8 +625,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     PMCLK(x, n, 0);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_bf16_ts(tmem + COL_U + s * 64, tmem + COL_SB + s * 64 + k * 8,
-                                    smem_desc_sw128(rb + RS_W + k * 2048, 2 * TILE, 1024), ID_U, true);
+                        mma_bf16_ts(tmem + COL_U + s * 64, tmem + COL_SB + s * 64 + k * 8, wdesc[k], ID_U, true);
                     PMCLK(x, n, 1);
                     mma_commit(&bar[C_U_FULL]);
 #ifdef GDN_TRACE_MMA
@@ -650,7 +652,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 PMCLK(x, n, 3);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
-                    mma_bf16_ts(tmem + COL_S, tmem + COL_U + s * 64 + 32 + k * 8,
+                    mma_bf16_ts(tmem + COL_S, tmem + COL_U + s * 64 + 32 * (k >> 1) + 16 + 8 * (k & 1),
                                 smem_desc_sw128(st + k * 2048, TILE, 1024), ID_S, true);
                 PMCLK(x, n, 4);
                 mma_commit(&bar[C_S_FULL]);
@@ -685,6 +687,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         const int j = q4 * 32 + lane;                 // TMEM lane = value column j
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
         const bool tr0 = warp == 4 && lane == 0;      // trace stamps
+        const bool has_final = p.S_final != nullptr;
         const size_t hstate = (size_t)kHeadDim * kHeadDim;
         const int d0 = 64 * h2;
         bool ok = true;
@@ -748,10 +751,10 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 tmem_st32(t_row + COL_S + d0, v);
                 tmem_st32(t_row + COL_S + d0 + 32, v + 32);
             }
-            // U^T (fp32, 64 columns) -> two packed bf16 copies in place: U^T (columns
-            // 0-31, for the O MMAs) and (U diag(g))^T (columns 32-63, for the state
-            // update, so that K needs no scaling).  Both warpgroups load their half
-            // before either writes (the packed copies overlap the fp32 halves).
+            // U^T (fp32, 64 columns) -> two packed bf16 copies in place, each warpgroup
+            // over its own 32 columns: U^T of its 32 rows r (columns 32h .. 32h+15, for
+            // the O MMAs) and (U diag(g))^T (columns 32h+16 .. 32h+31, for the state
+            // update, so that K needs no scaling).
             if (tr0) PMCLK(x, n, 13);
             if (lane == 0) {   // the next chunk's ring slot and S^T bf16 buffer, while UG runs
                 const int m = n + 1;
@@ -769,15 +772,14 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 uint32_t pk[16];
                 tmem_ld32(t_row + COL_U + s * 64 + 32 * h2, uu);
                 tmem_wait_ld();
-                named_sync(kConvBar, 256);
 #pragma unroll
                 for (int xx = 0; xx < 16; ++xx) pk[xx] = pack_bf16x2(uu[2 * xx], uu[2 * xx + 1]);
-                tmem_st16u(t_row + COL_U + s * 64 + 16 * h2, pk);
+                tmem_st16u(t_row + COL_U + s * 64 + 32 * h2, pk);
                 const float *gg = gv + C + 32 * h2;   // g_r of this half's rows r
 #pragma unroll
                 for (int xx = 0; xx < 16; ++xx)
                     pk[xx] = pack_bf16x2(uu[2 * xx] * gg[2 * xx], uu[2 * xx + 1] * gg[2 * xx + 1]);
-                tmem_st16u(t_row + COL_U + s * 64 + 32 + 16 * h2, pk);
+                tmem_st16u(t_row + COL_U + s * 64 + 32 * h2 + 16, pk);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar[C_RB_EMPTY + nr]);   // gates of n no longer read here
@@ -789,7 +791,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             PTRACE(n, 8, x == 0 && j == 0 && h2 == 0);
             PCHAIN(x, n, 6, j == 0 && h2 == 0);
             // last chunk of a head: store its final state once the update is done
-            if (u.c == nck - 1 && p.S_final) {
+            if (u.c == nck - 1 && has_final) {
                 ok = named_and(kConvBar, 256, lane != 0 || ctl.wait(C_S_FULL, n & 1));
                 if (!ok) break;
                 tc_fence_after();
@@ -811,6 +813,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         const uint32_t t_row = tmem + ((uint32_t)(q4 * 32) << 16);
         const bool leader = pt == 0;
         const size_t row_stride = (size_t)p.Hv * kHeadDim;
+        const int T = p.T;
         const int mt = lane >> 3, mi = lane & 7;
         bool ok = true;
         int pending = -1;                             // leader: K stage a store may still read
@@ -842,7 +845,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 if (u.c + 1 < nck) ++u.c;
                 else u = unit_of_ool(p, x, n);
             }
-            const int rows = min(C, p.T - u.c * C);
+            const int rows = min(C, T - u.c * C);
             if (rows == C) {
                 uint32_t a0[16], b0[16], a1[16], b1[16];
                 const uint32_t ta = tmem + ((uint32_t)(q4 * 32) << 16) + col_o;
