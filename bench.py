@@ -108,13 +108,14 @@ def load_peaks():
 
 
 def kernel_traffic(key, workload):
-    """DRAM bytes of one timed step from the committed ncu summary: only if the entry
-    was captured on this workload (its ``workload_name``) from the current sources of
-    every kernel of the step (their hash); else None."""
+    """DRAM bytes of one timed step from the committed ncu summary (entry
+    ``"<key>:<workload>"``): only if it was captured on this workload (its
+    ``workload_name``) from the current sources of every kernel of the step (their
+    hash); else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            entry = json.load(f)[key]
+            entry = json.load(f)[f"{key}:{workload}"]
         if entry.get("workload_name") != workload:
             return None
         h = hashlib.sha256()
@@ -531,8 +532,21 @@ ENTRY_TIMED = {"pipelined": "the whole pipelined launch (prep and chain CTAs) an
 PREFILL_TARGET_FRAC = 0.5
 
 
+def leg_entry(w, entry):
+    """The entry point a prefill leg times: the pipelined entry needs SMs for its
+    preparation CTAs beside one chain CTA per head, so with more heads than half the
+    SMs (B * Hv > SMs / 2) it runs its heads in waves with too few preparation CTAs;
+    such workloads go through the split entry (which then runs the one-CTA kernel)."""
+    if entry == "pipelined":
+        sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+        if 2 * w.B * w.Hv > sms:
+            return "split"
+    return entry
+
+
 def prefill_leg(w, entry, steps, warmup, world, rank, peaks, peak_src):
     """One prefill workload through `entry` (inputs larger than L2: no flush)."""
+    entry = leg_entry(w, entry)
     r = time_prefill(w, steps, warmup, world, rank, entry=entry, flush_l2=False)
     tok = w.B * w.T
     t = r["per_launch_ms"] * 1e-3
