@@ -85,7 +85,7 @@ __device__ __forceinline__ unsigned long long gtimer() {
 __device__ long long g_pclk0[kGridCTAs];
 // clock64 stamps of the chain's MMA issuer: UG start / issued / done, SG start / issued /
 // done (the done stamps only in builds that spin on the completion, GDN_TRACE_MMA)
-__device__ long long g_pmclk[kGridCTAs][kGridChunks][16];
+__device__ long long g_pmclk[kGridCTAs][kGridChunks][24];
 #define PMCLK(x, n, k) do { if ((x) < kGridCTAs && (n) < kGridChunks) g_pmclk[(x)][(n)][(k)] = clock64(); } while (0)
 #define PCTA(slot) do { if (threadIdx.x == 0 && blockIdx.x < kGridCTAs) { g_pcta[blockIdx.x][(slot)] = gtimer(); \
     unsigned sid; asm volatile("mov.u32 %0, %%smid;" : "=r"(sid)); g_pcta[blockIdx.x][2] = sid; \
@@ -114,7 +114,7 @@ constexpr uint32_t RS_GATE = 6 * TILE;                // gamma[64], g[64] fp32
 constexpr uint32_t RS_TILES = 6 * TILE;               // operand tiles of a slot (loaded as one copy)
 constexpr uint32_t RS_GATE_BYTES = 512;               // the gate vectors (a second copy)
 constexpr uint32_t RS_BYTES = 49 * 1024;              // slot stride in the ring (1024-multiple)
-constexpr int kRing = 8;                              // slots per chain CTA
+constexpr int kRing = 16;                             // slots per chain CTA
 constexpr int kFlagWords = 32;                        // one 128-byte line per chain CTA's flags
 
 // ---------------------------------------------------------------- chain role
@@ -459,6 +459,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     tma_load_4d(st + TILE, tm_k, &bar[C_KQ_FULL + s], 64, u.hq, t0, u.b);
                     PTRACE(nkq, 11, x == 0);
                     PCHAIN(x, nkq, 12, true);
+                    PMCLK(x, nkq, 20);
                     ++nkq;
                     issued = true;
                 }
@@ -569,12 +570,15 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
             bool ok = true;
             for (int n = 0; n < N && ok; ++n) {
                 const int r = n % NRB;
+                PMCLK(x, n, 16);
                 const unsigned flag = ld_acquire(&ready[n % kRing]);
                 if (n >= NRB && !(ok = ctl.wait(C_RB_EMPTY + r, ((n / NRB) - 1) & 1))) break;
+                PMCLK(x, n, 17);
                 PTRACE(n, 12, x == 0);
                 if (flag < (unsigned)n + 1u && !(ok = ctl.wait_flag(&ready[n % kRing], (unsigned)n + 1u, 64))) break;
                 PTRACE(n, 0, x == 0);
                 PCHAIN(x, n, 1, true);
+                PMCLK(x, n, 18);
                 fence_proxy_async_global();
                 const unsigned char *src = ring + (size_t)(n % kRing) * RS_BYTES;
                 mbar_arrive_expect_tx(&bar[C_RB_FULL + r], RS_TILES + RS_GATE_BYTES);
@@ -585,6 +589,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     if (!(ok = ctl.wait(C_RB_FULL + (n - 1) % NRB, ((n - 1) / NRB) & 1))) break;
                     PTRACE(n - 1, 1, x == 0);
                     PCHAIN(x, n - 1, 2, true);
+                    PMCLK(x, n - 1, 19);
                     st_release(&p.consumed[(size_t)x * kFlagWords], (unsigned)n);
                 }
             }
@@ -805,8 +810,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         // buffer is free; the bf16 tile O[r][j] goes by stmatrix into the chunk's K
         // stage (free once the chunk's S and O MMAs are done: KQ_EMPTY) and out by two
         // TMA stores; the stage returns to the K loads (C_K_FREE) once the store has
-        // read it, checked at the next chunk.  A chunk cut by the end of its sequence
-        // is stored row by row.
+        // read it.  A chunk cut by the end of its sequence is stored row by row.
         const int pt = tid - 384;
         const int q4 = warp & 3;
         const int j = q4 * 32 + lane;
@@ -816,7 +820,6 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
         const int T = p.T;
         const int mt = lane >> 3, mi = lane & 7;
         bool ok = true;
-        int pending = -1;                             // leader: K stage a store may still read
         Unit u = unit_of(p, x, 0);
         // 16 lanes (j) x 32 columns (r) of O^T from tmem_ld16x256b_x4 -> O[r][j] bf16 in
         // the 128B-swizzled staging tiles (j 0-63, j 64-127)
@@ -857,11 +860,6 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 tmem_wait_ld();
                 tc_fence_before();
                 warp_arrive(&bar[C_O_FREE + s]);      // the O buffer is free once read out
-                if (leader && pending >= 0) {
-                    bulk_wait_group_read0();
-                    mbar_arrive(&bar[C_K_FREE + pending]);
-                    pending = -1;
-                }
                 ok = named_and(4, 128, lane != 0 || ctl.wait(C_KQ_EMPTY + nk, (n / NKQ) & 1));
                 if (!ok) break;
                 const uint32_t stage = sbase + OFF_KQ + nk * K_STAGE;
@@ -875,7 +873,8 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                     tma_store_4d(tm_o, sm + OFF_KQ + nk * K_STAGE, 0, u.h, u.c * C, u.b);
                     tma_store_4d(tm_o, sm + OFF_KQ + nk * K_STAGE + TILE, 64, u.h, u.c * C, u.b);
                     bulk_commit_group();
-                    pending = nk;
+                    bulk_wait_group_read0();          // the stage returns to the K loads as
+                    mbar_arrive(&bar[C_K_FREE + nk]);  // soon as the store has read it
                 }
             } else {
                 __nv_bfloat16 *dst = p.o + ((size_t)u.b * p.T + (size_t)u.c * C) * row_stride +
@@ -883,14 +882,7 @@ __device__ __noinline__ void chain_role(const CUtensorMap *tm_k, const CUtensorM
                 store_o_rows(dst, t_row + col_o, rows, row_stride);
                 tc_fence_before();
                 warp_arrive(&bar[C_O_FREE + s]);
-                if (leader) {
-                    if (pending >= 0) {
-                        bulk_wait_group_read0();
-                        mbar_arrive(&bar[C_K_FREE + pending]);
-                        pending = -1;
-                    }
-                    mbar_arrive(&bar[C_K_FREE + nk]);
-                }
+                if (leader) mbar_arrive(&bar[C_K_FREE + nk]);
             }
             PTRACE(n, 10, x == 0 && j == 0);
             PCHAIN(x, n, 7, j == 0);
@@ -1090,7 +1082,9 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
             const Item it = item_of(p, pidx + jj * p.n_prep, g);
             const int b = it.hh0 / p.Hv, h = it.hh0 - b * p.Hv + i;
             if (gate_warp) load_gates_pipe(p, b, h, it.c, lane, na0, na1, nb0, nb1);
-            if (pt == 0) ncons = ld_relaxed(&p.consumed[(size_t)(it.gi * g + i) * kFlagWords]);
+            // (the first kRing chunks need no check: no load, nothing to wait for)
+            if (pt == 0 && it.k * p.nchunks + it.c >= kRing)
+                ncons = ld_relaxed(&p.consumed[(size_t)(it.gi * g + i) * kFlagWords]);
         };
         prefetch(0, wg);
         bool ok = true;
@@ -1122,7 +1116,7 @@ __device__ __noinline__ void prep_role(const CUtensorMap *tm_k, const CUtensorMa
                 bool free_ok = true;
                 if (pt == 0 && n >= kRing) {
                     if (cons >= (unsigned)(n - kRing + 1)) fence_acquire_gpu();
-                    else free_ok = ctl.wait_flag(&p.consumed[(size_t)x * kFlagWords], (unsigned)(n - kRing + 1), 1024);
+                    else free_ok = ctl.wait_flag(&p.consumed[(size_t)x * kFlagWords], (unsigned)(n - kRing + 1), 256);
                 }
                 ok = named_and(nb, 128, free_ok);
                 if (!ok) break;
