@@ -120,6 +120,44 @@ __host__ __device__ constexpr bool many_arrivals(int i) {
 }
 static_assert(B_O_FULL + 2 <= (int)NBAR, "barrier count");
 
+// Bounded waits for this kernel: the first try inline, the loop out of line, so
+// that the waiting code of the many call sites costs the per-chunk loops no
+// instruction-cache room.  A wait that gives up raises the abort flag and the
+// device error word; every role then stops.
+struct TcCtl {
+    uint64_t *bar;
+    volatile int *abort_flag;
+    __device__ __forceinline__ bool wait(int i, uint32_t parity) const {
+        return mbar_try_wait(&bar[i], parity) || wait_loop(i, parity);
+    }
+    __device__ __noinline__ bool wait_loop(int i, uint32_t parity) const {
+        const long long t0 = clock64();
+        for (;;) {
+            if (mbar_try_wait_suspend(&bar[i], parity, 20000)) return true;
+            if (*abort_flag) return false;
+            if (clock64() - t0 > (1ll << 32)) {
+                *abort_flag = 1;
+                atomicOr(&g_tc_error, 1u);
+                return false;
+            }
+        }
+    }
+};
+
+// O rows of a chunk cut by the end of its sequence (rows < C exist), from the
+// warp's TMEM lanes at t_col; out of line (rare).
+__device__ __noinline__ void tc_store_o_rows(__nv_bfloat16 *dst, uint32_t t_col, int rows, size_t row_stride) {
+#pragma unroll 1
+    for (int r0 = 0; r0 < C; r0 += 32) {
+        float ov[32];
+        tmem_ld32(t_col + r0, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+            if (r0 + x < rows) dst[(size_t)(r0 + x) * row_stride] = __float2bfloat16_rn(ov[x]);
+    }
+}
+
 __global__ void __maxnreg__(128)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -132,7 +170,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
-    const Ctl ctl{bar, abort_flag};
+    const TcCtl ctl{bar, abort_flag};
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.x;
@@ -568,16 +606,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
                 return true;
             }
-            __nv_bfloat16 *dst = out_h + (size_t)cp * C * row_stride;
-#pragma unroll 1
-            for (int r0 = 0; r0 < C; r0 += 32) {
-                float ov[32];
-                tmem_ld32(t_row + col_o + r0, ov);
-                tmem_wait_ld();
-#pragma unroll
-                for (int x = 0; x < 32; ++x)
-                    if (r0 + x < rows) dst[(size_t)(r0 + x) * row_stride] = __float2bfloat16_rn(ov[x]);
-            }
+            tc_store_o_rows(out_h + (size_t)cp * C * row_stride, t_row + col_o, rows, row_stride);
             tc_fence_before();
             mbar_arrive(&bar[B_O_FREE + (cp & 1)]);
             return true;
