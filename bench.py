@@ -265,9 +265,7 @@ def launches_per_call(w, entry):
         return 1
     if binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv) == 0:
         return 1
-    two = (binding.split_workspace_bytes(w.B, w.T, w.Hv, 0, w.dk, w.dv)
-           == binding.split_workspace_bytes(w.B, w.T, w.Hv, 2, w.dk, w.dv))
-    return 2 if two else 3
+    return 3   # segment launch of the chunk kernel, segment chain (or final state), fix-up
 
 
 def time_prefill(w, steps, warmup, world, rank, entry="pipelined", flush_l2=True):

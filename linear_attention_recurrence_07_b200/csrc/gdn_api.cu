@@ -313,11 +313,12 @@ gdn_status gdn_device_status(void *stream)
 {
     cudaError_t err = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (err != cudaSuccess) return cuda_status(err);
-    unsigned a = 0, b = 0;
+    unsigned a = 0, b = 0, c = 0;
     err = gdn::chunk_pipe_take_error(&a);
     if (err == cudaSuccess) err = gdn::chunk_tc_take_error(&b);
+    if (err == cudaSuccess) err = gdn::split_take_error(&c);
     if (err != cudaSuccess) return cuda_status(err);
-    return (a | b) ? GDN_ERR_TIMEOUT : GDN_OK;
+    return (a | b | c) ? GDN_ERR_TIMEOUT : GDN_OK;
 }
 
 const char *gdn_status_string(gdn_status status)

@@ -68,6 +68,7 @@ cudaError_t launch_chunk_pipe(const ChunkArgs &a, int chain_ctas, long long wait
 // Read and clear a kernel file's device error word (bit 0: a bounded wait gave up).
 cudaError_t chunk_pipe_take_error(unsigned *out);
 cudaError_t chunk_tc_take_error(unsigned *out);
+cudaError_t split_take_error(unsigned *out);
 
 // sst: null, or where the first segments write S_start(1)^T in bf16 (see TcParams).
 cudaError_t launch_chunk_tc_segments(const ChunkArgs &a, int seg_len, int nseg, float *segD,

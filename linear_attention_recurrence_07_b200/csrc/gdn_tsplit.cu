@@ -13,11 +13,11 @@
 //   2. seg_chain_kernel walks the segments of each (sequence, head):
 //      S_start(k+1) = M_k S_start(k) + D_k in fp32, keeping every S_start(k)^T
 //      in bf16;
-//   3. out_fix_kernel adds R S_start(k) to the outputs of segment k >= 1
-//      (bf16 warp MMAs, fp32 accumulation, one rounding to bf16).
+//   3. fix_tc_kernel adds R S_start(k) to the outputs of segment k >= 1 on the
+//      tensor core (tcgen05, fp32 accumulation in TMEM, one rounding to bf16).
 // With two segments, S_start(1) = D_0: the chunk kernel writes its bf16 transpose
-// itself, and the fix-up and the final state M_1 D_0 + D_1 no longer depend on
-// each other, so one launch (split2_finish_kernel) runs both side by side.
+// itself, so step 2 shrinks to the final state M_1 D_0 + D_1 (split2_state_kernel,
+// only when the caller asks for it) and the fix-up no longer waits for it.
 // The serial chain of chunk steps is one segment long instead of the sequence.
 #include "tc_common.cuh"
 
@@ -26,10 +26,6 @@ namespace {
 
 constexpr int kChainThreads = 256;
 constexpr int kChainCols = 32;            // state columns per CTA of seg_chain_kernel
-constexpr int kFixRows = 64;              // output rows per tile of out_fix_kernel
-constexpr int kFixTiles = 2;              // tiles per CTA (the S_start tile is staged once)
-constexpr int kLdR = kHeadDim + 8;        // padded bf16 row strides in shared memory
-constexpr int kLdS = kHeadDim + 8;
 constexpr int kLdM = kHeadDim + 1;        // padded row stride of the staged M (floats): the
                                           // threads of a warp read rows i0 + x at one d, in
                                           // distinct banks
@@ -125,139 +121,148 @@ seg_chain_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
                                              blockIdx.z * kChainCols, true, chain_smem);
 }
 
-__device__ __forceinline__ uint32_t ld_u32(const __nv_bfloat16 *p) {
-    return *reinterpret_cast<const uint32_t *>(p);
-}
-
-// o[t] += R[t - seg_len] S_start(k) for the rows t of segment k >= 1.  One CTA of
-// 128 threads per kFixTiles x kFixRows rows (row group `grp`, counting the groups
-// of every later segment in order) of one (head, sequence); 4 warps of 16 rows x
-// 128 columns per tile.
-__device__ __forceinline__ void fix_rows(const __nv_bfloat16 *__restrict__ Rr,
-                                         const __nv_bfloat16 *__restrict__ sstT,
-                                         __nv_bfloat16 *__restrict__ o, int T, int seg_len, int nseg,
-                                         int Hv, int grp, int h, int b, __nv_bfloat16 *fix_smem)
-{
-    __nv_bfloat16 *sS = fix_smem;                        // S_start^T: [j][kLdS]
-    __nv_bfloat16 *sR = fix_smem + kHeadDim * kLdS;      // R tile: [kFixRows][kLdR]
-    __nv_bfloat16 *sO = sR + kFixRows * kLdR;            // o tile: [kFixRows][kLdR]
-    const int tid = threadIdx.x;
-    const int TR = T - seg_len;                          // rows of R
-    const int groups = (seg_len + kFixTiles * kFixRows - 1) / (kFixTiles * kFixRows);
-    const int k = 1 + grp / groups;                      // segment
-    const int seg_r0 = (k - 1) * seg_len;                // its first R row
-    const int r_begin = seg_r0 + (grp % groups) * kFixTiles * kFixRows;
-    const int r_end = min(min(r_begin + kFixTiles * kFixRows, seg_r0 + seg_len), TR);
-    const size_t row_stride = (size_t)Hv * kHeadDim;
-    const __nv_bfloat16 *St = sstT + (((size_t)b * (nseg - 1) + (k - 1)) * Hv + h) * kHeadDim * kHeadDim;
-#pragma unroll 16
-    for (int e = tid; e < kHeadDim * (kHeadDim / 8); e += 128) {
-        const int j = e / (kHeadDim / 8), c8 = e % (kHeadDim / 8);
-        *reinterpret_cast<uint4 *>(&sS[j * kLdS + 8 * c8]) =
-            *reinterpret_cast<const uint4 *>(St + (size_t)j * kHeadDim + 8 * c8);
-    }
-    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, tq = lane & 3;
-    for (int r0 = r_begin; r0 < r_end; r0 += kFixRows) {
-        __syncthreads();                                 // sS staged; previous tile stored
-        // R rows and the matching o^0 rows (o row of R row rr is rr + seg_len), 16-byte
-        // coalesced loads; rows past the segment are zero / not stored
-#pragma unroll 8
-        for (int e = tid; e < kFixRows * (kHeadDim / 8); e += 128) {
-            const int r = e / (kHeadDim / 8), c8 = e % (kHeadDim / 8);
-            uint4 v = make_uint4(0u, 0u, 0u, 0u), w = v;
-            if (r0 + r < r_end) {
-                v = *reinterpret_cast<const uint4 *>(Rr + ((size_t)b * TR + r0 + r) * row_stride +
-                                                     (size_t)h * kHeadDim + 8 * c8);
-                w = *reinterpret_cast<const uint4 *>(o + ((size_t)b * T + r0 + r + seg_len) * row_stride +
-                                                     (size_t)h * kHeadDim + 8 * c8);
-            }
-            *reinterpret_cast<uint4 *>(&sR[r * kLdR + 8 * c8]) = v;
-            *reinterpret_cast<uint4 *>(&sO[r * kLdR + 8 * c8]) = w;
-        }
-        __syncthreads();
-        // the accumulators start from o^0
-        float acc[16][4];
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const __nv_bfloat16 *orow = &sO[(16 * warp + g + 8 * half) * kLdR];
-#pragma unroll
-            for (int n = 0; n < 16; ++n) {
-                const float2 cur = __bfloat1622float2(
-                    *reinterpret_cast<const __nv_bfloat162 *>(orow + 8 * n + 2 * tq));
-                acc[n][2 * half] = cur.x;
-                acc[n][2 * half + 1] = cur.y;
-            }
-        }
-        const __nv_bfloat16 *a_lo = &sR[(16 * warp + g) * kLdR];
-        const __nv_bfloat16 *a_hi = &sR[(16 * warp + g + 8) * kLdR];
-#pragma unroll
-        for (int ks = 0; ks < kHeadDim / 16; ++ks) {
-            const int kc = 16 * ks + 2 * tq;
-            const uint32_t a0 = ld_u32(a_lo + kc), a1 = ld_u32(a_hi + kc);
-            const uint32_t a2 = ld_u32(a_lo + kc + 8), a3 = ld_u32(a_hi + kc + 8);
-#pragma unroll
-            for (int n = 0; n < 16; ++n) {
-                const __nv_bfloat16 *bp = &sS[(8 * n + g) * kLdS + kc];
-                const uint32_t b0 = ld_u32(bp), b1 = ld_u32(bp + 8);
-                asm volatile(
-                    "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-                    "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-                    : "+f"(acc[n][0]), "+f"(acc[n][1]), "+f"(acc[n][2]), "+f"(acc[n][3])
-                    : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-            }
-        }
-        // results back into the o tile (each warp its own 16 rows), then 16-byte stores
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            __nv_bfloat16 *orow = &sO[(16 * warp + g + 8 * half) * kLdR];
-#pragma unroll
-            for (int n = 0; n < 16; ++n)
-                *reinterpret_cast<__nv_bfloat162 *>(orow + 8 * n + 2 * tq) =
-                    __floats2bfloat162_rn(acc[n][2 * half], acc[n][2 * half + 1]);
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int e = tid; e < kFixRows * (kHeadDim / 8); e += 128) {
-            const int r = e / (kHeadDim / 8), c8 = e % (kHeadDim / 8);
-            if (r0 + r < r_end)
-                *reinterpret_cast<uint4 *>(o + ((size_t)b * T + r0 + r + seg_len) * row_stride +
-                                           (size_t)h * kHeadDim + 8 * c8) =
-                    *reinterpret_cast<const uint4 *>(&sO[r * kLdR + 8 * c8]);
-        }
-    }
-}
-
-__global__ void __launch_bounds__(128)
-out_fix_kernel(const __nv_bfloat16 *__restrict__ Rr, const __nv_bfloat16 *__restrict__ sstT,
-               __nv_bfloat16 *__restrict__ o, int T, int seg_len, int nseg, int Hv)
-{
-    extern __shared__ __align__(16) __nv_bfloat16 fix_smem[];
-    fix_rows(Rr, sstT, o, T, seg_len, nseg, Hv, blockIdx.x, blockIdx.y, blockIdx.z, fix_smem);
-}
-
-// Two segments: CTAs [0, n_state) compute the final state M_1 D_0 + D_1 (kStateCols
-// columns of one (head, sequence) each), the rest the output fix-up of segment 1,
-// whose S_start(1)^T the chunk kernel has written.
+// Two segments: the final state M_1 D_0 + D_1, kStateCols columns of one (head,
+// sequence) per CTA.
 constexpr int kStateCols = 16;            // 128 threads: one 4 x 4 tile each
 __global__ void __launch_bounds__(128)
-split2_finish_kernel(const float *__restrict__ segD, const float *__restrict__ segM,
-                     const __nv_bfloat16 *__restrict__ Rr, const __nv_bfloat16 *__restrict__ sstT,
-                     __nv_bfloat16 *__restrict__ o, float *S_final, int T, int seg_len, int Hv, int B)
+split2_state_kernel(const float *__restrict__ segD, const float *__restrict__ segM, float *S_final, int Hv)
 {
-    extern __shared__ __align__(16) unsigned char finish_smem[];
+    extern __shared__ __align__(16) float state_smem[];
     constexpr int per_head = kHeadDim / kStateCols;
-    const int n_state = S_final ? B * Hv * per_head : 0;
+    const int jb = blockIdx.x % per_head, bh = blockIdx.x / per_head;
+    chain_columns<128, kStateCols>(segD, segM, nullptr, S_final, 2, Hv, bh % Hv, bh / Hv, jb * kStateCols,
+                                   false, state_smem);
+}
+
+// o[t] += R[t - seg_len] S_start(k) for 128 rows of segment k >= 1 of one (sequence,
+// V head), on the tensor core.  The R rows (A: rows t, K = d) and S_start(k)^T (B:
+// rows j, K = d; both K-major) come in by TMA, 32 KB each as four 64 x 64 bf16 boxes
+// in the 128-byte swizzle; eight tcgen05 MMAs (M = N = 128, K = 16 each) accumulate
+// in TMEM; thread r reads row r back, adds the chunk kernel's o^0 and writes one bf16
+// rounding.  R rows past the segment or the sequence are loaded (zero past the end of
+// R) but not stored.  CTA x: tile x % tps of segment 1 + (x / tps) % (nseg - 1) of
+// (sequence, head) x / (tps (nseg - 1)), tps = ceil(seg_len / 128).
+constexpr int kFixTcRows = 128;
+constexpr uint32_t kFixTcTile = 64 * 64 * 2;                // one 64 x 64 bf16 box
+constexpr uint32_t kFixTcSmem = 8 * kFixTcTile + 64 + 1024; // A, B, barriers + flag, alignment
+
+__global__ void __launch_bounds__(128, 1)
+fix_tc_kernel(const __grid_constant__ CUtensorMap tm_r, const __grid_constant__ CUtensorMap tm_s,
+              __nv_bfloat16 *__restrict__ o, int T, int seg_len, int nseg, int Hv)
+{
+    extern __shared__ __align__(1024) unsigned char fix_raw[];
+    const int tps = (seg_len + kFixTcRows - 1) / kFixTcRows;
     const int x = blockIdx.x;
-    if (x < n_state) {
-        const int jb = x % per_head, bh = x / per_head;
-        chain_columns<128, kStateCols>(segD, segM, nullptr, S_final, 2, Hv, bh % Hv, bh / Hv,
-                                       jb * kStateCols, false, reinterpret_cast<float *>(finish_smem));
-        return;
+    const int tile = x % tps, km1 = (x / tps) % (nseg - 1), bh = x / (tps * (nseg - 1));
+    const int h = bh % Hv, b = bh / Hv;
+    const int TR = T - seg_len;                                      // rows of R
+    const int r0 = km1 * seg_len + tile * kFixTcRows;                // first R row of the tile
+    const int r_end = min(min(r0 + kFixTcRows, (km1 + 1) * seg_len), TR);
+    if (r0 >= r_end) return;                                         // a tile past a short last segment
+    unsigned char *sm = fix_raw + ((1024u - (smem_u32(fix_raw) & 1023u)) & 1023u);
+    unsigned char *sA = sm, *sB = sm + 4 * kFixTcTile;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + 8 * kFixTcTile);   // 0: loads, 1: MMAs
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + 8 * kFixTcTile + 16);
+    volatile int *s_ok = reinterpret_cast<volatile int *>(sm + 8 * kFixTcTile + 32);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    if (tid == 0) {
+        prefetch_tensormap(&tm_r);
+        prefetch_tensormap(&tm_s);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
     }
-    const int groups = (seg_len + kFixTiles * kFixRows - 1) / (kFixTiles * kFixRows);
-    const int y = x - n_state;                           // (b, h, group)
-    fix_rows(Rr, sstT, o, T, seg_len, 2, Hv, y % groups, (y / groups) % Hv, y / (groups * Hv),
-             reinterpret_cast<__nv_bfloat16 *>(finish_smem));
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], 8 * kFixTcTile);
+        const int srow = ((b * (nseg - 1) + km1) * Hv + h) * kHeadDim;   // S_start(k)^T row j = 0
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {   // box q: d-half q >> 1, 64-row half q & 1
+            tma_load_4d(sA + q * kFixTcTile, &tm_r, &bar[0], 64 * (q >> 1), h, r0 + 64 * (q & 1), b);
+            tma_load_4d(sB + q * kFixTcTile, &tm_s, &bar[0], 64 * (q >> 1), 0, srow + 64 * (q & 1), 0);
+        }
+        const bool loaded = mbar_wait(&bar[0], 0, 1ll << 30);
+        if (loaded) {
+            tc_fence_after();
+            constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {   // K-step k: d 16k .. 16k+15
+                const uint32_t off = (k >> 2) * 2 * kFixTcTile + (k & 3) * 32;
+                mma_bf16(tmem, smem_desc_sw128(smem_u32(sA) + off, 16, 1024),
+                         smem_desc_sw128(smem_u32(sB) + off, 16, 1024), idesc, k > 0);
+            }
+        } else {
+            atomicOr(&g_tc_error, 1u);
+        }
+        *s_ok = loaded ? 1 : 0;
+        mma_commit(&bar[1]);   // with no MMA issued it arrives at once
+    }
+    // thread r: row r of the tile (TMEM lane r) -> o[b][seg_len + r0 + r][h][:]
+    const int r = tid;
+    const bool live = r0 + r < r_end;
+    const size_t row_stride = (size_t)Hv * kHeadDim;
+    uint4 *orow = reinterpret_cast<uint4 *>(o + ((size_t)b * T + seg_len + r0 + r) * row_stride +
+                                            (size_t)h * kHeadDim);
+    uint4 old[16];
+    if (live) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) old[c] = orow[c];
+    }
+    __syncthreads();   // *s_ok written
+    const bool done = mbar_wait(&bar[1], 0, 1ll << 30);
+    if (!done && tid == 0) atomicOr(&g_tc_error, 1u);
+    const bool store = live && done && *s_ok;
+    tc_fence_after();
+    const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {   // columns j 32c .. 32c+31
+        float acc[32];
+        tmem_ld32(t_row + 32 * c, acc);
+        tmem_wait_ld();
+        if (store) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const __nv_bfloat162 *ov = reinterpret_cast<const __nv_bfloat162 *>(&old[4 * c + q]);
+                uint32_t pk[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(ov[e]);
+                    pk[e] = pack_bf16x2(f.x + acc[8 * q + 2 * e], f.y + acc[8 * q + 2 * e + 1]);
+                }
+                orow[4 * c + q] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
+    }
+}
+
+// Launches fix_tc_kernel over every later segment's rows.
+cudaError_t launch_fix_tc(const ChunkArgs &a, int seg_len, int nseg, const __nv_bfloat16 *R,
+                          const __nv_bfloat16 *sstT, cudaStream_t stream)
+{
+    CUtensorMap tr, ts;
+    if (!make_map(&tr, R, a.B, a.T - seg_len, a.Hv) ||
+        !make_map(&ts, sstT, 1, a.B * (nseg - 1) * a.Hv * kHeadDim, 1))
+        return cudaErrorInvalidValue;
+    cudaError_t err = cudaFuncSetAttribute(fix_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kFixTcSmem);
+    if (err != cudaSuccess) return err;
+    const int tps = (seg_len + kFixTcRows - 1) / kFixTcRows;
+    fix_tc_kernel<<<(unsigned)(a.B * a.Hv * (nseg - 1) * tps), 128, kFixTcSmem, stream>>>(
+        tr, ts, static_cast<__nv_bfloat16 *>(a.o), a.T, seg_len, nseg, a.Hv);
+    return cudaGetLastError();
 }
 
 constexpr size_t align_up(size_t x) { return (x + 1023) & ~(size_t)1023; }
@@ -304,19 +309,20 @@ cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *worksp
     __nv_bfloat16 *R = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_R);
     __nv_bfloat16 *sstT = reinterpret_cast<__nv_bfloat16 *>(ws + pl.off_S);
 
-    const size_t fix_smem = (size_t)(2 * kFixRows * kLdR + kHeadDim * kLdS) * sizeof(__nv_bfloat16);
-    const int groups = (pl.seg_len + kFixTiles * kFixRows - 1) / (kFixTiles * kFixRows);
     if (pl.nseg == 2) {
         cudaError_t err = launch_chunk_tc_segments(a, pl.seg_len, pl.nseg, segD, segM, R, sstT, stream);
         if (err != cudaSuccess) return err;
-        const size_t state_smem = ((size_t)kHeadDim * kLdM + (size_t)kHeadDim * kStateCols) * sizeof(float);
-        const size_t smem = state_smem > fix_smem ? state_smem : fix_smem;
-        err = cudaFuncSetAttribute(split2_finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (err != cudaSuccess) return err;
-        const int n_state = a.S_final ? a.B * a.Hv * (kHeadDim / kStateCols) : 0;
-        split2_finish_kernel<<<(unsigned)(n_state + a.B * a.Hv * groups), 128, smem, stream>>>(
-            segD, segM, R, sstT, static_cast<__nv_bfloat16 *>(a.o), a.S_final, a.T, pl.seg_len, a.Hv, a.B);
-        return cudaGetLastError();
+        if (a.S_final) {   // the final state M_1 D_0 + D_1 (fp32, CUDA cores)
+            const size_t smem = ((size_t)kHeadDim * kLdM + (size_t)kHeadDim * kStateCols) * sizeof(float);
+            err = cudaFuncSetAttribute(split2_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+            if (err != cudaSuccess) return err;
+            split2_state_kernel<<<(unsigned)(a.B * a.Hv * (kHeadDim / kStateCols)), 128, smem, stream>>>(
+                segD, segM, a.S_final, a.Hv);
+            err = cudaGetLastError();
+            if (err != cudaSuccess) return err;
+        }
+        return launch_fix_tc(a, pl.seg_len, pl.nseg, R, sstT, stream);
     }
     cudaError_t err = launch_chunk_tc_segments(a, pl.seg_len, pl.nseg, segD, segM, R, nullptr, stream);
     if (err != cudaSuccess) return err;
@@ -328,13 +334,17 @@ cudaError_t launch_chunk_tc_split(const ChunkArgs &a, int segments, void *worksp
                        chain_smem, stream>>>(segD, segM, sstT, a.S_final, pl.nseg, a.Hv);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    // each CTA covers up to kFixTiles x kFixRows rows of one segment
-    err = cudaFuncSetAttribute(out_fix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fix_smem);
-    if (err != cudaSuccess) return err;
-    out_fix_kernel<<<dim3((unsigned)((pl.nseg - 1) * groups), (unsigned)a.Hv, (unsigned)a.B),
-                     128, fix_smem, stream>>>(R, sstT, static_cast<__nv_bfloat16 *>(a.o), a.T, pl.seg_len,
-                                       pl.nseg, a.Hv);
-    return cudaGetLastError();
+    return launch_fix_tc(a, pl.seg_len, pl.nseg, R, sstT, stream);
+}
+
+// Reads and clears this file's error word (bit 0: a bounded wait of the fix-up gave up).
+cudaError_t split_take_error(unsigned *out)
+{
+    unsigned v = 0, zero = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_tc_error, sizeof(v));
+    if (err == cudaSuccess && v) err = cudaMemcpyToSymbol(g_tc_error, &zero, sizeof(zero));
+    *out = v;
+    return err;
 }
 
 }  // namespace gdn

@@ -579,6 +579,15 @@ def test_prefill_split_in_place_and_workspace_checks():
     binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], S, o, S, segments=2)
     torch.cuda.synchronize()
     assert torch.equal(o, o_ref) and torch.equal(S, S_ref)
+    # without S_final the state kernels are skipped; the outputs stay the same bits
+    for segments in (2, 3):
+        o_ref_n, _ = run_split(d, segments)
+        o_n = torch.full_like(o_ref, float("nan"))
+        binding.gdn_chunk_fwd_split(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], o_n, None,
+                                    segments=segments)
+        torch.cuda.synchronize()
+        assert torch.equal(o_n, o_ref_n), f"segments={segments}: o differs without S_final"
+    assert binding.device_status() == "GDN_OK"
     need = binding.split_workspace_bytes(1, 300, 6, 2)
     short = torch.empty(need - 1024, dtype=torch.uint8, device=DEV)
     with pytest.raises(binding.GdnError, match="INVALID_ARG"):
