@@ -62,6 +62,17 @@ def bwd_flops_per_token(w):
     return 21 * w.dk * w.dv * w.Hv
 
 
+def bwd_chunk_flops_per_token(w, C=64):
+    """Algorithmic FLOPs of the chunkwise backward per token: per V head the start
+    states (U = U~ - W S and the state update, 2 dk dv each), W and U~ (2C(dk+dv)),
+    the gradient chain (K dS', Q^T dO, W^T dU: 2 dk dv each; P^T dO: 2C dv), and
+    per chunk dO S^T, dU S^T, U dS'^T (2 dk dv each), dP, T^T dU, dU V^T (2C dv
+    each), (dP o Gam) K, (dP o Gam)^T Q, T^T dW, dW K^T, M K, M^T K (2C dk each),
+    T^T dT and Z T^T (2C^2 each); the grams once per QK head (4 C dk)."""
+    per_v = 16 * w.dk * w.dv + 2 * C * (8 * w.dk + 5 * w.dv) + 4 * C * C
+    return w.Hv * per_v + 4 * C * w.dk * w.Hqk
+
+
 def prefill_flops_per_token(w, C=64):
     """Algorithmic FLOPs of the chunkwise form per token: per V head the products
     U~, W (2C(dk+dv)), U = U~ - W S, Q S, S update (2 dk dv each) and the masked
@@ -386,9 +397,9 @@ def time_calls(call, steps, warmup, world):
             "launches": steps, "window": (wall0, wall1)}
 
 
-def time_backward(w, steps, warmup, world):
-    """gdn_bwd on the prefill workload: dO random, no S0 / dS_final (the
-    workload's own S0 is none either)."""
+def time_backward(w, steps, warmup, world, entry="chunk"):
+    """gdn_bwd_chunk (entry "chunk") or gdn_bwd ("token") on the prefill workload:
+    dO random, no S0 / dS_final (the workload's own S0 is none either)."""
     d = inputs.workload_inputs(w, device="cuda")
     g = torch.Generator(device="cuda").manual_seed(w.seed + 7)
     dO = torch.randn((w.B, w.T, w.Hv, w.dv), generator=g, device="cuda").to(w.dtype)
@@ -399,12 +410,13 @@ def time_backward(w, steps, warmup, world):
     da = torch.empty((w.B, w.T, w.Hv), **f32)
     db = torch.empty_like(da)
     dS0 = torch.empty((w.B, w.Hv, w.dk, w.dv), **f32)
-    ws = torch.empty(binding.bwd_workspace_bytes(w.B, w.T, w.Hv, w.dk, w.dv), dtype=torch.uint8,
-                     device="cuda")
+    ws_bytes, fn = ((binding.bwd_chunk_workspace_bytes, binding.gdn_bwd_chunk) if entry == "chunk"
+                    else (binding.bwd_workspace_bytes, binding.gdn_bwd))
+    ws = torch.empty(ws_bytes(w.B, w.T, w.Hv, w.dk, w.dv), dtype=torch.uint8, device="cuda")
 
     def call(i):
-        binding.gdn_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], dO, None,
-                        dq, dk, dv, da, db, dS0, workspace=ws)
+        fn(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], dO, None,
+           dq, dk, dv, da, db, dS0, workspace=ws)
 
     return time_calls(call, steps, warmup, world)
 
@@ -586,7 +598,7 @@ def profile_case(args):
         x = inputs.decode_inputs(w, 0, device="cuda", B=B)
         for _ in range(args.launches):
             binding.decode_step(x["q"], x["k"], x["v"], x["alpha"], x["beta"], S)
-    elif case == "bwd":
+    elif case in ("bwd", "bwd-chunk"):
         w = inputs.PREFILL_4K
         T = args.T or w.T
         d = inputs.workload_inputs(w, device="cuda", T=T)
@@ -596,10 +608,11 @@ def profile_case(args):
         grads = [torch.empty((w.B, T, w.Hqk, w.dk), **f32), torch.empty((w.B, T, w.Hqk, w.dk), **f32),
                  torch.empty((w.B, T, w.Hv, w.dv), **f32), torch.empty((w.B, T, w.Hv), **f32),
                  torch.empty((w.B, T, w.Hv), **f32), torch.empty((w.B, w.Hv, w.dk, w.dv), **f32)]
-        ws = torch.empty(max(binding.bwd_workspace_bytes(w.B, T, w.Hv), 1), dtype=torch.uint8, device="cuda")
+        ws_bytes, fn = ((binding.bwd_chunk_workspace_bytes, binding.gdn_bwd_chunk) if case == "bwd-chunk"
+                        else (binding.bwd_workspace_bytes, binding.gdn_bwd))
+        ws = torch.empty(max(ws_bytes(w.B, T, w.Hv), 1), dtype=torch.uint8, device="cuda")
         for _ in range(args.launches):
-            binding.gdn_bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], dO, None, *grads,
-                            workspace=ws)
+            fn(d["q"], d["k"], d["v"], d["alpha"], d["beta"], d["S0"], dO, None, *grads, workspace=ws)
     else:
         raise SystemExit(f"unknown profile case {case}")
     torch.cuda.synchronize()
@@ -616,7 +629,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--verify-steps", type=int, default=50)
     ap.add_argument("--varlen-steps", type=int, default=20)
-    ap.add_argument("--bwd-steps", type=int, default=5)
+    ap.add_argument("--bwd-steps", type=int, default=20)
+    ap.add_argument("--bwd-token-steps", type=int, default=3)
     ap.add_argument("--batched-steps", type=int, default=10)
     ap.add_argument("--long-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -625,7 +639,7 @@ def main():
                          "the fastest on B=1, T=4096; the others are timed beside it)")
     ap.add_argument("--prefill-kernel", choices=sorted(binding.PREFILL_KERNELS), default="auto",
                     help="kernel gdn_chunk_fwd / _split / _varlen run (default: the library's choice)")
-    ap.add_argument("--profile-case", choices=["prefill", "prefill-batched", "prefill-long", "decode",
+    ap.add_argument("--profile-case", choices=["prefill", "prefill-batched", "prefill-long", "decode", "bwd-chunk",
                                                "bwd"], default=None)
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--T", type=int, default=None)
@@ -664,7 +678,8 @@ def main():
     with ClockSampler(local) as clocks2:
         ver = time_verify(wv, args.verify_steps, args.warmup, world)
         vl = time_varlen(wl, args.varlen_steps, args.warmup, world)
-        bw = time_backward(w, args.bwd_steps, 3, world)
+        bw = time_backward(w, args.bwd_steps, 3, world, entry="chunk")
+        bwt = time_backward(w, args.bwd_token_steps, 1, world, entry="token")
     e2e = time_prefill_e2e(w, args.e2e_steps, 3, world, entry=entry)
 
     tokens_per_step = w.B * w.T
@@ -729,15 +744,26 @@ def main():
             "gpu_launches": ver["launches"],
         },
         "backward": {
-            "metric": "backward tokens/s (gdn_bwd: dq, dk, dv, dalpha, dbeta, dS0)",
+            "metric": "backward tokens/s (gdn_bwd_chunk: dq, dk, dv, dalpha, dbeta, dS0)",
             "workload": w.name, "B": w.B, "T": w.T,
             "value": job_throughput(tokens_per_step, args.bwd_steps, world, bw["total_ms"]),
             "unit": "tokens/s", "ms_per_call": bw["total_ms"] / args.bwd_steps,
-            "roofline": dict(roofline("alu", bwd_flops_per_token(w) * tokens_per_step
+            "vs_forward": (bw["total_ms"] / args.bwd_steps) / pre["per_launch_ms"],
+            "roofline": dict(roofline("tensor", bwd_chunk_flops_per_token(w) * tokens_per_step
                                       / (bw["per_launch_ms"] * 1e-3) / 1e12,
-                                      FP32_ALU_TFLOPS, "TFLOP/s", None),
-                             peak_source="fp32 lanes x max SM clock (148 x 128 x 2 x 1965 MHz)"),
-            "gpu_launches": bw["launches"],
+                                      peaks["bf16_tflops"], "TFLOP/s", None),
+                             peak_source=f"{peak_src} bf16 burst",
+                             algorithmic_flops_per_launch=bwd_chunk_flops_per_token(w) * tokens_per_step),
+            "gpu_launches": 4 * bw["launches"],
+            "token_serial": {
+                "entry": "gdn_bwd (fp32 CUDA cores, one token at a time)",
+                "ms_per_call": bwt["total_ms"] / args.bwd_token_steps,
+                "roofline": dict(roofline("alu", bwd_flops_per_token(w) * tokens_per_step
+                                          / (bwt["per_launch_ms"] * 1e-3) / 1e12,
+                                          FP32_ALU_TFLOPS, "TFLOP/s", None),
+                                 peak_source="fp32 lanes x max SM clock (148 x 128 x 2 x 1965 MHz)"),
+                "gpu_launches": bwt["launches"],
+            },
         },
         "varlen_prefill": {
             "metric": "packed-prefill tokens/s (gdn_chunk_fwd_varlen)",

@@ -393,6 +393,41 @@ gdn_status gdn_bwd(const void *q, const void *k, const void *v, const float *alp
                    int B, int T, int Hqk, int Hv, int dk_, int dv_, gdn_dtype dtype,
                    void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * gdn_bwd_chunk -- the same gradients as gdn_bwd, computed in the chunkwise (WY)
+ * form on tensor cores; bf16 q, k, v, dO only.
+ *
+ * Defines: the chain rule through the chunk equations of the WY evaluation of
+ * section 2.1 "Gated DeltaNet" of "Qwen3.8-Flash-Next 技术总结 -- Qwen4 架构的探路者"
+ * (the pages name the WY representation as what makes the layer trainable in
+ * parallel).  Per chunk of 64 tokens, from the chunk's start state S, with
+ * b = cumsum(log alpha), gamma = exp(b), Gam = exp(b_r - b_i) (i <= r),
+ * g = exp(b_63 - b), T = (I + strict_lower(diag(beta)(Gam o K K^T)))^-1:
+ *   W = T diag(beta gamma) K, U = T diag(beta) V - W S, O = diag(gamma) Q S + (Gam o Q K^T) U,
+ *   S' = gamma_63 S + K^T diag(g) U;
+ * serially from the last chunk, dU = diag(g) K dS' + (Gam o Q K^T)^T dO and
+ * dS = gamma_63 dS' + Q^T diag(gamma) dO - W^T dU; every other gradient per
+ * chunk from S, dS', U and dU.  Four launches: preparation (per chunk and QK
+ * head), forward state chain and gradient chain (per V head and 32 value
+ * columns), per-chunk gradients (per chunk and QK head).  Operands are bf16 (the
+ * start states, U, W, T, dU and dS' included), accumulation fp32; each output is
+ * within 2e-2 of max|ref| of the exact gradients (the forward's bf16 bar), and
+ * bitwise the same from call to call (no atomics).
+ *
+ * In / Out: as gdn_bwd, dtype GDN_BF16 (GDN_F32 -> GDN_ERR_UNSUPPORTED).
+ * workspace: device scratch of at least gdn_bwd_chunk_workspace(B, T, Hv, dk, dv)
+ *      bytes (about 128 KiB per chunk of 64 tokens and V head), 256-byte
+ *      aligned, owned by the caller; contents on entry do not matter; calls
+ *      sharing it must not overlap.  May be NULL when that size is 0 (T == 0).
+ * Sizes and errors as gdn_bwd; ceil(T / 64) <= 2^31 - 1 and Hqk <= 65535.
+ */
+size_t gdn_bwd_chunk_workspace(int B, int T, int Hv, int dk, int dv);
+gdn_status gdn_bwd_chunk(const void *q, const void *k, const void *v, const float *alpha,
+                         const float *beta, const float *S0, const void *dO, const float *dS_final,
+                         float *dq, float *dk, float *dv, float *dalpha, float *dbeta, float *dS0,
+                         int B, int T, int Hqk, int Hv, int dk_, int dv_, gdn_dtype dtype,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
 /* Static, NUL-terminated name of a status code. */
 const char *gdn_status_string(gdn_status status);
 

@@ -75,6 +75,10 @@ def library():
         lib.gdn_bwd.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp, fp, fp, fp, fp, fp, fp,
                                 I, I, I, I, I, I, I, vp, ctypes.c_size_t, vp]
         lib.gdn_bwd.restype = I
+        lib.gdn_bwd_chunk_workspace.argtypes = [I, I, I, I, I]
+        lib.gdn_bwd_chunk_workspace.restype = ctypes.c_size_t
+        lib.gdn_bwd_chunk.argtypes = lib.gdn_bwd.argtypes
+        lib.gdn_bwd_chunk.restype = I
         lib.gdn_chunk_fwd_pipelined_workspace.argtypes = [I, I, I, I, I]
         lib.gdn_chunk_fwd_pipelined_workspace.restype = ctypes.c_size_t
         lib.gdn_chunk_fwd_pipelined.argtypes = [vp, vp, vp, fp, fp, fp, vp, fp,
@@ -267,14 +271,13 @@ def bwd_workspace_bytes(B, T, Hv, dk=128, dv=128):
     return library().gdn_bwd_workspace(B, T, Hv, dk, dv)
 
 
-def gdn_bwd(q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, dS0,
-            workspace=None, stream=None):
-    """Gradients of sum <dO, o> + <dS_final, S_final> (C entry point ``gdn_bwd``).
+def bwd_chunk_workspace_bytes(B, T, Hv, dk=128, dv=128):
+    """Device scratch bytes gdn_bwd_chunk needs (C entry point ``gdn_bwd_chunk_workspace``)."""
+    return library().gdn_bwd_chunk_workspace(B, T, Hv, dk, dv)
 
-    q, k, v, dO: the forward's dtype; alpha, beta, S0, dS_final fp32 (S0 and
-    dS_final may be None).  Outputs (fp32, overwritten): dq, dk like q; dv like v;
-    dalpha, dbeta like alpha; dS0 [B, Hv, dk, dv].  ``workspace``: uint8 CUDA
-    tensor of at least bwd_workspace_bytes(...) bytes; None allocates one."""
+
+def _run_bwd(entry, ws_bytes, q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, dS0,
+             workspace, stream):
     B, T, Hqk, dkk = q.shape
     Hv, dvv = v.shape[2], v.shape[3]
     dev = q.device
@@ -291,15 +294,35 @@ def gdn_bwd(q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, d
         if t is not None:
             _expect(t, name, (B, Hv, dkk, dvv), f32, dev)
     if workspace is None:
-        workspace = torch.empty(max(bwd_workspace_bytes(B, T, Hv, dkk, dvv), 1), dtype=torch.uint8,
-                                device=dev)
+        workspace = torch.empty(max(ws_bytes(B, T, Hv, dkk, dvv), 1), dtype=torch.uint8, device=dev)
     elif workspace.device != dev or workspace.dtype != torch.uint8:
         raise GdnError("workspace must be a uint8 tensor on the inputs' device")
-    _check(_call(dev, library().gdn_bwd, _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0), _ptr(dO),
-                             _ptr(dS_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(dbeta),
-                             _ptr(dS0), B, T, Hqk, Hv, dkk, dvv, _DTYPES[q.dtype], _ptr(workspace),
-                             workspace.numel(), _stream_handle(stream, dev)),
-           "gdn_bwd")
+    _check(_call(dev, getattr(library(), entry), _ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta), _ptr(S0),
+                 _ptr(dO), _ptr(dS_final), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dalpha), _ptr(dbeta),
+                 _ptr(dS0), B, T, Hqk, Hv, dkk, dvv, _DTYPES[q.dtype], _ptr(workspace),
+                 workspace.numel(), _stream_handle(stream, dev)),
+           entry)
+
+
+def gdn_bwd(q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, dS0,
+            workspace=None, stream=None):
+    """Gradients of sum <dO, o> + <dS_final, S_final> (C entry point ``gdn_bwd``).
+
+    q, k, v, dO: the forward's dtype; alpha, beta, S0, dS_final fp32 (S0 and
+    dS_final may be None).  Outputs (fp32, overwritten): dq, dk like q; dv like v;
+    dalpha, dbeta like alpha; dS0 [B, Hv, dk, dv].  ``workspace``: uint8 CUDA
+    tensor of at least bwd_workspace_bytes(...) bytes; None allocates one."""
+    _run_bwd("gdn_bwd", bwd_workspace_bytes, q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv,
+             dalpha, dbeta, dS0, workspace, stream)
+
+
+def gdn_bwd_chunk(q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, dS0,
+                  workspace=None, stream=None):
+    """The gradients of gdn_bwd in the chunkwise form on tensor cores (C entry point
+    ``gdn_bwd_chunk``); bf16 q, k, v, dO, the same arguments; ``workspace`` of at
+    least bwd_chunk_workspace_bytes(...) bytes, None allocates one."""
+    _run_bwd("gdn_bwd_chunk", bwd_chunk_workspace_bytes, q, k, v, alpha, beta, S0, dO, dS_final, dq, dk,
+             dv, dalpha, dbeta, dS0, workspace, stream)
 
 
 def gdn_chunk_fwd_split_noalloc(q, k, v, alpha, beta, S0, o, S_final, segments=0, chunk=64,

@@ -373,4 +373,37 @@ gdn_status gdn_bwd(const void *q, const void *k, const void *v, const float *alp
     return cuda_status(gdn::launch_bwd(L, dtype, static_cast<cudaStream_t>(stream)));
 }
 
+size_t gdn_bwd_chunk_workspace(int B, int T, int Hv, int dk, int dv)
+{
+    if (dk != gdn::kHeadDim || dv != gdn::kHeadDim) return 0;
+    return gdn::bwd_chunk_workspace(B, T, Hv);
+}
+
+gdn_status gdn_bwd_chunk(const void *q, const void *k, const void *v, const float *alpha,
+                         const float *beta, const float *S0, const void *dO, const float *dS_final,
+                         float *dq, float *dk, float *dv, float *dalpha, float *dbeta, float *dS0,
+                         int B, int T, int Hqk, int Hv, int dk_, int dv_, gdn_dtype dtype,
+                         void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (B < 0 || T < 0) return GDN_ERR_INVALID_ARG;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_INVALID_ARG;
+    gdn_status st = check_heads(Hqk, Hv, dk_, dv_);
+    if (st != GDN_OK) return st;
+    if (dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B == 0) return GDN_OK;
+    if (B > 65535 || Hqk > 65535 || Hv > 65535) return GDN_ERR_UNSUPPORTED;
+    if (!dS0) return GDN_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !alpha || !beta || !dO || !dq || !dk || !dv || !dalpha || !dbeta))
+        return GDN_ERR_INVALID_ARG;
+    const void *ptrs[] = {q, k, v, alpha, beta, S0, dO, dS_final, dq, dk, dv, dalpha, dbeta, dS0};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_INVALID_ARG;
+    const size_t need = gdn::bwd_chunk_workspace(B, T, Hv);
+    if (need > 0 && (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return GDN_ERR_INVALID_ARG;
+    gdn::BwdLaunch L{q, k, v, dO, alpha, beta, S0, dS_final, dq, dk, dv, dalpha, dbeta, dS0,
+                     static_cast<float *>(workspace), B, T, Hqk, Hv};
+    return cuda_status(gdn::launch_bwd_chunk(L, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

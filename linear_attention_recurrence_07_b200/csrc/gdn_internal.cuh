@@ -58,6 +58,10 @@ struct BwdLaunch {
 };
 size_t bwd_workspace(int B, int T, int Hv);
 cudaError_t launch_bwd(const BwdLaunch &L, gdn_dtype dtype, cudaStream_t stream);
+// Chunkwise backward (gdn_bwd_chunk.cu, bf16 inputs): prep, forward state chain,
+// gradient chain and per-chunk gradients; workspace of bwd_chunk_workspace bytes.
+size_t bwd_chunk_workspace(int B, int T, int Hv);
+cudaError_t launch_bwd_chunk(const BwdLaunch &L, cudaStream_t stream);
 
 // Pipelined prefill (gdn_chunk_pipe.cu): prep CTAs stream each chunk's WY operands
 // to state-carrying chain CTAs through a ring in the workspace (cooperative launch).

@@ -36,7 +36,7 @@ def test_header_declares_the_entry_points():
               "gdn_version", "gdn_set_prefill_kernel", "gdn_get_prefill_kernel",
               "gdn_prefill_kernel_for", "gdn_decode_tokens", "gdn_decode_step_slots",
               "gdn_chunk_fwd_varlen", "gdn_chunk_fwd_split", "gdn_chunk_fwd_split_workspace",
-              "gdn_bwd", "gdn_bwd_workspace"):
+              "gdn_bwd", "gdn_bwd_workspace", "gdn_bwd_chunk", "gdn_bwd_chunk_workspace"):
         assert n in names, names
 
 
@@ -252,4 +252,36 @@ def test_bwd_argument_checks(lib):
     assert call(ws=None) == binding.GDN_ERR_INVALID_ARG
     assert call(nbytes=1024) == binding.GDN_ERR_INVALID_ARG
     assert call(ws=ctypes.c_void_p(0x1010)) == binding.GDN_ERR_INVALID_ARG   # not 256-byte aligned
+    assert call(B=0) == binding.GDN_OK
+
+
+def test_bwd_chunk_workspace_sizes(lib):
+    # per (sequence, V head, chunk of 64): W, U, dU (64 x 128 bf16), T, P (64 x 64
+    # bf16), S, dS' (128 x 128 bf16), b (64 fp32) and four fp32 sums; each array
+    # 256-byte aligned
+    per = 3 * 64 * 128 * 2 + 2 * 64 * 64 * 2 + 2 * 128 * 128 * 2 + 64 * 4
+    assert binding.bwd_chunk_workspace_bytes(1, 4096, 48) == 48 * 64 * (per + 16)
+    assert binding.bwd_chunk_workspace_bytes(2, 17, 6) == 12 * per + 256
+    assert binding.bwd_chunk_workspace_bytes(1, 0, 48) == 0
+    assert lib.gdn_bwd_chunk_workspace(1, 64, 48, 64, 128) == 0
+
+
+def test_bwd_chunk_argument_checks(lib):
+    def call(B=1, T=64, Hqk=1, Hv=1, dk=128, dv=128, dtype=1, ptr=FAKE, dS0=FAKE, ws=FAKE,
+             nbytes=1 << 40, out=FAKE):
+        return lib.gdn_bwd_chunk(ptr, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, out, FAKE, FAKE, FAKE,
+                                 FAKE, dS0, B, T, Hqk, Hv, dk, dv, dtype, ws, nbytes, None)
+    assert call(B=-1) == binding.GDN_ERR_INVALID_ARG
+    assert call(dtype=3) == binding.GDN_ERR_INVALID_ARG
+    assert call(dtype=0) == binding.GDN_ERR_UNSUPPORTED    # fp32 inputs: gdn_bwd
+    assert call(Hqk=2, Hv=3) == binding.GDN_ERR_UNSUPPORTED
+    assert call(dv=64) == binding.GDN_ERR_UNSUPPORTED
+    assert call(B=70000) == binding.GDN_ERR_UNSUPPORTED
+    assert call(ptr=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(out=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(dS0=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(ptr=MISALIGNED) == binding.GDN_ERR_INVALID_ARG
+    assert call(ws=None) == binding.GDN_ERR_INVALID_ARG
+    assert call(nbytes=1024) == binding.GDN_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(0x1010)) == binding.GDN_ERR_INVALID_ARG
     assert call(B=0) == binding.GDN_OK
