@@ -408,7 +408,7 @@ gdn_status gdn_bwd(const void *q, const void *k, const void *v, const float *alp
  * serially from the last chunk, dU = diag(g) K dS' + (Gam o Q K^T)^T dO and
  * dS = gamma_63 dS' + Q^T diag(gamma) dO - W^T dU; every other gradient per
  * chunk from S, dS', U and dU.  Four launches: preparation (per chunk and QK
- * head), forward state chain and gradient chain (per V head and 32 value
+ * head), forward state chain and gradient chain (per V head and 64 value
  * columns), per-chunk gradients (per chunk and QK head).  Operands are bf16 (the
  * start states, U, W, T, dU and dS' included), accumulation fp32; each output is
  * within 2e-2 of max|ref| of the exact gradients (the forward's bf16 bar), and

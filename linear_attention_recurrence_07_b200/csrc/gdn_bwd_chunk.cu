@@ -25,9 +25,9 @@
 // accumulation) fed by ldmatrix from padded shared-memory tiles:
 //   1. prep_kernel, per (chunk, QK head): grams, the triangular solve (fp32), and
 //      per V head W, U~, T, P and b into the workspace;
-//   2. fwd_chain_kernel, per (V head, 32 value columns): the chunk start states S
+//   2. fwd_chain_kernel, per (V head, 64 value columns): the chunk start states S
 //      (bf16, kept for step 4) and U = U~ - W S (over U~ in the workspace);
-//   3. grad_chain_kernel, per (V head, 32 value columns), chunks from the end: dS'
+//   3. grad_chain_kernel, per (V head, 64 value columns), chunks from the end: dS'
 //      (bf16) and dU per chunk, sum(dS' o S) per chunk, and dS0;
 //   4. grad_chunk_kernel, per (chunk, QK head), its V heads in turn: every other
 //      gradient, dq and dk summed over the V heads in registers (no atomics: the
@@ -44,8 +44,6 @@ constexpr int C = kChunk;            // 64 tokens per chunk
 constexpr int D = kHeadDim;          // 128
 constexpr int LDT = D + 8;           // row stride (elements) of 64 x 128 and 128 x 128 bf16 tiles
 constexpr int LDQ = C + 8;           // 64 x 64 bf16 tiles
-constexpr int JB = 32;               // value columns per chain CTA
-constexpr int LDJ = JB + 8;          // 64 x 32 and 128 x 32 bf16 tiles
 constexpr int LDF = C + 1;           // 64 x 64 fp32 tiles
 constexpr int kThreads = 256;        // 8 warps in every kernel
 constexpr float kLogFloor = -87.f;   // log alpha clamp (alpha = 0 stays finite)
@@ -59,8 +57,9 @@ struct Ws {
     bf16 *S;       // [ch][128][128] S at the chunk start, [d][j]
     bf16 *dSp;     // [ch][128][128] gradient of the chunk's end state, [d][j]
     bf16 *dU;      // [ch][64][128]  dU
-    float *gb;     // [ch][64]       b = cumsum(log alpha) inside the chunk
-    float *gC;     // [ch][4]        sum(dS' o S) over each 32-column block
+    float *gate;   // [ch][3][64]    b = cumsum(log alpha) inside the chunk, gamma = exp(b),
+                   //                g = exp(b_63 - b)
+    float *gC;     // [ch][2]        sum(dS' o S) over each 64-column block
 };
 
 struct Params {
@@ -101,7 +100,7 @@ __device__ __forceinline__ void warp_mma(float (&acc)[NT][4], const bf16 *A, int
                                          int ldb, int m0, int n0, int K, int lane)
 {
     static_assert(NT % 2 == 0, "n tiles in pairs");
-#pragma unroll 2
+#pragma unroll 8
     for (int k0 = 0; k0 < K; k0 += 16) {
         uint32_t a[4];
         if (AL == 0)
@@ -145,6 +144,8 @@ __device__ __forceinline__ void cp16(void *dst, const void *src, bool valid) {
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // ROWS x (8 NCH) bf16 from src (row r at src + r * src_ld) into dst (row stride ld);
 // rows >= valid_rows are zero-filled without being read.
@@ -158,6 +159,11 @@ __device__ __forceinline__ void load_tile(bf16 *dst, int ld, const bf16 *src, si
         const bool ok = r < valid_rows;
         cp16(dst + r * ld + 8 * c, src + (size_t)(ok ? r : 0) * src_ld + 8 * c, ok);
     }
+}
+
+// The 192 gate floats of a chunk (768 bytes) by 48 cp.async of 16 bytes.
+__device__ __forceinline__ void load_gate(float *dst, const float *src, int tid) {
+    if (tid < 48) cp16(dst + 4 * tid, src + 4 * tid, true);
 }
 
 // K K^T and Q K^T of one chunk (64 x 64, fp32) from the bf16 tiles; 8 warps.
@@ -180,10 +186,61 @@ __device__ __forceinline__ void chunk_grams(const bf16 *sK, const bf16 *sQ, floa
         }
 }
 
+// T = (I + A)^-1 for the strictly lower 64 x 64 A (fp32, row stride LDF), by 16 x 16
+// blocks: the diagonal blocks by forward substitution (one thread per column, the
+// column in registers), then block rows 1..3 in turn,
+//   T_ij = -T_ii sum_{j <= k < i} A_ik T_kj   (j < i),
+// every element of a stage in parallel.  xs: 768 floats of scratch.  Upper blocks
+// are written as zeros.  Called by all threads; ends with the result visible.
+__device__ __forceinline__ void invert_unit_lower(const float *fA, float *fT, float *xs, int tid)
+{
+    if (tid < 64) {
+        const int base = 16 * (tid >> 4), c = tid & 15;
+        float t[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float s = r == c ? 1.f : 0.f;
+#pragma unroll
+            for (int m = 0; m < r; ++m) s -= fA[(base + r) * LDF + base + m] * t[m];
+            t[r] = r < c ? 0.f : s;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) fT[(base + r) * LDF + base + c] = t[r];
+    } else {
+        for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {   // blocks (i, j), i < j
+            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int i = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+            const int j = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            fT[(16 * i + r) * LDF + 16 * j + c] = 0.f;
+        }
+    }
+    __syncthreads();
+    for (int i = 1; i < 4; ++i) {
+        for (int e = tid; e < i * 256; e += kThreads) {
+            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            float s = 0.f;
+            for (int k = j; k < i; ++k)
+#pragma unroll
+                for (int m = 0; m < 16; ++m)
+                    s += fA[(16 * i + r) * LDF + 16 * k + m] * fT[(16 * k + m) * LDF + 16 * j + c];
+            xs[e] = s;
+        }
+        __syncthreads();
+        for (int e = tid; e < i * 256; e += kThreads) {
+            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            float s = 0.f;
+#pragma unroll
+            for (int m = 0; m < 16; ++m) s += fT[(16 * i + r) * LDF + 16 * i + m] * xs[(j << 8) + (m << 4) + c];
+            fT[(16 * i + r) * LDF + 16 * j + c] = -s;
+        }
+        __syncthreads();
+    }
+}
+
 // ================================================================== 1. preparation
 // Per (chunk n, QK head hq, sequence b): grams once, then for each V head of the
-// group the decay b, the solve T = (I + A)^-1 (fp32, forward substitution; each
-// warp owns 8 columns, 4 lanes per column), W, U~, P; all to the workspace.
+// group the decay b, the solve T = (I + A)^-1 (fp32, blocked: see invert_unit_lower),
+// W, U~, P; all to the workspace.
 constexpr size_t P_K = 0;
 constexpr size_t P_Q = P_K + 64 * LDT * 2;
 constexpr size_t P_X = P_Q + 64 * LDT * 2;      // diag(beta gamma) K
@@ -193,8 +250,8 @@ constexpr size_t P_KK = P_T + 64 * LDQ * 2;
 constexpr size_t P_QK = P_KK + 64 * LDF * 4;
 constexpr size_t P_A = P_QK + 64 * LDF * 4;
 constexpr size_t P_TF = P_A + 64 * LDF * 4;     // T, fp32
-constexpr size_t P_G = P_TF + 64 * LDF * 4;     // b[64], beta[64]
-constexpr size_t P_BYTES = P_G + 2 * 64 * 4;
+constexpr size_t P_G = P_TF + 64 * LDF * 4;     // b[64], beta[64], gamma[64]
+constexpr size_t P_BYTES = P_G + 3 * 64 * 4;
 
 __global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
 {
@@ -204,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
     bf16 *sT = reinterpret_cast<bf16 *>(smem + P_T);
     float *fKK = reinterpret_cast<float *>(smem + P_KK), *fQK = reinterpret_cast<float *>(smem + P_QK);
     float *fA = reinterpret_cast<float *>(smem + P_A), *fT = reinterpret_cast<float *>(smem + P_TF);
-    float *sb = reinterpret_cast<float *>(smem + P_G), *sbeta = sb + 64;
+    float *sb = reinterpret_cast<float *>(smem + P_G), *sbeta = sb + 64, *sgam = sb + 128;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
     const int grp = p.Hv / p.Hqk;
@@ -235,50 +292,53 @@ __global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
                 if (lane >= o) s += y;
             }
             const float excl = s - (l0 + l1);
-            sb[r0] = excl + l0;
-            sb[r1] = excl + l0 + l1;
+            const float blast = __shfl_sync(0xffffffffu, s, 31);
+            const float b0 = excl + l0, b1 = excl + l0 + l1;
+            sb[r0] = b0;
+            sb[r1] = b1;
             sbeta[r0] = r0 < L ? be[(size_t)r0 * p.Hv] : 0.f;
             sbeta[r1] = r1 < L ? be[(size_t)r1 * p.Hv] : 0.f;
-            p.ws.gb[ch * 64 + r0] = sb[r0];
-            p.ws.gb[ch * 64 + r1] = sb[r1];
+            const float ga0 = expf(b0), ga1 = expf(b1);
+            sgam[r0] = ga0;
+            sgam[r1] = ga1;
+            float *gv = p.ws.gate + ch * 192;
+            *reinterpret_cast<float2 *>(gv + r0) = make_float2(b0, b1);
+            *reinterpret_cast<float2 *>(gv + 64 + r0) = make_float2(ga0, ga1);
+            *reinterpret_cast<float2 *>(gv + 128 + r0) = make_float2(expf(blast - b0), expf(blast - b1));
         }
         __syncthreads();
-        // A[r][m] = beta_r exp(b_r - b_m) KK[r][m] for m < r
-        for (int e = tid; e < 64 * 64; e += kThreads) {
-            const int r = e >> 6, m = e & 63;
-            fA[r * LDF + m] = m < r ? sbeta[r] * expf(sb[r] - sb[m]) * fKK[r * LDF + m] : 0.f;
-        }
-        __syncthreads();
-        // T[r][c] = [r == c] - sum_{c <= m < r} A[r][m] T[m][c]; column c = warp + 8 (lane >> 2)
+        // Gam[r][m] = exp(b_r - b_m) once per lower element: A[r][m] = beta_r Gam KK (m < r),
+        // P[r][m] = Gam QK (m <= r) -> workspace
         {
-            const int c = warp + 8 * (lane >> 2), q4 = lane & 3;
-            for (int r = 0; r < 64; ++r) {
-                float s = 0.f;
-                for (int m = c + q4; m < r; m += 4) s += fA[r * LDF + m] * fT[m * LDF + c];
-                s += __shfl_xor_sync(0xffffffffu, s, 1);
-                s += __shfl_xor_sync(0xffffffffu, s, 2);
-                if (q4 == 0) fT[r * LDF + c] = r < c ? 0.f : (r == c ? 1.f : -s);
-                __syncwarp();
+            bf16 *gP = p.ws.P + ch * 64 * 64;
+            for (int e = tid; e < 64 * 32; e += kThreads) {
+                const int r = e >> 5, m2 = 2 * (e & 31);
+                float pv[2];
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const int m = m2 + x;
+                    const float gam = m <= r ? __expf(sb[r] - sb[m]) : 0.f;
+                    fA[r * LDF + m] = m < r ? sbeta[r] * gam * fKK[r * LDF + m] : 0.f;
+                    pv[x] = gam * fQK[r * LDF + m];
+                }
+                *reinterpret_cast<uint32_t *>(gP + r * 64 + m2) = pack2(pv[0], pv[1]);
             }
         }
+        __syncthreads();
+        invert_unit_lower(fA, fT, reinterpret_cast<float *>(sX), tid);   // sX is free until below
         cp_wait_all();
         __syncthreads();
-        // bf16 T (tile and workspace), diag(beta gamma) K, diag(beta) V, P
+        // bf16 T (tile and workspace), diag(beta gamma) K, diag(beta) V
         bf16 *gT = p.ws.Tm + ch * 64 * 64;
-        bf16 *gP = p.ws.P + ch * 64 * 64;
         for (int e = tid; e < 64 * 32; e += kThreads) {
             const int r = e >> 5, c2 = 2 * (e & 31);
             const uint32_t t2 = pack2(fT[r * LDF + c2], fT[r * LDF + c2 + 1]);
             *reinterpret_cast<uint32_t *>(sT + r * LDQ + c2) = t2;
             *reinterpret_cast<uint32_t *>(gT + r * 64 + c2) = t2;
-            float p0 = 0.f, p1 = 0.f;
-            if (c2 <= r) p0 = expf(sb[r] - sb[c2]) * fQK[r * LDF + c2];
-            if (c2 + 1 <= r) p1 = expf(sb[r] - sb[c2 + 1]) * fQK[r * LDF + c2 + 1];
-            *reinterpret_cast<uint32_t *>(gP + r * 64 + c2) = pack2(p0, p1);
         }
         for (int e = tid; e < 64 * 64; e += kThreads) {
             const int r = e >> 6, c2 = 2 * (e & 63);
-            const float bg = sbeta[r] * expf(sb[r]), bt = sbeta[r];
+            const float bg = sbeta[r] * sgam[r], bt = sbeta[r];
             const float2 kv = unpack2(sK + r * LDT + c2), vv = unpack2(sV + r * LDT + c2);
             *reinterpret_cast<uint32_t *>(sX + r * LDT + c2) = pack2(bg * kv.x, bg * kv.y);
             *reinterpret_cast<uint32_t *>(sV + r * LDT + c2) = pack2(bt * vv.x, bt * vv.y);
@@ -307,243 +367,251 @@ __global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
 }
 
 // ================================================================== 2. forward chain
-// Per (32-column block jb, V head h, sequence b): S (128 x 32 fp32, mma accumulators,
+// Per (FJ-column block, V head h, sequence b): S (128 x FJ fp32, mma accumulators,
 // warp w rows 16w..16w+15) from S0, then per chunk: S -> workspace (bf16),
-// U = U~ - W S -> workspace, S <- gamma_{C-1} S + K^T diag(g) U.  The next chunk's
-// W and U~ load while the state update runs, its K while U of the chunk after is
-// formed.
-constexpr size_t F_W = 0;
-constexpr size_t F_K = F_W + 64 * LDT * 2;
-constexpr size_t F_UT = F_K + 64 * LDT * 2;     // U~ block, 64 x 32
-constexpr size_t F_S = F_UT + 64 * LDJ * 2;     // S block, bf16, 128 x 32 ([d][j])
-constexpr size_t F_U = F_S + 128 * LDJ * 2;     // diag(g) U block, bf16
-constexpr size_t F_G = F_U + 64 * LDJ * 2;      // g[64]
-constexpr size_t F_BYTES = F_G + 64 * 4;
+// U = U~ - W S -> workspace, S <- gamma_{C-1} S + K^T diag(g) U.  A two-stage ring
+// holds each chunk's W, K, U~ block and decay, loaded one whole chunk ahead, so the
+// serial path never waits for memory.
+constexpr int FJ = 64;                          // value columns per CTA (one CTA per SM at B=1, 48 heads)
+constexpr int FLDJ = FJ + 8;
+constexpr size_t FS_W = 0;                      // one ring stage
+constexpr size_t FS_K = FS_W + 64 * LDT * 2;
+constexpr size_t FS_UT = FS_K + 64 * LDT * 2;   // U~ block, 64 x FJ
+constexpr size_t FS_GB = FS_UT + 64 * FLDJ * 2; // gates: b, gamma, g (64 each)
+constexpr size_t FS_BYTES = FS_GB + 192 * 4;
+constexpr size_t F_S = 2 * FS_BYTES;            // S block, bf16, 128 x FJ ([d][j])
+constexpr size_t F_U = F_S + 128 * FLDJ * 2;    // diag(g) U block, bf16
+constexpr size_t F_BYTES = F_U + 64 * FLDJ * 2;
 
-__global__ void __launch_bounds__(kThreads, 2) fwd_chain_kernel(const Params p)
+constexpr int FNT = FJ / 8;                     // n tiles of the state block per warp
+
+__global__ void __launch_bounds__(kThreads, FJ == 32 ? 2 : 1) fwd_chain_kernel(const Params p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
-    bf16 *sW = reinterpret_cast<bf16 *>(smem + F_W), *sK = reinterpret_cast<bf16 *>(smem + F_K);
-    bf16 *sUt = reinterpret_cast<bf16 *>(smem + F_UT), *sS = reinterpret_cast<bf16 *>(smem + F_S);
-    bf16 *sU = reinterpret_cast<bf16 *>(smem + F_U);
-    float *sg = reinterpret_cast<float *>(smem + F_G);
+    bf16 *sS = reinterpret_cast<bf16 *>(smem + F_S), *sU = reinterpret_cast<bf16 *>(smem + F_U);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int j0 = JB * blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int j0 = FJ * blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int hq = h / (p.Hv / p.Hqk);
     const size_t qk_ld = (size_t)p.Hqk * D;
     const size_t ch0 = ((size_t)b * p.Hv + h) * p.NC;
-    float s[4][4];   // S rows 16 warp + (lane >> 2) (+8), columns 8 nt + 2 (lane & 3) (+1)
+    float s[FNT][4];   // S rows 16 warp + (lane >> 2) (+8), columns 8 nt + 2 (lane & 3) (+1)
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < FNT; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = 16 * warp + (lane >> 2) + 8 * (e >> 1), c = 8 * nt + 2 * (lane & 3) + (e & 1);
             s[nt][e] = p.S0 ? p.S0[((size_t)b * p.Hv + h) * D * D + (size_t)r * D + j0 + c] : 0.f;
         }
-    auto load_wu = [&](int n) {
-        load_tile<64, 16>(sW, LDT, p.ws.W + (ch0 + n) * 64 * D, D, 64, tid);
-        load_tile<64, 4>(sUt, LDJ, p.ws.U + (ch0 + n) * 64 * D + j0, D, 64, tid);
-    };
-    auto load_k = [&](int n) {
-        load_tile<64, 16>(sK, LDT, p.k + ((size_t)b * p.T + n * C) * qk_ld + (size_t)hq * D, qk_ld,
+    auto load = [&](int n) {
+        unsigned char *st = smem + (n & 1) * FS_BYTES;
+        load_tile<64, 16>(reinterpret_cast<bf16 *>(st + FS_W), LDT, p.ws.W + (ch0 + n) * 64 * D, D, 64, tid);
+        load_tile<64, 16>(reinterpret_cast<bf16 *>(st + FS_K), LDT,
+                          p.k + ((size_t)b * p.T + n * C) * qk_ld + (size_t)hq * D, qk_ld,
                           min(C, p.T - n * C), tid);
+        load_tile<64, FJ / 8>(reinterpret_cast<bf16 *>(st + FS_UT), FLDJ, p.ws.U + (ch0 + n) * 64 * D + j0, D,
+                              64, tid);
+        load_gate(reinterpret_cast<float *>(st + FS_GB), p.ws.gate + (ch0 + n) * 192, tid);
+        cp_commit();
     };
-    load_wu(0);
-    load_k(0);
-    cp_commit();
+    load(0);
+    if (p.NC > 1) load(1);
     for (int n = 0; n < p.NC; ++n) {
         const size_t ch = ch0 + n;
-        cp_wait_all();
-        if (tid < 64) {
-            const float *gb = p.ws.gb + ch * 64;
-            sg[tid] = expf(gb[63] - gb[tid]);
-        }
+        const unsigned char *st = smem + (n & 1) * FS_BYTES;
+        const bf16 *sW = reinterpret_cast<const bf16 *>(st + FS_W), *sK = reinterpret_cast<const bf16 *>(st + FS_K);
+        const bf16 *sUt = reinterpret_cast<const bf16 *>(st + FS_UT);
+        const float *sgb = reinterpret_cast<const float *>(st + FS_GB);
         // S at the chunk start -> bf16 tile and workspace
         bf16 *gS = p.ws.S + ch * D * D + j0;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < FNT; ++nt)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int r = 16 * warp + (lane >> 2) + 8 * hf, c = 8 * nt + 2 * (lane & 3);
                 const uint32_t v2 = pack2(s[nt][2 * hf], s[nt][2 * hf + 1]);
-                *reinterpret_cast<uint32_t *>(sS + r * LDJ + c) = v2;
+                *reinterpret_cast<uint32_t *>(sS + r * FLDJ + c) = v2;
                 *reinterpret_cast<uint32_t *>(gS + (size_t)r * D + c) = v2;
             }
-        __syncthreads();
-        const float glast = expf(p.ws.gb[ch * 64 + 63]);
-        // U = U~ - W S: 64 x 32, warp tile 16 x 16
+        if (n + 1 < p.NC) cp_wait<1>(); else cp_wait<0>();
+        __syncthreads();   // stage n landed; S tile complete
+        const float glast = sgb[64 + 63];
+        // U = U~ - W S: 64 x FJ, warp tile 16 x FJ/2
         {
-            const int m0 = 16 * (warp & 3), n0 = 16 * (warp >> 2);
-            float u[2][4];
+            const int m0 = 16 * (warp & 3), n0 = (FJ / 2) * (warp >> 2);
+            float u[FNT / 2][4];
             zero_acc(u);
-            warp_mma<0, 1, 2>(u, sW, LDT, sS, LDJ, m0, n0, D, lane);
+            warp_mma<0, 1, FNT / 2>(u, sW, LDT, sS, FLDJ, m0, n0, D, lane);
             bf16 *gU = p.ws.U + ch * 64 * D + j0;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < FNT / 2; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + (lane >> 2) + 8 * hf, c = n0 + 8 * nt + 2 * (lane & 3);
-                    const float2 ut = unpack2(sUt + r * LDJ + c);
+                    const float2 ut = unpack2(sUt + r * FLDJ + c);
                     const float u0 = ut.x - u[nt][2 * hf], u1 = ut.y - u[nt][2 * hf + 1];
+                    const float gr = sgb[128 + r];
                     *reinterpret_cast<uint32_t *>(gU + (size_t)r * D + c) = pack2(u0, u1);
-                    *reinterpret_cast<uint32_t *>(sU + r * LDJ + c) = pack2(sg[r] * u0, sg[r] * u1);
+                    *reinterpret_cast<uint32_t *>(sU + r * FLDJ + c) = pack2(gr * u0, gr * u1);
                 }
         }
-        __syncthreads();
-        if (n + 1 < p.NC) {
-            load_wu(n + 1);
-            cp_commit();
-        }
-        // S <- gamma_{C-1} S + K^T diag(g) U: 128 x 32, warp tile 16 x 32, K = 64
+        __syncthreads();   // diag(g) U complete
+        // S <- gamma_{C-1} S + K^T diag(g) U: 128 x FJ, warp tile 16 x FJ, K = 64
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+        for (int nt = 0; nt < FNT; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] *= glast;
-        warp_mma<1, 1, 4>(s, sK, LDT, sU, LDJ, 16 * warp, 0, C, lane);
-        __syncthreads();
-        if (n + 1 < p.NC) {
-            load_k(n + 1);
-            cp_commit();
-        }
+        warp_mma<1, 1, FNT>(s, sK, LDT, sU, FLDJ, 16 * warp, 0, C, lane);
+        __syncthreads();   // stage n, S tile and U tile no longer read
+        if (n + 2 < p.NC) load(n + 2);
     }
 }
 
 // ================================================================== 3. gradient chain
-// Per (32-column block jb, V head h, sequence b), chunks from the last: dS (128 x 32
-// fp32 accumulators) from dS_final; per chunk: dS' = dS -> workspace (bf16) and
-// sum(dS' o S) -> gC, dU = diag(g) K dS' + P^T dO -> workspace,
-// dS <- gamma_{C-1} dS' + Q^T diag(gamma) dO - W^T dU.  At the end dS0 = dS.
-constexpr size_t G_K = 0;
-constexpr size_t G_Q = G_K + 64 * LDT * 2;
-constexpr size_t G_W = G_Q + 64 * LDT * 2;
-constexpr size_t G_P = G_W + 64 * LDT * 2;      // P, 64 x 64
-constexpr size_t G_O = G_P + 64 * LDQ * 2;      // dO block, 64 x 32
-constexpr size_t G_OG = G_O + 64 * LDJ * 2;     // diag(gamma) dO block
-constexpr size_t G_D = G_OG + 64 * LDJ * 2;     // dS' block, bf16, 128 x 32
-constexpr size_t G_DU = G_D + 128 * LDJ * 2;    // -dU block, bf16
-constexpr size_t G_G = G_DU + 64 * LDJ * 2;     // g[64], gamma[64], partial sums[8]
-constexpr size_t G_BYTES = G_G + (64 + 64 + 8) * 4;
+// Per (64-column block jb, V head h, sequence b), chunks from the last: dS (128 x 64
+// fp32 accumulators, warp w rows 16w..16w+15) from dS_final; per chunk: dS' = dS ->
+// workspace (bf16), dU = diag(g) K dS' + P^T dO -> workspace, sum(dS' o S) -> gC,
+// dS <- gamma_{C-1} dS' + Q^T diag(gamma) dO - W^T dU.  At the end dS0 = dS.  A
+// two-stage ring holds each chunk's K, Q, W, P, dO block, start-state block and
+// decay, loaded one whole chunk ahead.
+constexpr int GJ = 64;                          // value columns per CTA
+constexpr int GLDJ = GJ + 8;
+constexpr int kGcSlots = D / GJ;                // partial sums of sum(dS' o S) per chunk
+constexpr size_t GS_K = 0;                      // one ring stage
+constexpr size_t GS_Q = GS_K + 64 * LDT * 2;
+constexpr size_t GS_W = GS_Q + 64 * LDT * 2;
+constexpr size_t GS_P = GS_W + 64 * LDT * 2;    // P, 64 x 64
+constexpr size_t GS_O = GS_P + 64 * LDQ * 2;    // dO block, 64 x 64
+constexpr size_t GS_SB = GS_O + 64 * GLDJ * 2;  // S block at the chunk start, 128 x 64
+constexpr size_t GS_GB = GS_SB + 128 * GLDJ * 2;
+constexpr size_t GS_BYTES = GS_GB + 192 * 4;
+constexpr size_t G_D = 2 * GS_BYTES;            // dS' block, bf16, 128 x 64
+constexpr size_t G_OG = G_D + 128 * GLDJ * 2;   // diag(gamma) dO block
+constexpr size_t G_DU = G_OG + 64 * GLDJ * 2;   // -dU block
+constexpr size_t G_PART = G_DU + 64 * GLDJ * 2; // partial sums[8]
+constexpr size_t G_BYTES = G_PART + 8 * 4;
 
-__global__ void __launch_bounds__(kThreads, 2) grad_chain_kernel(const Params p)
+__global__ void __launch_bounds__(kThreads, 1) grad_chain_kernel(const Params p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
-    bf16 *sK = reinterpret_cast<bf16 *>(smem + G_K), *sQ = reinterpret_cast<bf16 *>(smem + G_Q);
-    bf16 *sW = reinterpret_cast<bf16 *>(smem + G_W), *sP = reinterpret_cast<bf16 *>(smem + G_P);
-    bf16 *sO = reinterpret_cast<bf16 *>(smem + G_O), *sOg = reinterpret_cast<bf16 *>(smem + G_OG);
-    bf16 *sD = reinterpret_cast<bf16 *>(smem + G_D), *sdU = reinterpret_cast<bf16 *>(smem + G_DU);
-    float *sg = reinterpret_cast<float *>(smem + G_G), *sgam = sg + 64, *spart = sg + 128;
+    bf16 *sD = reinterpret_cast<bf16 *>(smem + G_D), *sOg = reinterpret_cast<bf16 *>(smem + G_OG);
+    bf16 *sdU = reinterpret_cast<bf16 *>(smem + G_DU);
+    float *spart = reinterpret_cast<float *>(smem + G_PART);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int jb = blockIdx.x, j0 = JB * jb, h = blockIdx.y, b = blockIdx.z;
+    const int jb = blockIdx.x, j0 = GJ * jb, h = blockIdx.y, b = blockIdx.z;
     const int hq = h / (p.Hv / p.Hqk);
     const size_t qk_ld = (size_t)p.Hqk * D, v_ld = (size_t)p.Hv * D;
     const size_t ch0 = ((size_t)b * p.Hv + h) * p.NC;
     const size_t hs = ((size_t)b * p.Hv + h) * D * D;
-    float ds[4][4];
+    float ds[8][4];   // rows 16 warp + (lane >> 2) (+8), columns 8 nt + 2 (lane & 3) (+1)
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = 16 * warp + (lane >> 2) + 8 * (e >> 1), c = 8 * nt + 2 * (lane & 3) + (e & 1);
             ds[nt][e] = p.dS_final ? p.dS_final[hs + (size_t)r * D + j0 + c] : 0.f;
         }
-    auto load_kpo = [&](int n) {
+    auto load = [&](int n) {
+        unsigned char *st = smem + (n & 1) * GS_BYTES;
         const int L = min(C, p.T - n * C);
         const size_t tok = (size_t)b * p.T + n * C;
-        load_tile<64, 16>(sK, LDT, p.k + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
-        load_tile<64, 8>(sP, LDQ, p.ws.P + (ch0 + n) * 64 * 64, 64, 64, tid);
-        load_tile<64, 4>(sO, LDJ, p.dO + tok * v_ld + (size_t)h * D + j0, v_ld, L, tid);
+        load_tile<64, 16>(reinterpret_cast<bf16 *>(st + GS_K), LDT, p.k + tok * qk_ld + (size_t)hq * D, qk_ld, L,
+                          tid);
+        load_tile<64, 16>(reinterpret_cast<bf16 *>(st + GS_Q), LDT, p.q + tok * qk_ld + (size_t)hq * D, qk_ld, L,
+                          tid);
+        load_tile<64, 16>(reinterpret_cast<bf16 *>(st + GS_W), LDT, p.ws.W + (ch0 + n) * 64 * D, D, 64, tid);
+        load_tile<64, 8>(reinterpret_cast<bf16 *>(st + GS_P), LDQ, p.ws.P + (ch0 + n) * 64 * 64, 64, 64, tid);
+        load_tile<64, 8>(reinterpret_cast<bf16 *>(st + GS_O), GLDJ, p.dO + tok * v_ld + (size_t)h * D + j0, v_ld,
+                         L, tid);
+        load_tile<128, 8>(reinterpret_cast<bf16 *>(st + GS_SB), GLDJ, p.ws.S + (ch0 + n) * D * D + j0, D, 128,
+                          tid);
+        load_gate(reinterpret_cast<float *>(st + GS_GB), p.ws.gate + (ch0 + n) * 192, tid);
+        cp_commit();
     };
-    auto load_qw = [&](int n) {
-        const int L = min(C, p.T - n * C);
-        const size_t tok = (size_t)b * p.T + n * C;
-        load_tile<64, 16>(sQ, LDT, p.q + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
-        load_tile<64, 16>(sW, LDT, p.ws.W + (ch0 + n) * 64 * D, D, 64, tid);
-    };
-    load_kpo(p.NC - 1);
-    load_qw(p.NC - 1);
-    cp_commit();
+    load(p.NC - 1);
+    if (p.NC > 1) load(p.NC - 2);
     for (int n = p.NC - 1; n >= 0; --n) {
         const size_t ch = ch0 + n;
-        cp_wait_all();
-        if (tid < 64) {
-            const float *gb = p.ws.gb + ch * 64;
-            sg[tid] = expf(gb[63] - gb[tid]);
-            sgam[tid] = expf(gb[tid]);
-        }
-        // dS' -> bf16 tile and workspace; sum(dS' o S) over this block
-        float gc = 0.f;
+        const unsigned char *st = smem + (n & 1) * GS_BYTES;
+        const bf16 *sK = reinterpret_cast<const bf16 *>(st + GS_K), *sQ = reinterpret_cast<const bf16 *>(st + GS_Q);
+        const bf16 *sW = reinterpret_cast<const bf16 *>(st + GS_W), *sP = reinterpret_cast<const bf16 *>(st + GS_P);
+        const bf16 *sO = reinterpret_cast<const bf16 *>(st + GS_O), *sSb = reinterpret_cast<const bf16 *>(st + GS_SB);
+        const float *sgb = reinterpret_cast<const float *>(st + GS_GB);
+        // dS' -> bf16 tile and workspace
         {
             bf16 *gD = p.ws.dSp + ch * D * D + j0;
-            const bf16 *gS = p.ws.S + ch * D * D + j0;
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = 16 * warp + (lane >> 2) + 8 * hf, c = 8 * nt + 2 * (lane & 3);
                     const uint32_t v2 = pack2(ds[nt][2 * hf], ds[nt][2 * hf + 1]);
-                    *reinterpret_cast<uint32_t *>(sD + r * LDJ + c) = v2;
+                    *reinterpret_cast<uint32_t *>(sD + r * GLDJ + c) = v2;
                     *reinterpret_cast<uint32_t *>(gD + (size_t)r * D + c) = v2;
-                    const float2 sv = unpack2(gS + (size_t)r * D + c);
-                    gc += ds[nt][2 * hf] * sv.x + ds[nt][2 * hf + 1] * sv.y;
                 }
         }
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) gc += __shfl_xor_sync(0xffffffffu, gc, o);
-        if (lane == 0) spart[warp] = gc;
-        __syncthreads();   // sg, sgam, sD, spart
-        if (tid == 0) {
-            float t = 0.f;
-            for (int w = 0; w < 8; ++w) t += spart[w];
-            p.ws.gC[ch * 4 + jb] = t;
-        }
-        for (int e = tid; e < 64 * 16; e += kThreads) {   // diag(gamma) dO
-            const int r = e >> 4, c2 = 2 * (e & 15);
-            const float2 o2 = unpack2(sO + r * LDJ + c2);
-            *reinterpret_cast<uint32_t *>(sOg + r * LDJ + c2) = pack2(sgam[r] * o2.x, sgam[r] * o2.y);
-        }
-        const float glast = expf(p.ws.gb[ch * 64 + 63]);
-        // dU = diag(g) K dS' + P^T dO: 64 x 32, warp tile 16 x 16
+        if (n >= 1) cp_wait<1>(); else cp_wait<0>();
+        __syncthreads();   // stage n landed; dS' tile complete
+        const float glast = sgb[64 + 63];
+        // dU = diag(g) K dS' + P^T dO: 64 x 64, warp tile 16 x 32
         {
-            const int m0 = 16 * (warp & 3), n0 = 16 * (warp >> 2);
-            float du[2][4];
+            const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+            float du[4][4];
             zero_acc(du);
-            warp_mma<0, 1, 2>(du, sK, LDT, sD, LDJ, m0, n0, D, lane);
+            warp_mma<0, 1, 4>(du, sK, LDT, sD, GLDJ, m0, n0, D, lane);
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) du[nt][e] *= sg[m0 + (lane >> 2) + 8 * (e >> 1)];
-            warp_mma<1, 1, 2>(du, sP, LDQ, sO, LDJ, m0, n0, C, lane);
+                for (int e = 0; e < 4; ++e) du[nt][e] *= sgb[128 + m0 + (lane >> 2) + 8 * (e >> 1)];
+            warp_mma<1, 1, 4>(du, sP, LDQ, sO, GLDJ, m0, n0, C, lane);
             bf16 *gdU = p.ws.dU + ch * 64 * D + j0;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + (lane >> 2) + 8 * hf, c = n0 + 8 * nt + 2 * (lane & 3);
                     const float a0 = du[nt][2 * hf], a1 = du[nt][2 * hf + 1];
                     *reinterpret_cast<uint32_t *>(gdU + (size_t)r * D + c) = pack2(a0, a1);
-                    *reinterpret_cast<uint32_t *>(sdU + r * LDJ + c) = pack2(-a0, -a1);
+                    *reinterpret_cast<uint32_t *>(sdU + r * GLDJ + c) = pack2(-a0, -a1);
                 }
         }
-        __syncthreads();   // sdU, sOg complete; sK, sP, sO free
-        if (n > 0) {
-            load_kpo(n - 1);
-            cp_commit();
+        for (int e = tid; e < 64 * (GJ / 2); e += kThreads) {   // diag(gamma) dO
+            const int r = e / (GJ / 2), c2 = 2 * (e % (GJ / 2));
+            const float2 o2 = unpack2(sO + r * GLDJ + c2);
+            const float ga = sgb[64 + r];
+            *reinterpret_cast<uint32_t *>(sOg + r * GLDJ + c2) = pack2(ga * o2.x, ga * o2.y);
         }
-        // dS <- gamma_{C-1} dS' + Q^T diag(gamma) dO - W^T dU: 128 x 32, K = 64
+        {   // sum(dS' o S) over this block
+            float gc = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int r = 16 * warp + (lane >> 2) + 8 * hf, c = 8 * nt + 2 * (lane & 3);
+                    const float2 sv = unpack2(sSb + r * GLDJ + c);
+                    gc += ds[nt][2 * hf] * sv.x + ds[nt][2 * hf + 1] * sv.y;
+                }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) gc += __shfl_xor_sync(0xffffffffu, gc, o);
+            if (lane == 0) spart[warp] = gc;
+        }
+        __syncthreads();   // -dU, diag(gamma) dO, partial sums complete
+        if (tid == 0) {
+            float t = 0.f;
+            for (int w = 0; w < 8; ++w) t += spart[w];
+            p.ws.gC[ch * kGcSlots + jb] = t;
+        }
+        // dS <- gamma_{C-1} dS' + Q^T diag(gamma) dO - W^T dU: 128 x 64, K = 64
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) ds[nt][e] *= glast;
-        warp_mma<1, 1, 4>(ds, sQ, LDT, sOg, LDJ, 16 * warp, 0, C, lane);
-        warp_mma<1, 1, 4>(ds, sW, LDT, sdU, LDJ, 16 * warp, 0, C, lane);
-        __syncthreads();   // sQ, sW, sOg, sdU free
-        if (n > 0) {
-            load_qw(n - 1);
-            cp_commit();
-        }
+        warp_mma<1, 1, 8>(ds, sQ, LDT, sOg, GLDJ, 16 * warp, 0, C, lane);
+        warp_mma<1, 1, 8>(ds, sW, LDT, sdU, GLDJ, 16 * warp, 0, C, lane);
+        __syncthreads();   // stage n and the dS', dO, dU tiles no longer read
+        if (n >= 2) load(n - 2);
     }
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             const int r = 16 * warp + (lane >> 2) + 8 * hf, c = 8 * nt + 2 * (lane & 3);
@@ -599,10 +667,40 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
     const size_t tok = (size_t)b * p.T + t0;
     const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2), n0p = 32 * (warp >> 2), wh = warp >> 2;
     const int g4 = lane >> 2, t4 = lane & 3;
+    // a head's tiles: V, dO, U, dU, S (freed after dT is formed) and T (freed after dA)
+    auto load_main = [&](int i) {
+        const int h = hq * grp + i;
+        const size_t ch = ((size_t)b * p.Hv + h) * p.NC + n;
+        load_tile<64, 16>(sV, LDT, p.v + tok * v_ld + (size_t)h * D, v_ld, L, tid);
+        load_tile<64, 16>(sO, LDT, p.dO + tok * v_ld + (size_t)h * D, v_ld, L, tid);
+        load_tile<64, 16>(sU, LDT, p.ws.U + ch * 64 * D, D, 64, tid);
+        load_tile<64, 16>(sdU, LDT, p.ws.dU + ch * 64 * D, D, 64, tid);
+        load_tile<128, 16>(sS, LDT, p.ws.S + ch * D * D, D, 128, tid);
+        cp_commit();
+    };
+    auto load_t = [&](int i) {
+        const size_t ch = ((size_t)b * p.Hv + hq * grp + i) * p.NC + n;
+        load_tile<64, 8>(sT, LDQ, p.ws.Tm + ch * 64 * 64, 64, 64, tid);
+        cp_commit();
+    };
+    float nb = 0.f, nbeta = 0.f, ngam = 0.f, ng = 0.f;   // the next head's gates (tid < 64)
+    auto fetch_gates = [&](int i) {
+        if (tid < 64) {
+            const int h = hq * grp + i;
+            const float *gv = p.ws.gate + (((size_t)b * p.Hv + h) * p.NC + n) * 192;
+            nb = gv[tid];
+            nbeta = tid < L ? p.beta[(tok + tid) * p.Hv + h] : 0.f;
+            ngam = gv[64 + tid];
+            ng = gv[128 + tid];
+        }
+    };
     load_tile<64, 16>(sQ, LDT, p.q + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
     load_tile<64, 16>(sK, LDT, p.k + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
     cp_commit();
-    cp_wait_all();
+    load_main(0);
+    load_t(0);
+    fetch_gates(0);
+    cp_wait<2>();
     __syncthreads();
     chunk_grams(sK, sQ, fKK, fQK, warp, lane);
     float dq[8][4], dk[8][4], x[8][4];
@@ -623,23 +721,15 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
     for (int i = 0; i < grp; ++i) {
         const int h = hq * grp + i;
         const size_t ch = ((size_t)b * p.Hv + h) * p.NC + n;
-        __syncthreads();   // grams written; the previous head's tiles and sums no longer read
-        load_tile<64, 16>(sV, LDT, p.v + tok * v_ld + (size_t)h * D, v_ld, L, tid);
-        load_tile<64, 16>(sO, LDT, p.dO + tok * v_ld + (size_t)h * D, v_ld, L, tid);
-        load_tile<64, 16>(sU, LDT, p.ws.U + ch * 64 * D, D, 64, tid);
-        load_tile<64, 16>(sdU, LDT, p.ws.dU + ch * 64 * D, D, 64, tid);
-        load_tile<128, 16>(sS, LDT, p.ws.S + ch * D * D, D, 128, tid);
-        load_tile<64, 8>(sT, LDQ, p.ws.Tm + ch * 64 * 64, 64, 64, tid);
-        cp_commit();
+        __syncthreads();   // grams written; the previous head's gates and sums no longer read
         if (tid < 64) {
-            const float bb = p.ws.gb[ch * 64 + tid];
-            vb[tid] = bb;
-            vbeta[tid] = tid < L ? p.beta[(tok + tid) * p.Hv + h] : 0.f;
-            vgam[tid] = expf(bb);
-            vg[tid] = expf(p.ws.gb[ch * 64 + 63] - bb);
+            vb[tid] = nb;
+            vbeta[tid] = nbeta;
+            vgam[tid] = ngam;
+            vg[tid] = ng;
         }
         cp_wait_all();
-        __syncthreads();
+        __syncthreads();   // this head's tiles (loaded during the previous head) and gates
         // X1 = dO S^T: dQ += diag(gamma) X1; dgamma partial = rowsum(Q o X1)
         zero_acc(x);
         warp_mma<0, 0, 8>(x, sO, LDT, sS, LDT, m0, n0, D, lane);
@@ -688,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int s = c + e;
-                        const float gam = s <= r ? expf(vb[r] - vb[s]) : 0.f;
+                        const float gam = s <= r ? __expf(vb[r] - vb[s]) : 0.f;
                         const float dpg = pp[nt][2 * hf + e] * gam;
                         o2[e] = dpg;
                         const float gg = dpg * fQK[r * LDF + s];
@@ -788,7 +878,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
                     *reinterpret_cast<uint32_t *>(sX2 + r * LDQ + c) = pack2(a0, a1);
                 }
         }
-        __syncthreads();   // dT complete
+        __syncthreads();   // dT complete; V, dO, U, dU, dS' no longer read
+        if (i + 1 < grp) load_main(i + 1);
         // Z = T^T dT -> X1
         {
             float z[4][4];
@@ -823,7 +914,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
                         float t3 = 0.f, gg = 0.f, mv = 0.f;
                         if (s < r) {
                             const float da = -a[nt][2 * hf + e];
-                            const float gam = expf(vb[r] - vb[s]);
+                            const float gam = __expf(vb[r] - vb[s]);
                             const float dgk = da * gam * fKK[r * LDF + s];
                             t3 = dgk;
                             gg = vbeta[r] * dgk;
@@ -849,14 +940,18 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
                     if (g4 == 0) cols[(1 * 4 + (warp & 3)) * 64 + n0p + 8 * nt + 2 * t4 + e] = v;
                 }
         }
-        __syncthreads();   // M complete; every row / column sum written
+        __syncthreads();   // M complete; every row / column sum written; T no longer read
+        if (i + 1 < grp) {
+            load_t(i + 1);
+            fetch_gates(i + 1);
+        }
         warp_mma<0, 1, 8>(dk, sX2, LDQ, sK, LDT, m0, n0, C, lane);   // dK += M K
         warp_mma<1, 1, 8>(dk, sX2, LDQ, sK, LDT, m0, n0, C, lane);   // dK += M^T K
         // gate gradients (warp 0, two rows per lane), then d log alpha by a reverse scan
         if (warp == 0) {
             float gc = 0.f;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) gc += p.ws.gC[ch * 4 + q];
+            for (int q = 0; q < kGcSlots; ++q) gc += p.ws.gC[ch * kGcSlots + q];
             float db[2], dbeta_v[2], gsum = 0.f;
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
@@ -909,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
 
 // Workspace layout: the arrays of Ws in order, each 256-byte aligned.
 struct WsLayout {
-    size_t W, U, Tm, P, S, dSp, dU, gb, gC, bytes;
+    size_t W, U, Tm, P, S, dSp, dU, gate, gC, bytes;
 };
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 WsLayout ws_layout(int B, int T, int Hv)
@@ -925,8 +1020,8 @@ WsLayout ws_layout(int B, int T, int Hv)
     l.S = take(nch * D * D * 2);
     l.dSp = take(nch * D * D * 2);
     l.dU = take(nch * 64 * D * 2);
-    l.gb = take(nch * 64 * 4);
-    l.gC = take(nch * 4 * 4);
+    l.gate = take(nch * 192 * 4);
+    l.gC = take(nch * kGcSlots * 4);
     l.bytes = o;
     return l;
 }
@@ -967,7 +1062,7 @@ cudaError_t launch_bwd_chunk(const BwdLaunch &L, cudaStream_t stream)
     p.ws = Ws{reinterpret_cast<bf16 *>(w + l.W), reinterpret_cast<bf16 *>(w + l.U),
               reinterpret_cast<bf16 *>(w + l.Tm), reinterpret_cast<bf16 *>(w + l.P),
               reinterpret_cast<bf16 *>(w + l.S), reinterpret_cast<bf16 *>(w + l.dSp),
-              reinterpret_cast<bf16 *>(w + l.dU), reinterpret_cast<float *>(w + l.gb),
+              reinterpret_cast<bf16 *>(w + l.dU), reinterpret_cast<float *>(w + l.gate),
               reinterpret_cast<float *>(w + l.gC)};
     p.B = L.B;
     p.T = L.T;
@@ -984,10 +1079,9 @@ cudaError_t launch_bwd_chunk(const BwdLaunch &L, cudaStream_t stream)
     if ((err = cudaFuncSetAttribute(grad_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K_BYTES)))
         return err;
     const dim3 per_chunk((unsigned)p.NC, (unsigned)L.Hqk, (unsigned)L.B);
-    const dim3 per_block((unsigned)(D / JB), (unsigned)L.Hv, (unsigned)L.B);
     prep_kernel<<<per_chunk, kThreads, P_BYTES, stream>>>(p);
-    fwd_chain_kernel<<<per_block, kThreads, F_BYTES, stream>>>(p);
-    grad_chain_kernel<<<per_block, kThreads, G_BYTES, stream>>>(p);
+    fwd_chain_kernel<<<dim3((unsigned)(D / FJ), (unsigned)L.Hv, (unsigned)L.B), kThreads, F_BYTES, stream>>>(p);
+    grad_chain_kernel<<<dim3((unsigned)(D / GJ), (unsigned)L.Hv, (unsigned)L.B), kThreads, G_BYTES, stream>>>(p);
     grad_chunk_kernel<<<per_chunk, kThreads, K_BYTES, stream>>>(p);
     return cudaGetLastError();
 }

@@ -257,10 +257,10 @@ def test_bwd_argument_checks(lib):
 
 def test_bwd_chunk_workspace_sizes(lib):
     # per (sequence, V head, chunk of 64): W, U, dU (64 x 128 bf16), T, P (64 x 64
-    # bf16), S, dS' (128 x 128 bf16), b (64 fp32) and four fp32 sums; each array
+    # bf16), S, dS' (128 x 128 bf16), b, gamma, g (64 fp32 each) and two fp32 sums; each array
     # 256-byte aligned
-    per = 3 * 64 * 128 * 2 + 2 * 64 * 64 * 2 + 2 * 128 * 128 * 2 + 64 * 4
-    assert binding.bwd_chunk_workspace_bytes(1, 4096, 48) == 48 * 64 * (per + 16)
+    per = 3 * 64 * 128 * 2 + 2 * 64 * 64 * 2 + 2 * 128 * 128 * 2 + 3 * 64 * 4
+    assert binding.bwd_chunk_workspace_bytes(1, 4096, 48) == 48 * 64 * (per + 8)
     assert binding.bwd_chunk_workspace_bytes(2, 17, 6) == 12 * per + 256
     assert binding.bwd_chunk_workspace_bytes(1, 0, 48) == 0
     assert lib.gdn_bwd_chunk_workspace(1, 64, 48, 64, 128) == 0
