@@ -186,81 +186,81 @@ __device__ __forceinline__ void chunk_grams(const bf16 *sK, const bf16 *sQ, floa
         }
 }
 
-// T = (I + A)^-1 for the strictly lower 64 x 64 A (fp32, row stride LDF), by 16 x 16
-// blocks: the diagonal blocks by forward substitution (one thread per column, the
-// column in registers), then block rows 1..3 in turn,
+// T = (I + A)^-1 for the strictly lower 64 x 64 A (fp32, row stride LDF), in place,
+// by 16 x 16 blocks: the diagonal blocks by forward substitution (one thread per
+// column, the column in registers until every thread has read its block of A),
+// then block rows 1..3 in turn,
 //   T_ij = -T_ii sum_{j <= k < i} A_ik T_kj   (j < i),
-// every element of a stage in parallel.  xs: 768 floats of scratch.  Upper blocks
-// are written as zeros.  Called by all threads; ends with the result visible.
-__device__ __forceinline__ void invert_unit_lower(const float *fA, float *fT, float *xs, int tid)
+// every element of a stage in parallel: block row i still holds A while its X_ij
+// are formed, and the rows above it already hold T.  The upper blocks of A are
+// zero, as T's are.  xs: 768 floats of scratch.  Called by all threads; ends with
+// the result visible.
+__device__ __forceinline__ void invert_unit_lower(float *fAT, float *xs, int tid)
 {
+    float t[16];
+    const int base = 16 * (tid >> 4), c = tid & 15;
     if (tid < 64) {
-        const int base = 16 * (tid >> 4), c = tid & 15;
-        float t[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
             float s = r == c ? 1.f : 0.f;
 #pragma unroll
-            for (int m = 0; m < r; ++m) s -= fA[(base + r) * LDF + base + m] * t[m];
+            for (int m = 0; m < r; ++m) s -= fAT[(base + r) * LDF + base + m] * t[m];
             t[r] = r < c ? 0.f : s;
         }
+    }
+    __syncthreads();   // every diagonal block of A read
+    if (tid < 64) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) fT[(base + r) * LDF + base + c] = t[r];
-    } else {
-        for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {   // blocks (i, j), i < j
-            const int blk = e >> 8, r = (e >> 4) & 15, c = e & 15;
-            const int i = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-            const int j = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-            fT[(16 * i + r) * LDF + 16 * j + c] = 0.f;
-        }
+        for (int r = 0; r < 16; ++r) fAT[(base + r) * LDF + base + c] = t[r];
     }
     __syncthreads();
     for (int i = 1; i < 4; ++i) {
         for (int e = tid; e < i * 256; e += kThreads) {
-            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
             float s = 0.f;
             for (int k = j; k < i; ++k)
 #pragma unroll
                 for (int m = 0; m < 16; ++m)
-                    s += fA[(16 * i + r) * LDF + 16 * k + m] * fT[(16 * k + m) * LDF + 16 * j + c];
+                    s += fAT[(16 * i + r) * LDF + 16 * k + m] * fAT[(16 * k + m) * LDF + 16 * j + cc];
             xs[e] = s;
         }
         __syncthreads();
         for (int e = tid; e < i * 256; e += kThreads) {
-            const int j = e >> 8, r = (e >> 4) & 15, c = e & 15;
+            const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
             float s = 0.f;
 #pragma unroll
-            for (int m = 0; m < 16; ++m) s += fT[(16 * i + r) * LDF + 16 * i + m] * xs[(j << 8) + (m << 4) + c];
-            fT[(16 * i + r) * LDF + 16 * j + c] = -s;
+            for (int m = 0; m < 16; ++m) s += fAT[(16 * i + r) * LDF + 16 * i + m] * xs[(j << 8) + (m << 4) + cc];
+            fAT[(16 * i + r) * LDF + 16 * j + cc] = -s;
         }
         __syncthreads();
     }
 }
 
 // ================================================================== 1. preparation
-// Per (chunk n, QK head hq, sequence b): grams once, then for each V head of the
-// group the decay b, the solve T = (I + A)^-1 (fp32, blocked: see invert_unit_lower),
-// W, U~, P; all to the workspace.
+// Per (chunk n, QK head hq, sequence b): grams once (K K^T fp32, Q K^T bf16), then
+// for each V head of the group the decay vectors, A, the solve T = (I + A)^-1 (fp32,
+// blocked, in place), P = Gam o Q K^T, and W = (T diag(beta gamma)) K,
+// U~ = (T diag(beta)) V with the gates folded into the columns of T; all to the
+// workspace.  111 KB of shared memory: two CTAs per SM.
 constexpr size_t P_K = 0;
 constexpr size_t P_Q = P_K + 64 * LDT * 2;
-constexpr size_t P_X = P_Q + 64 * LDT * 2;      // diag(beta gamma) K
-constexpr size_t P_V = P_X + 64 * LDT * 2;      // V, then diag(beta) V
-constexpr size_t P_T = P_V + 64 * LDT * 2;      // T, bf16
-constexpr size_t P_KK = P_T + 64 * LDQ * 2;
-constexpr size_t P_QK = P_KK + 64 * LDF * 4;
-constexpr size_t P_A = P_QK + 64 * LDF * 4;
-constexpr size_t P_TF = P_A + 64 * LDF * 4;     // T, fp32
-constexpr size_t P_G = P_TF + 64 * LDF * 4;     // b[64], beta[64], gamma[64]
+constexpr size_t P_V = P_Q + 64 * LDT * 2;
+constexpr size_t P_TW = P_V + 64 * LDT * 2;     // T diag(beta gamma), bf16 (the solve's scratch before)
+constexpr size_t P_TU = P_TW + 64 * LDQ * 2;    // T diag(beta), bf16
+constexpr size_t P_QK = P_TU + 64 * LDQ * 2;    // Q K^T, bf16
+constexpr size_t P_KK = P_QK + 64 * LDQ * 2;    // K K^T, fp32
+constexpr size_t P_AT = P_KK + 64 * LDF * 4;    // A, then T (fp32)
+constexpr size_t P_G = P_AT + 64 * LDF * 4;     // b[64], beta[64], gamma[64]
 constexpr size_t P_BYTES = P_G + 3 * 64 * 4;
 
-__global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
+__global__ void __launch_bounds__(kThreads, 2) prep_kernel(const Params p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     bf16 *sK = reinterpret_cast<bf16 *>(smem + P_K), *sQ = reinterpret_cast<bf16 *>(smem + P_Q);
-    bf16 *sX = reinterpret_cast<bf16 *>(smem + P_X), *sV = reinterpret_cast<bf16 *>(smem + P_V);
-    bf16 *sT = reinterpret_cast<bf16 *>(smem + P_T);
-    float *fKK = reinterpret_cast<float *>(smem + P_KK), *fQK = reinterpret_cast<float *>(smem + P_QK);
-    float *fA = reinterpret_cast<float *>(smem + P_A), *fT = reinterpret_cast<float *>(smem + P_TF);
+    bf16 *sV = reinterpret_cast<bf16 *>(smem + P_V);
+    bf16 *sTw = reinterpret_cast<bf16 *>(smem + P_TW), *sTu = reinterpret_cast<bf16 *>(smem + P_TU);
+    bf16 *sQK = reinterpret_cast<bf16 *>(smem + P_QK);
+    float *fKK = reinterpret_cast<float *>(smem + P_KK), *fAT = reinterpret_cast<float *>(smem + P_AT);
     float *sb = reinterpret_cast<float *>(smem + P_G), *sbeta = sb + 64, *sgam = sb + 128;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
@@ -270,15 +270,35 @@ __global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
     load_tile<64, 16>(sK, LDT, p.k + ((size_t)b * p.T + t0) * qk_ld + (size_t)hq * D, qk_ld, L, tid);
     load_tile<64, 16>(sQ, LDT, p.q + ((size_t)b * p.T + t0) * qk_ld + (size_t)hq * D, qk_ld, L, tid);
     cp_commit();
-    cp_wait_all();
+    load_tile<64, 16>(sV, LDT, p.v + ((size_t)b * p.T + t0) * v_ld + (size_t)(hq * grp) * D, v_ld, L, tid);
+    cp_commit();
+    cp_wait<1>();
     __syncthreads();
-    chunk_grams(sK, sQ, fKK, fQK, warp, lane);
+    {   // K K^T (fp32) and Q K^T (bf16): 64 x 64, warp tile 16 x 32
+        const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+        float kk[4][4], qk[4][4];
+        zero_acc(kk);
+        zero_acc(qk);
+        warp_mma<0, 0, 4>(kk, sK, LDT, sK, LDT, m0, n0, D, lane);
+        warp_mma<0, 0, 4>(qk, sQ, LDT, sK, LDT, m0, n0, D, lane);
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                const int r = m0 + (lane >> 2) + 8 * hf, c = n0 + 8 * nt + 2 * (lane & 3);
+                fKK[r * LDF + c] = kk[nt][2 * hf];
+                fKK[r * LDF + c + 1] = kk[nt][2 * hf + 1];
+                *reinterpret_cast<uint32_t *>(sQK + r * LDQ + c) = pack2(qk[nt][2 * hf], qk[nt][2 * hf + 1]);
+            }
+    }
     for (int i = 0; i < grp; ++i) {
         const int h = hq * grp + i;
         const size_t ch = ((size_t)b * p.Hv + h) * p.NC + n;
         __syncthreads();   // grams written; the previous head's tiles no longer read
-        load_tile<64, 16>(sV, LDT, p.v + ((size_t)b * p.T + t0) * v_ld + (size_t)h * D, v_ld, L, tid);
-        cp_commit();
+        if (i > 0) {
+            load_tile<64, 16>(sV, LDT, p.v + ((size_t)b * p.T + t0) * v_ld + (size_t)h * D, v_ld, L, tid);
+            cp_commit();
+        }
         if (warp == 0) {   // b = cumsum(log alpha), two rows per lane; padded rows add 0
             const float *al = p.alpha + ((size_t)b * p.T + t0) * p.Hv + h;
             const float *be = p.beta + ((size_t)b * p.T + t0) * p.Hv + h;
@@ -313,38 +333,36 @@ __global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
             bf16 *gP = p.ws.P + ch * 64 * 64;
             for (int e = tid; e < 64 * 32; e += kThreads) {
                 const int r = e >> 5, m2 = 2 * (e & 31);
+                const float2 qk2 = unpack2(sQK + r * LDQ + m2);
+                const float qkv[2] = {qk2.x, qk2.y};
                 float pv[2];
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
                     const int m = m2 + x;
                     const float gam = m <= r ? __expf(sb[r] - sb[m]) : 0.f;
-                    fA[r * LDF + m] = m < r ? sbeta[r] * gam * fKK[r * LDF + m] : 0.f;
-                    pv[x] = gam * fQK[r * LDF + m];
+                    fAT[r * LDF + m] = m < r ? sbeta[r] * gam * fKK[r * LDF + m] : 0.f;
+                    pv[x] = gam * qkv[x];
                 }
                 *reinterpret_cast<uint32_t *>(gP + r * 64 + m2) = pack2(pv[0], pv[1]);
             }
         }
         __syncthreads();
-        invert_unit_lower(fA, fT, reinterpret_cast<float *>(sX), tid);   // sX is free until below
+        invert_unit_lower(fAT, reinterpret_cast<float *>(sTw), tid);   // sTw is free until below
+        // T -> workspace (bf16); T diag(beta gamma), T diag(beta) -> tiles
+        {
+            bf16 *gT = p.ws.Tm + ch * 64 * 64;
+            for (int e = tid; e < 64 * 32; e += kThreads) {
+                const int r = e >> 5, c2 = 2 * (e & 31);
+                const float ta = fAT[r * LDF + c2], tb = fAT[r * LDF + c2 + 1];
+                *reinterpret_cast<uint32_t *>(gT + r * 64 + c2) = pack2(ta, tb);
+                *reinterpret_cast<uint32_t *>(sTw + r * LDQ + c2) =
+                    pack2(ta * sbeta[c2] * sgam[c2], tb * sbeta[c2 + 1] * sgam[c2 + 1]);
+                *reinterpret_cast<uint32_t *>(sTu + r * LDQ + c2) = pack2(ta * sbeta[c2], tb * sbeta[c2 + 1]);
+            }
+        }
         cp_wait_all();
-        __syncthreads();
-        // bf16 T (tile and workspace), diag(beta gamma) K, diag(beta) V
-        bf16 *gT = p.ws.Tm + ch * 64 * 64;
-        for (int e = tid; e < 64 * 32; e += kThreads) {
-            const int r = e >> 5, c2 = 2 * (e & 31);
-            const uint32_t t2 = pack2(fT[r * LDF + c2], fT[r * LDF + c2 + 1]);
-            *reinterpret_cast<uint32_t *>(sT + r * LDQ + c2) = t2;
-            *reinterpret_cast<uint32_t *>(gT + r * 64 + c2) = t2;
-        }
-        for (int e = tid; e < 64 * 64; e += kThreads) {
-            const int r = e >> 6, c2 = 2 * (e & 63);
-            const float bg = sbeta[r] * sgam[r], bt = sbeta[r];
-            const float2 kv = unpack2(sK + r * LDT + c2), vv = unpack2(sV + r * LDT + c2);
-            *reinterpret_cast<uint32_t *>(sX + r * LDT + c2) = pack2(bg * kv.x, bg * kv.y);
-            *reinterpret_cast<uint32_t *>(sV + r * LDT + c2) = pack2(bt * vv.x, bt * vv.y);
-        }
-        __syncthreads();
-        // W = T diag(beta gamma) K, U~ = T diag(beta) V: 64 x 128, K = 64
+        __syncthreads();   // V landed; the scaled T tiles complete
+        // W = (T diag(beta gamma)) K, U~ = (T diag(beta)) V: 64 x 128, K = 64
         {
             const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2);
             float acc[8][4];
@@ -352,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) prep_kernel(const Params p)
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
                 zero_acc(acc);
-                warp_mma<0, 1, 8>(acc, sT, LDQ, which ? sV : sX, LDT, m0, n0, C, lane);
+                warp_mma<0, 1, 8>(acc, which ? sTu : sTw, LDQ, which ? sV : sK, LDT, m0, n0, C, lane);
                 bf16 *dst = which ? gU : gW;
 #pragma unroll
                 for (int nt = 0; nt < 8; ++nt)
