@@ -95,12 +95,12 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
 // of a tile starts on a 16-byte boundary.
 // Fragment layout of acc[nt][e]: row m0 + (lane >> 2) + 8 (e >> 1), column
 // n0 + 8 nt + 2 (lane & 3) + (e & 1).
-template <int AL, int BL, int NT>
+template <int AL, int BL, int NT, int UNROLL = 8>
 __device__ __forceinline__ void warp_mma(float (&acc)[NT][4], const bf16 *A, int lda, const bf16 *Bm,
                                          int ldb, int m0, int n0, int K, int lane)
 {
     static_assert(NT % 2 == 0, "n tiles in pairs");
-#pragma unroll 8
+#pragma unroll UNROLL
     for (int k0 = 0; k0 < K; k0 += 16) {
         uint32_t a[4];
         if (AL == 0)
@@ -115,6 +115,41 @@ __device__ __forceinline__ void warp_mma(float (&acc)[NT][4], const bf16 *A, int
                 ldsm4(sa(Bm + (nb + (lane & 7) + 8 * (lane >> 4)) * ldb + k0 + 8 * ((lane >> 3) & 1)), bb);
             else
                 ldsm4t(sa(Bm + (k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ldb + nb + 8 * (lane >> 4)), bb);
+            mma16816(acc[nt], a, bb[0], bb[1]);
+            mma16816(acc[nt + 1], a, bb[2], bb[3]);
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float lo, float hi) {
+    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&v));
+    const __nv_bfloat162 h = __floats2bfloat162_rn(f.x * lo, f.y * hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// acc += (diag(ks) A)^T-side product: as warp_mma<1, 1, NT> (A stored [k][m], B stored
+// [k][n]) with every A element of index k scaled by ks[k] in the fragment (one bf16
+// rounding), so a per-k scale needs no scaled copy of a tile.
+template <int NT>
+__device__ __forceinline__ void warp_mma_kscaled(float (&acc)[NT][4], const bf16 *A, int lda, const float *ks,
+                                                 const bf16 *Bm, int ldb, int m0, int n0, int K, int lane)
+{
+    static_assert(NT % 2 == 0, "n tiles in pairs");
+    const int t2 = 2 * (lane & 3);
+#pragma unroll 8
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        uint32_t a[4];
+        ldsm4t(sa(A + (k0 + (lane & 7) + 8 * (lane >> 4)) * lda + m0 + 8 * ((lane >> 3) & 1)), a);
+        const float s0 = ks[k0 + t2], s1 = ks[k0 + t2 + 1], s2 = ks[k0 + 8 + t2], s3 = ks[k0 + 9 + t2];
+        a[0] = scale_bf16x2(a[0], s0, s1);
+        a[1] = scale_bf16x2(a[1], s0, s1);
+        a[2] = scale_bf16x2(a[2], s2, s3);
+        a[3] = scale_bf16x2(a[3], s2, s3);
+#pragma unroll
+        for (int nt = 0; nt < NT; nt += 2) {
+            uint32_t bb[4];
+            const int nb = n0 + 8 * nt;
+            ldsm4t(sa(Bm + (k0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ldb + nb + 8 * (lane >> 4)), bb);
             mma16816(acc[nt], a, bb[0], bb[1]);
             mma16816(acc[nt + 1], a, bb[2], bb[3]);
         }
@@ -149,12 +184,12 @@ __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0
 
 // ROWS x (8 NCH) bf16 from src (row r at src + r * src_ld) into dst (row stride ld);
 // rows >= valid_rows are zero-filled without being read.
-template <int ROWS, int NCH>
+template <int ROWS, int NCH, int NTHR = kThreads>
 __device__ __forceinline__ void load_tile(bf16 *dst, int ld, const bf16 *src, size_t src_ld, int valid_rows,
                                           int tid)
 {
 #pragma unroll 4
-    for (int e = tid; e < ROWS * NCH; e += kThreads) {
+    for (int e = tid; e < ROWS * NCH; e += NTHR) {
         const int r = e / NCH, c = e % NCH;
         const bool ok = r < valid_rows;
         cp16(dst + r * ld + 8 * c, src + (size_t)(ok ? r : 0) * src_ld + 8 * c, ok);
@@ -166,18 +201,24 @@ __device__ __forceinline__ void load_gate(float *dst, const float *src, int tid)
     if (tid < 48) cp16(dst + 4 * tid, src + 4 * tid, true);
 }
 
-// K K^T and Q K^T of one chunk (64 x 64, fp32) from the bf16 tiles; 8 warps.
+// K K^T and Q K^T of one chunk (64 x 64, fp32) from the bf16 tiles, in the warp
+// tiling of grad_chunk_kernel (K3W warps, warp tile 16 x 64 / (K3W / 4)).
+constexpr int K3W = 16;                  // warps of grad_chunk_kernel
+constexpr int K3T = 32 * K3W;
+constexpr int K3H = K3W / 4;             // warps sharing a 16-row block
+constexpr int NTA = 128 / K3H / 8;       // n tiles of a 64 x 128 product per warp
+constexpr int NTB = 64 / K3H / 8;        // n tiles of a 64 x 64 product per warp
 __device__ __forceinline__ void chunk_grams(const bf16 *sK, const bf16 *sQ, float *fKK, float *fQK, int warp,
                                             int lane)
 {
-    const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-    float kk[4][4], qk[4][4];
+    const int m0 = 16 * (warp & 3), n0 = 8 * NTB * (warp >> 2);
+    float kk[NTB][4], qk[NTB][4];
     zero_acc(kk);
     zero_acc(qk);
-    warp_mma<0, 0, 4>(kk, sK, LDT, sK, LDT, m0, n0, D, lane);
-    warp_mma<0, 0, 4>(qk, sQ, LDT, sK, LDT, m0, n0, D, lane);
+    warp_mma<0, 0, NTB>(kk, sK, LDT, sK, LDT, m0, n0, D, lane);
+    warp_mma<0, 0, NTB>(qk, sQ, LDT, sK, LDT, m0, n0, D, lane);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < NTB; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int r = m0 + (lane >> 2) + 8 * (e >> 1), s = n0 + 8 * nt + 2 * (lane & 3) + (e & 1);
@@ -503,15 +544,14 @@ constexpr size_t GS_SB = GS_O + 64 * GLDJ * 2;  // S block at the chunk start, 1
 constexpr size_t GS_GB = GS_SB + 128 * GLDJ * 2;
 constexpr size_t GS_BYTES = GS_GB + 192 * 4;
 constexpr size_t G_D = 2 * GS_BYTES;            // dS' block, bf16, 128 x 64
-constexpr size_t G_OG = G_D + 128 * GLDJ * 2;   // diag(gamma) dO block
-constexpr size_t G_DU = G_OG + 64 * GLDJ * 2;   // -dU block
+constexpr size_t G_DU = G_D + 128 * GLDJ * 2;   // -dU block
 constexpr size_t G_PART = G_DU + 64 * GLDJ * 2; // partial sums[8]
 constexpr size_t G_BYTES = G_PART + 8 * 4;
 
 __global__ void __launch_bounds__(kThreads, 1) grad_chain_kernel(const Params p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
-    bf16 *sD = reinterpret_cast<bf16 *>(smem + G_D), *sOg = reinterpret_cast<bf16 *>(smem + G_OG);
+    bf16 *sD = reinterpret_cast<bf16 *>(smem + G_D);
     bf16 *sdU = reinterpret_cast<bf16 *>(smem + G_DU);
     float *spart = reinterpret_cast<float *>(smem + G_PART);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -569,35 +609,6 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chain_kernel(const Params p)
         }
         if (n >= 1) cp_wait<1>(); else cp_wait<0>();
         __syncthreads();   // stage n landed; dS' tile complete
-        const float glast = sgb[64 + 63];
-        // dU = diag(g) K dS' + P^T dO: 64 x 64, warp tile 16 x 32
-        {
-            const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
-            float du[4][4];
-            zero_acc(du);
-            warp_mma<0, 1, 4>(du, sK, LDT, sD, GLDJ, m0, n0, D, lane);
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) du[nt][e] *= sgb[128 + m0 + (lane >> 2) + 8 * (e >> 1)];
-            warp_mma<1, 1, 4>(du, sP, LDQ, sO, GLDJ, m0, n0, C, lane);
-            bf16 *gdU = p.ws.dU + ch * 64 * D + j0;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int r = m0 + (lane >> 2) + 8 * hf, c = n0 + 8 * nt + 2 * (lane & 3);
-                    const float a0 = du[nt][2 * hf], a1 = du[nt][2 * hf + 1];
-                    *reinterpret_cast<uint32_t *>(gdU + (size_t)r * D + c) = pack2(a0, a1);
-                    *reinterpret_cast<uint32_t *>(sdU + r * GLDJ + c) = pack2(-a0, -a1);
-                }
-        }
-        for (int e = tid; e < 64 * (GJ / 2); e += kThreads) {   // diag(gamma) dO
-            const int r = e / (GJ / 2), c2 = 2 * (e % (GJ / 2));
-            const float2 o2 = unpack2(sO + r * GLDJ + c2);
-            const float ga = sgb[64 + r];
-            *reinterpret_cast<uint32_t *>(sOg + r * GLDJ + c2) = pack2(ga * o2.x, ga * o2.y);
-        }
         {   // sum(dS' o S) over this block
             float gc = 0.f;
 #pragma unroll
@@ -612,18 +623,42 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chain_kernel(const Params p)
             for (int o = 16; o >= 1; o >>= 1) gc += __shfl_xor_sync(0xffffffffu, gc, o);
             if (lane == 0) spart[warp] = gc;
         }
-        __syncthreads();   // -dU, diag(gamma) dO, partial sums complete
+        // dS <- gamma_{C-1} dS' + (diag(gamma) Q)^T dO (the part that does not wait for
+        // dU); dU = diag(g) K dS' + P^T dO: 64 x 64, warp tile 16 x 32.  The three
+        // products are independent and overlap in the MMA pipe.
+        const float glast = sgb[64 + 63];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ds[nt][e] *= glast;
+        warp_mma_kscaled<8>(ds, sQ, LDT, sgb + 64, sO, GLDJ, 16 * warp, 0, C, lane);
+        {
+            const int m0 = 16 * (warp & 3), n0 = 32 * (warp >> 2);
+            float du[4][4], pd[4][4];
+            zero_acc(du);
+            zero_acc(pd);
+            warp_mma<0, 1, 4>(du, sK, LDT, sD, GLDJ, m0, n0, D, lane);
+            warp_mma<1, 1, 4>(pd, sP, LDQ, sO, GLDJ, m0, n0, C, lane);
+            bf16 *gdU = p.ws.dU + ch * 64 * D + j0;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int r = m0 + (lane >> 2) + 8 * hf, c = n0 + 8 * nt + 2 * (lane & 3);
+                    const float gr = sgb[128 + r];
+                    const float a0 = gr * du[nt][2 * hf] + pd[nt][2 * hf];
+                    const float a1 = gr * du[nt][2 * hf + 1] + pd[nt][2 * hf + 1];
+                    *reinterpret_cast<uint32_t *>(gdU + (size_t)r * D + c) = pack2(a0, a1);
+                    *reinterpret_cast<uint32_t *>(sdU + r * GLDJ + c) = pack2(-a0, -a1);
+                }
+        }
+        __syncthreads();   // -dU and the partial sums complete
         if (tid == 0) {
             float t = 0.f;
             for (int w = 0; w < 8; ++w) t += spart[w];
             p.ws.gC[ch * kGcSlots + jb] = t;
         }
-        // dS <- gamma_{C-1} dS' + Q^T diag(gamma) dO - W^T dU: 128 x 64, K = 64
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ds[nt][e] *= glast;
-        warp_mma<1, 1, 8>(ds, sQ, LDT, sOg, GLDJ, 16 * warp, 0, C, lane);
+        // dS -= W^T dU: 128 x 64, K = 64
         warp_mma<1, 1, 8>(ds, sW, LDT, sdU, GLDJ, 16 * warp, 0, C, lane);
         __syncthreads();   // stage n and the dS', dO, dU tiles no longer read
         if (n >= 2) load(n - 2);
@@ -639,11 +674,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chain_kernel(const Params p)
 }
 
 // ================================================================== 4. chunk gradients
-// Per (chunk n, QK head hq, sequence b).  Warp tiles: 64 x 128 outputs 16 x 64
-// (rows 16 (w & 3), columns 64 (w >> 2)); 64 x 64 outputs 16 x 32.  Row sums of a
-// 64 x 128 or 64 x 64 product come from two warps, column sums of a 64 x 64 one
-// from four: each writes its own slot ([2][64] / [4][64]) and the slots are added
-// in a fixed order.
+// Per (chunk n, QK head hq, sequence b), K3W = 16 warps.  Warp tiles: 64 x 128
+// outputs 16 x 32 (rows 16 (w & 3), columns 32 (w >> 2)); 64 x 64 outputs 16 x 16.
+// Row sums of a product come from the K3H = 4 warps of a row block, column sums of
+// a 64 x 64 one from four: each writes its own slot ([4][64]) and the slots are
+// added in a fixed order.
 constexpr size_t K_Q = 0;
 constexpr size_t K_K = K_Q + 64 * LDT * 2;
 constexpr size_t K_V = K_K + 64 * LDT * 2;
@@ -658,13 +693,15 @@ constexpr size_t K_X2 = K_X1 + 64 * LDQ * 2;    // dT, then M
 constexpr size_t K_KK = K_X2 + 64 * LDQ * 2;
 constexpr size_t K_QK = K_KK + 64 * LDF * 4;
 constexpr size_t K_VEC = K_QK + 64 * LDF * 4;   // b, beta, gamma, g (64 each)
-constexpr int NROW = 7;                         // row-sum arrays, [2][64] each
+constexpr int NROW = 7;                         // row-sum arrays, [K3H][64] each
 constexpr size_t K_ROW = K_VEC + 4 * 64 * 4;
-constexpr size_t K_COL = K_ROW + NROW * 2 * 64 * 4;   // two column-sum arrays, [4][64] each
+constexpr size_t K_COL = K_ROW + NROW * K3H * 64 * 4;   // two column-sum arrays, [4][64] each
 constexpr size_t K_BYTES = K_COL + 2 * 4 * 64 * 4;
 enum { R_DGAM = 0, R_DBG, R_DB2, R_DG, R_GGP, R_GGA, R_DB3 };
 
-__global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
+constexpr int K3U = 4;                          // k-loop unroll of its MMAs (registers)
+
+__global__ void __launch_bounds__(K3T, 1) grad_chunk_kernel(const Params p)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     bf16 *sQ = reinterpret_cast<bf16 *>(smem + K_Q), *sK = reinterpret_cast<bf16 *>(smem + K_K);
@@ -675,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
     bf16 *sX1 = reinterpret_cast<bf16 *>(smem + K_X1), *sX2 = reinterpret_cast<bf16 *>(smem + K_X2);
     float *fKK = reinterpret_cast<float *>(smem + K_KK), *fQK = reinterpret_cast<float *>(smem + K_QK);
     float *vb = reinterpret_cast<float *>(smem + K_VEC), *vbeta = vb + 64, *vgam = vb + 128, *vg = vb + 192;
-    float *rows = reinterpret_cast<float *>(smem + K_ROW);   // [NROW][2][64]
+    float *rows = reinterpret_cast<float *>(smem + K_ROW);   // [NROW][K3H][64]
     float *cols = reinterpret_cast<float *>(smem + K_COL);   // [2][4][64]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n = blockIdx.x, hq = blockIdx.y, b = blockIdx.z;
@@ -683,22 +720,22 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
     const int t0 = n * C, L = min(C, p.T - t0);
     const size_t qk_ld = (size_t)p.Hqk * D, v_ld = (size_t)p.Hv * D;
     const size_t tok = (size_t)b * p.T + t0;
-    const int m0 = 16 * (warp & 3), n0 = 64 * (warp >> 2), n0p = 32 * (warp >> 2), wh = warp >> 2;
+    const int m0 = 16 * (warp & 3), n0 = 8 * NTA * (warp >> 2), n0p = 8 * NTB * (warp >> 2), wh = warp >> 2;
     const int g4 = lane >> 2, t4 = lane & 3;
     // a head's tiles: V, dO, U, dU, S (freed after dT is formed) and T (freed after dA)
     auto load_main = [&](int i) {
         const int h = hq * grp + i;
         const size_t ch = ((size_t)b * p.Hv + h) * p.NC + n;
-        load_tile<64, 16>(sV, LDT, p.v + tok * v_ld + (size_t)h * D, v_ld, L, tid);
-        load_tile<64, 16>(sO, LDT, p.dO + tok * v_ld + (size_t)h * D, v_ld, L, tid);
-        load_tile<64, 16>(sU, LDT, p.ws.U + ch * 64 * D, D, 64, tid);
-        load_tile<64, 16>(sdU, LDT, p.ws.dU + ch * 64 * D, D, 64, tid);
-        load_tile<128, 16>(sS, LDT, p.ws.S + ch * D * D, D, 128, tid);
+        load_tile<64, 16, K3T>(sV, LDT, p.v + tok * v_ld + (size_t)h * D, v_ld, L, tid);
+        load_tile<64, 16, K3T>(sO, LDT, p.dO + tok * v_ld + (size_t)h * D, v_ld, L, tid);
+        load_tile<64, 16, K3T>(sU, LDT, p.ws.U + ch * 64 * D, D, 64, tid);
+        load_tile<64, 16, K3T>(sdU, LDT, p.ws.dU + ch * 64 * D, D, 64, tid);
+        load_tile<128, 16, K3T>(sS, LDT, p.ws.S + ch * D * D, D, 128, tid);
         cp_commit();
     };
     auto load_t = [&](int i) {
         const size_t ch = ((size_t)b * p.Hv + hq * grp + i) * p.NC + n;
-        load_tile<64, 8>(sT, LDQ, p.ws.Tm + ch * 64 * 64, 64, 64, tid);
+        load_tile<64, 8, K3T>(sT, LDQ, p.ws.Tm + ch * 64 * 64, 64, 64, tid);
         cp_commit();
     };
     float nb = 0.f, nbeta = 0.f, ngam = 0.f, ng = 0.f;   // the next head's gates (tid < 64)
@@ -712,8 +749,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
             ng = gv[128 + tid];
         }
     };
-    load_tile<64, 16>(sQ, LDT, p.q + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
-    load_tile<64, 16>(sK, LDT, p.k + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
+    load_tile<64, 16, K3T>(sQ, LDT, p.q + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
+    load_tile<64, 16, K3T>(sK, LDT, p.k + tok * qk_ld + (size_t)hq * D, qk_ld, L, tid);
     cp_commit();
     load_main(0);
     load_t(0);
@@ -721,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
     cp_wait<2>();
     __syncthreads();
     chunk_grams(sK, sQ, fKK, fQK, warp, lane);
-    float dq[8][4], dk[8][4], x[8][4];
+    float dq[NTA][4], dk[NTA][4], x[NTA][4];
     zero_acc(dq);
     zero_acc(dk);
     // row partial of a 64 x 128 / 64 x 64 fragment: v[hf] for rows m0 + g4 + 8 hf
@@ -731,11 +768,16 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
         v1 += __shfl_xor_sync(0xffffffffu, v1, 2);
         if (t4 == 0) {
-            rows[(which * 2 + wh) * 64 + m0 + g4] = v0;
-            rows[(which * 2 + wh) * 64 + m0 + g4 + 8] = v1;
+            rows[(which * K3H + wh) * 64 + m0 + g4] = v0;
+            rows[(which * K3H + wh) * 64 + m0 + g4 + 8] = v1;
         }
     };
-    auto row_sum = [&](int which, int r) { return rows[(which * 2) * 64 + r] + rows[(which * 2 + 1) * 64 + r]; };
+    auto row_sum = [&](int which, int r) {
+        float t = 0.f;
+#pragma unroll
+        for (int q = 0; q < K3H; ++q) t += rows[(which * K3H + q) * 64 + r];
+        return t;
+    };
     for (int i = 0; i < grp; ++i) {
         const int h = hq * grp + i;
         const size_t ch = ((size_t)b * p.Hv + h) * p.NC + n;
@@ -750,11 +792,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         __syncthreads();   // this head's tiles (loaded during the previous head) and gates
         // X1 = dO S^T: dQ += diag(gamma) X1; dgamma partial = rowsum(Q o X1)
         zero_acc(x);
-        warp_mma<0, 0, 8>(x, sO, LDT, sS, LDT, m0, n0, D, lane);
+        warp_mma<0, 0, NTA, K3U>(x, sO, LDT, sS, LDT, m0, n0, D, lane);
         {
             float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int nt = 0; nt < NTA; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + g4 + 8 * hf, c = n0 + 8 * nt + 2 * t4;
@@ -769,25 +811,25 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         }
         // X2 = dU S^T, dW = -X2 (bf16 tile)
         zero_acc(x);
-        warp_mma<0, 0, 8>(x, sdU, LDT, sS, LDT, m0, n0, D, lane);
+        warp_mma<0, 0, NTA, K3U>(x, sdU, LDT, sS, LDT, m0, n0, D, lane);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < NTA; ++nt)
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 const int r = m0 + g4 + 8 * hf, c = n0 + 8 * nt + 2 * t4;
                 *reinterpret_cast<uint32_t *>(sdW + r * LDT + c) = pack2(-x[nt][2 * hf], -x[nt][2 * hf + 1]);
             }
         __syncthreads();   // S no longer read; dW complete
-        load_tile<128, 16>(sS, LDT, p.ws.dSp + ch * D * D, D, 128, tid);   // dS' (waited below)
+        load_tile<128, 16, K3T>(sS, LDT, p.ws.dSp + ch * D * D, D, 128, tid);   // dS' (waited below)
         cp_commit();
         // dP = dO U^T (64 x 64); dP o Gam -> X1; Gam-weighted dP o QK row / column sums
         {
-            float pp[4][4];
+            float pp[NTB][4];
             zero_acc(pp);
-            warp_mma<0, 0, 4>(pp, sO, LDT, sU, LDT, m0, n0p, D, lane);
-            float r0 = 0.f, r1 = 0.f, cs[4][2];
+            warp_mma<0, 0, NTB, K3U>(pp, sO, LDT, sU, LDT, m0, n0p, D, lane);
+            float r0 = 0.f, r1 = 0.f, cs[NTB][2];
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+            for (int nt = 0; nt < NTB; ++nt) {
                 cs[nt][0] = cs[nt][1] = 0.f;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -808,7 +850,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
             }
             put_rows(R_GGP, r0, r1);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < NTB; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float v = cs[nt][e];
@@ -819,15 +861,15 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
                 }
         }
         __syncthreads();   // X1 = dP o Gam complete
-        warp_mma<0, 1, 8>(dq, sX1, LDQ, sK, LDT, m0, n0, C, lane);   // dQ += (dP o Gam) K
-        warp_mma<1, 1, 8>(dk, sX1, LDQ, sQ, LDT, m0, n0, C, lane);   // dK += (dP o Gam)^T Q
+        warp_mma<0, 1, NTA, K3U>(dq, sX1, LDQ, sK, LDT, m0, n0, C, lane);   // dQ += (dP o Gam) K
+        warp_mma<1, 1, NTA, K3U>(dk, sX1, LDQ, sQ, LDT, m0, n0, C, lane);   // dK += (dP o Gam)^T Q
         // T^T dW: dK += diag(beta gamma) T^T dW; dbg partial = rowsum(T^T dW o K)
         zero_acc(x);
-        warp_mma<1, 1, 8>(x, sT, LDQ, sdW, LDT, m0, n0, C, lane);
+        warp_mma<1, 1, NTA, K3U>(x, sT, LDQ, sdW, LDT, m0, n0, C, lane);
         {
             float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int nt = 0; nt < NTA; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + g4 + 8 * hf, c = n0 + 8 * nt + 2 * t4;
@@ -842,11 +884,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         }
         // T^T dU: dV = diag(beta) T^T dU; rowsum(T^T dU o V)
         zero_acc(x);
-        warp_mma<1, 1, 8>(x, sT, LDQ, sdU, LDT, m0, n0, C, lane);
+        warp_mma<1, 1, NTA, K3U>(x, sT, LDQ, sdU, LDT, m0, n0, C, lane);
         {
             float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int nt = 0; nt < NTA; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + g4 + 8 * hf, c = n0 + 8 * nt + 2 * t4;
@@ -863,11 +905,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         __syncthreads();   // dS' landed; X1 free
         // X3 = U dS'^T: dK += diag(g) X3; dg partial = rowsum(K o X3)
         zero_acc(x);
-        warp_mma<0, 0, 8>(x, sU, LDT, sS, LDT, m0, n0, D, lane);
+        warp_mma<0, 0, NTA, K3U>(x, sU, LDT, sS, LDT, m0, n0, D, lane);
         {
             float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+            for (int nt = 0; nt < NTA; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + g4 + 8 * hf, c = n0 + 8 * nt + 2 * t4;
@@ -881,13 +923,13 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         }
         // dT[r][m] = beta_m gamma_m (dW K^T)[r][m] + beta_m (dU V^T)[r][m] -> X2
         {
-            float y1[4][4], y2[4][4];
+            float y1[NTB][4], y2[NTB][4];
             zero_acc(y1);
             zero_acc(y2);
-            warp_mma<0, 0, 4>(y1, sdW, LDT, sK, LDT, m0, n0p, D, lane);
-            warp_mma<0, 0, 4>(y2, sdU, LDT, sV, LDT, m0, n0p, D, lane);
+            warp_mma<0, 0, NTB, K3U>(y1, sdW, LDT, sK, LDT, m0, n0p, D, lane);
+            warp_mma<0, 0, NTB, K3U>(y2, sdU, LDT, sV, LDT, m0, n0p, D, lane);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < NTB; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + g4 + 8 * hf, c = n0p + 8 * nt + 2 * t4;
@@ -900,11 +942,11 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         if (i + 1 < grp) load_main(i + 1);
         // Z = T^T dT -> X1
         {
-            float z[4][4];
+            float z[NTB][4];
             zero_acc(z);
-            warp_mma<1, 1, 4>(z, sT, LDQ, sX2, LDQ, m0, n0p, C, lane);
+            warp_mma<1, 1, NTB, K3U>(z, sT, LDQ, sX2, LDQ, m0, n0p, C, lane);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < NTB; ++nt)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     const int r = m0 + g4 + 8 * hf, c = n0p + 8 * nt + 2 * t4;
@@ -915,12 +957,12 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
         // dA = -Z T^T (strictly lower): dbeta term rowsum(dA o Gam o KK), Gam-weighted
         // dA o beta KK row / column sums, M = diag(beta) (dA o Gam) -> X2
         {
-            float a[4][4];
+            float a[NTB][4];
             zero_acc(a);
-            warp_mma<0, 0, 4>(a, sX1, LDQ, sT, LDQ, m0, n0p, C, lane);
-            float r0 = 0.f, r1 = 0.f, q0 = 0.f, q1 = 0.f, cs[4][2];
+            warp_mma<0, 0, NTB, K3U>(a, sX1, LDQ, sT, LDQ, m0, n0p, C, lane);
+            float r0 = 0.f, r1 = 0.f, q0 = 0.f, q1 = 0.f, cs[NTB][2];
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
+            for (int nt = 0; nt < NTB; ++nt) {
                 cs[nt][0] = cs[nt][1] = 0.f;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -948,7 +990,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
             put_rows(R_DB3, r0, r1);
             put_rows(R_GGA, q0, q1);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < NTB; ++nt)
 #pragma unroll
                 for (int e = 0; e < 2; ++e) {
                     float v = cs[nt][e];
@@ -963,8 +1005,8 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
             load_t(i + 1);
             fetch_gates(i + 1);
         }
-        warp_mma<0, 1, 8>(dk, sX2, LDQ, sK, LDT, m0, n0, C, lane);   // dK += M K
-        warp_mma<1, 1, 8>(dk, sX2, LDQ, sK, LDT, m0, n0, C, lane);   // dK += M^T K
+        warp_mma<0, 1, NTA, K3U>(dk, sX2, LDQ, sK, LDT, m0, n0, C, lane);   // dK += M K
+        warp_mma<1, 1, NTA, K3U>(dk, sX2, LDQ, sK, LDT, m0, n0, C, lane);   // dK += M^T K
         // gate gradients (warp 0, two rows per lane), then d log alpha by a reverse scan
         if (warp == 0) {
             float gc = 0.f;
@@ -1008,7 +1050,7 @@ __global__ void __launch_bounds__(kThreads, 1) grad_chunk_kernel(const Params p)
     }
     // dq, dk rows of this chunk (every V head of the group summed)
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < NTA; ++nt)
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
             const int r = m0 + g4 + 8 * hf, c = n0 + 8 * nt + 2 * t4;
@@ -1100,7 +1142,7 @@ cudaError_t launch_bwd_chunk(const BwdLaunch &L, cudaStream_t stream)
     prep_kernel<<<per_chunk, kThreads, P_BYTES, stream>>>(p);
     fwd_chain_kernel<<<dim3((unsigned)(D / FJ), (unsigned)L.Hv, (unsigned)L.B), kThreads, F_BYTES, stream>>>(p);
     grad_chain_kernel<<<dim3((unsigned)(D / GJ), (unsigned)L.Hv, (unsigned)L.B), kThreads, G_BYTES, stream>>>(p);
-    grad_chunk_kernel<<<per_chunk, kThreads, K_BYTES, stream>>>(p);
+    grad_chunk_kernel<<<per_chunk, K3T, K_BYTES, stream>>>(p);
     return cudaGetLastError();
 }
 
