@@ -64,12 +64,12 @@ def bwd_flops_per_token(w):
 
 def bwd_chunk_flops_per_token(w, C=64):
     """Algorithmic FLOPs of the chunkwise backward per token: per V head the start
-    states (U = U~ - W S and the state update, 2 dk dv each), W and U~ (2C(dk+dv)),
-    the gradient chain (K dS', Q^T dO, W^T dU: 2 dk dv each; P^T dO: 2C dv), and
-    per chunk dO S^T, dU S^T, U dS'^T (2 dk dv each), dP, T^T dU, dU V^T (2C dv
+    states (U = U~ - W S and the state update, 2 dk dv each), W and U~ (2C dk,
+    2C dv), the gradient chain (K dS', Q^T dO, W^T dU: 2 dk dv each; P^T dO: 2C dv),
+    and per chunk dO S^T, dU S^T, U dS'^T (2 dk dv each), dP, T^T dU, dU V^T (2C dv
     each), (dP o Gam) K, (dP o Gam)^T Q, T^T dW, dW K^T, M K, M^T K (2C dk each),
     T^T dT and Z T^T (2C^2 each); the grams once per QK head (4 C dk)."""
-    per_v = 16 * w.dk * w.dv + 2 * C * (8 * w.dk + 5 * w.dv) + 4 * C * C
+    per_v = 16 * w.dk * w.dv + 2 * C * (7 * w.dk + 5 * w.dv) + 4 * C * C
     return w.Hv * per_v + 4 * C * w.dk * w.Hqk
 
 
