@@ -25,7 +25,7 @@ def _pad(x, L, fill=0.0):
     return x if L == C else np.concatenate([x, np.full((C - L,) + x.shape[1:], fill)])
 
 
-def four_launches(q, k, v, al, be, dO, S0, dSf):
+def four_launches(q, k, v, al, be, dO, S0, dSf, mutation=None):
     B, T, Hqk, D = q.shape
     Hv = v.shape[2]
     grp = Hv // Hqk
@@ -43,7 +43,8 @@ def four_launches(q, k, v, al, be, dO, S0, dSf):
                 L = min(C, T - t0)
                 c = dict(L=L, t0=t0, K=_pad(k[b, t0:t0 + L, hq], L), Q=_pad(q[b, t0:t0 + L, hq], L),
                          V=_pad(v[b, t0:t0 + L, h], L), O=_pad(dO[b, t0:t0 + L, h], L),
-                         a=_pad(al[b, t0:t0 + L, h], L, 1.0), bt=_pad(be[b, t0:t0 + L, h], L))
+                         a=_pad(al[b, t0:t0 + L, h], L, 0.5 if mutation == "pad_alpha" else 1.0),
+                         bt=_pad(be[b, t0:t0 + L, h], L))
                 bb = np.cumsum(np.log(c["a"]))
                 c["Gam"] = np.where(low, np.exp(np.minimum(bb[:, None] - bb[None, :], 0.0)), 0.0)
                 c["gam"], c["g"] = np.exp(bb), np.exp(bb[-1] - bb)
@@ -68,7 +69,7 @@ def four_launches(q, k, v, al, be, dO, S0, dSf):
             for n in range(NC - 1, -1, -1):
                 c = prep[n]
                 dSp[n], gC[n] = dS, np.sum(dS * Ss[n])
-                dU = c["g"][:, None] * (c["K"] @ dS) + c["P"].T @ c["O"]
+                dU = c["g"][:, None] * (c["K"] @ dS) + (c["P"] if mutation == "P_untransposed" else c["P"].T) @ c["O"]
                 dUs[n] = dU
                 dS = c["gam"][-1] * dS + c["Q"].T @ (c["gam"][:, None] * c["O"]) - c["W"].T @ dU
             out["dS0"][b, h] = dS
@@ -77,7 +78,7 @@ def four_launches(q, k, v, al, be, dO, S0, dSf):
                 S, U, dU = Ss[n], Us[n], dUs[n]
                 K, Q, V, O, bt, gam, g, Gam, Tm = (c[x] for x in ("K", "Q", "V", "O", "bt", "gam", "g", "Gam", "Tm"))
                 X1 = O @ S.T
-                dq = gam[:, None] * X1
+                dq = (g if mutation == "g_for_gamma" else gam)[:, None] * X1
                 r_dgam = np.sum(Q * X1, 1)
                 dW = -(dU @ S.T)
                 dPG = (O @ U.T) * Gam
@@ -94,16 +95,20 @@ def four_launches(q, k, v, al, be, dO, S0, dSf):
                 dk += g[:, None] * X3
                 r_dg = np.sum(K * X3, 1)
                 dT = (bt * gam)[None, :] * (dW @ K.T) + bt[None, :] * (dU @ V.T)
+                if mutation == "dT_rows":   # the gates on the rows instead of the columns
+                    dT = (bt * gam)[:, None] * (dW @ K.T) + bt[:, None] * (dU @ V.T)
                 dA = np.tril(-((Tm.T @ dT) @ Tm.T), -1)
                 r_db3 = np.sum(dA * Gam * c["KK"], 1)
                 GGA = bt[:, None] * dA * Gam * c["KK"]
                 M = bt[:, None] * dA * Gam
-                dk += (M + M.T) @ K
+                dk += (M if mutation == "no_Mt" else M + M.T) @ K
                 dgamma = r_dgam + r_dbg * bt
                 dbeta = r_dbg * gam + r_db2 + r_db3
                 gg = r_dg * g
                 db = dgamma * gam + GGP.sum(1) + GGA.sum(1) - GGP.sum(0) - GGA.sum(0) - gg
-                db[-1] += gC[n] * gam[-1] + gg.sum()
+                if mutation == "col_sum_sign":
+                    db += 2 * (GGP.sum(0) + GGA.sum(0))
+                db[-1] += (0.0 if mutation == "drop_gC" else gC[n] * gam[-1]) + gg.sum()
                 dla = np.cumsum(db[::-1])[::-1]
                 L, t0 = c["L"], c["t0"]
                 out["dq"][b, t0:t0 + L, hq] += dq[:L]
@@ -128,3 +133,23 @@ def test_four_launch_arrangement_matches_the_oracle(T, s0, dsf):
     for name, r in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dS0"), ref):
         err = np.abs(got[name] - r).max() / max(np.abs(r).max(), 1e-300)
         assert err < 1e-10, f"{name}: {err:.2e}"
+
+
+@pytest.mark.parametrize("mutation", ["pad_alpha", "g_for_gamma", "no_Mt", "col_sum_sign", "drop_gC", "dT_rows",
+                                      "P_untransposed"])
+def test_each_planted_slip_is_caught(mutation):
+    """Each plausible slip in the arrangement (padding, a gate on the wrong side, a
+    dropped or sign-flipped term, a transposed operand) moves some gradient far past
+    rounding: the comparison above would fail."""
+    T = 77   # two chunks, the second ragged
+    d = inputs.prefill_inputs(1, T, 1, 3, dtype=torch.float32, s0_std=0.3, seed=977)
+    g = torch.Generator().manual_seed(5)
+    dO = torch.randn(1, T, 3, 128, generator=g)
+    dSf = torch.randn(1, 3, 128, 128, generator=g) * 0.1
+    f64 = lambda x: None if x is None else x.double().numpy()
+    ref = oracle.backward(d["q"], d["k"], d["v"], d["alpha"], d["beta"], dO, d["S0"], dSf)
+    got = four_launches(*(f64(x) for x in (d["q"], d["k"], d["v"], d["alpha"], d["beta"], dO, d["S0"], dSf)),
+                        mutation=mutation)
+    worst = max(np.abs(got[name] - r).max() / max(np.abs(r).max(), 1e-300)
+                for name, r in zip(("dq", "dk", "dv", "dalpha", "dbeta", "dS0"), ref))
+    assert worst > 1e-6, f"{mutation} not caught ({worst:.1e})"
