@@ -24,7 +24,7 @@
 // Four launches, all on warp-level bf16 tensor-core MMAs (m16n8k16, fp32
 // accumulation) fed by ldmatrix from padded shared-memory tiles:
 //   1. prep_kernel, per (chunk, QK head): grams, the triangular solve (fp32), and
-//      per V head W, U~, T, P and b into the workspace;
+//      per V head W, U~, T, P and the gate vectors b, gamma, g into the workspace;
 //   2. fwd_chain_kernel, per (V head, 64 value columns): the chunk start states S
 //      (bf16, kept for step 4) and U = U~ - W S (over U~ in the workspace);
 //   3. grad_chain_kernel, per (V head, 64 value columns), chunks from the end: dS'
@@ -45,7 +45,7 @@ constexpr int D = kHeadDim;          // 128
 constexpr int LDT = D + 8;           // row stride (elements) of 64 x 128 and 128 x 128 bf16 tiles
 constexpr int LDQ = C + 8;           // 64 x 64 bf16 tiles
 constexpr int LDF = C + 1;           // 64 x 64 fp32 tiles
-constexpr int kThreads = 256;        // 8 warps in every kernel
+constexpr int kThreads = 256;        // 8 warps (grad_chunk_kernel: K3W warps, below)
 constexpr float kLogFloor = -87.f;   // log alpha clamp (alpha = 0 stays finite)
 
 // Workspace, per (sequence, V head, chunk) ch = (b Hv + h) NC + n.
